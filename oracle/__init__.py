@@ -1,0 +1,311 @@
+"""CPU oracle for pooled-wave MoE dispatch/combine (ctypes wrapper over oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py``; never by the library.  It shares no code
+with the CUDA path and takes no input from it.
+
+Every function here is argument marshalling around the single-threaded C
+definitions in ``oracle.c``; the arithmetic lives there, each step citing the
+page passage it follows.  ``run()`` chains the stages in the method's order:
+route -> sender assignment -> pack -> (exchange = index relabel) -> receiver
+bucketing -> per-expert op -> combine.
+
+Parity status: every stage is pinned by the ``-m "not gpu"`` tests in
+``tests/test_oracle_*.py`` (brute force on tiny inputs, closed forms, library
+routines, invariants); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c (plain gcc, no FMA contraction, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-ffp-contract=off",
+                               "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Geom(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("T_s", ctypes.c_int64),
+                ("R", ctypes.c_int32), ("L", ctypes.c_int32), ("W", ctypes.c_int32),
+                ("P", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("pad", ctypes.c_int32),
+                ("C_s", ctypes.c_int64), ("C_r", ctypes.c_int64)]
+
+
+@dataclass
+class Geom:
+    """Batch geometry.  ``T_s`` is the number of tokens per source shard; the
+    sources present are ``T // T_s`` (all R of them for a full batch)."""
+
+    T: int
+    T_s: int
+    R: int
+    L: int
+    W: int
+    P: int
+    k: int
+    D: int
+    C_s: int
+    C_r: int
+
+    @property
+    def E(self) -> int:
+        return self.R * self.L
+
+    @property
+    def n_src(self) -> int:
+        return self.T // self.T_s
+
+    @property
+    def n_pools(self) -> int:
+        return self.n_src * self.R * self.W
+
+    @property
+    def n_slots(self) -> int:
+        return self.n_pools * self.C_s
+
+    def c(self) -> _Geom:
+        return _Geom(self.T, self.T_s, self.R, self.L, self.W, self.P, self.E, self.k,
+                     self.D, 0, self.C_s, self.C_r)
+
+
+_lib = None
+
+
+def _configure(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    gp = ctypes.POINTER(_Geom)
+    lib.orc_capacity.argtypes = [i64, i64, i32, i32, i32, i32, i32,
+                                 ctypes.POINTER(i64), ctypes.POINTER(i64)]
+    lib.orc_route.argtypes = [gp, vp, vp, vp]
+    lib.orc_assign_pooled.argtypes = [gp, vp, vp, vp, vp]
+    lib.orc_assign_pooled.restype = i64
+    lib.orc_pack.argtypes = [gp, i64, vp, vp, vp, vp, vp]
+    lib.orc_bucket.argtypes = [gp, vp, vp, vp, vp, vp, vp]
+    lib.orc_bucket.restype = i64
+    lib.orc_assign_ragged.argtypes = [gp, vp, vp, vp, vp, vp]
+    lib.orc_expert_pooled.argtypes = [gp, i64, vp, vp, vp, vp, vp, vp]
+    lib.orc_expert_ragged.argtypes = [gp, i64, vp, vp, vp, vp, vp]
+    lib.orc_combine.argtypes = [gp, vp, vp, vp, vp, vp]
+    lib.orc_combine_tokens.argtypes = [gp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp]
+    lib.orc_combine_mag.argtypes = [gp, vp, vp, vp, vp, vp]
+    lib.orc_bf16_round.argtypes = [vp, vp, i64]
+    lib.orc_expert_product.argtypes = [vp, vp, vp, i64]
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _configure(ctypes.CDLL(build()))
+    return _lib
+
+
+class variant:
+    """Context manager that routes every oracle call to another build of
+    oracle.c (the tests use it to plant mistakes and check a pin catches them)."""
+
+    def __init__(self, so_path: str):
+        self.lib = _configure(ctypes.CDLL(so_path))
+
+    def __enter__(self):
+        global _lib
+        self.saved, _lib = _load(), self.lib
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
+
+
+def _p(a: np.ndarray) -> int:
+    assert a.flags.c_contiguous, "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+def _c(a, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def capacity(T: int, T_s: int, E: int, k: int, P: int, cf_send_pct: int, cf_recv_pct: int):
+    """(C_s, C_r) as defined in oracle.c (ceil of factor x uniform-routing mean)."""
+    cs, cr = ctypes.c_int64(), ctypes.c_int64()
+    if _load().orc_capacity(T, T_s, E, k, P, cf_send_pct, cf_recv_pct,
+                            ctypes.byref(cs), ctypes.byref(cr)) != 0:
+        raise ValueError("bad capacity arguments")
+    return int(cs.value), int(cr.value)
+
+
+def geom_for(w, T: int | None = None, T_s: int | None = None) -> Geom:
+    """Geometry of workload ``w`` (a ``synth.Workload``).  ``T``/``T_s`` select a
+    sample of source shards; capacities always come from the full batch."""
+    T_full, Ts_full = w.T, w.T // w.R
+    C_s, C_r = capacity(T_full, Ts_full, w.E, w.k, w.P, w.cf_send_pct, w.cf_recv_pct)
+    return Geom(T=T_full if T is None else T, T_s=Ts_full if T_s is None else T_s,
+                R=w.R, L=w.L, W=w.W, P=w.P, k=w.k, D=w.D, C_s=C_s, C_r=C_r)
+
+
+def route(g: Geom, logits: np.ndarray):
+    lg = _c(logits, np.float32).reshape(g.T, g.E)
+    idx = np.empty((g.T, g.k), np.int32)
+    gates = np.empty((g.T, g.k), np.float64)
+    gc = g.c()
+    _load().orc_route(ctypes.byref(gc), _p(lg), _p(idx), _p(gates))
+    return idx, gates
+
+
+def assign_pooled(g: Geom, idx: np.ndarray):
+    idx = _c(idx, np.int32)
+    slot_map = np.empty((g.T, g.k), np.int32)
+    occ = np.empty((g.n_src, g.R, g.W), np.int32)
+    slot_tok = np.empty((g.n_slots,), np.int32)
+    gc = g.c()
+    dropped = _load().orc_assign_pooled(ctypes.byref(gc), _p(idx), _p(slot_map), _p(occ),
+                                        _p(slot_tok))
+    return slot_map, occ, slot_tok, int(dropped)
+
+
+def assign_ragged(g: Geom, idx: np.ndarray):
+    idx = _c(idx, np.int32)
+    slot_map = np.empty((g.T, g.k), np.int32)
+    row_off = np.empty((g.E + 1,), np.int32)
+    row_cnt = np.empty((g.E,), np.int32)
+    slot_tok = np.empty((g.T * g.k,), np.int32)
+    gc = g.c()
+    _load().orc_assign_ragged(ctypes.byref(gc), _p(idx), _p(slot_map), _p(row_off),
+                              _p(row_cnt), _p(slot_tok))
+    return slot_map, row_off, row_cnt, slot_tok
+
+
+def pack(g: Geom, n_slots: int, x: np.ndarray, idx: np.ndarray, slot_map: np.ndarray):
+    x = _c(x, np.uint16)
+    pool_x = np.empty((n_slots, g.D), np.uint16)
+    pool_hdr = np.empty((n_slots,), np.int32)
+    gc = g.c()
+    _load().orc_pack(ctypes.byref(gc), n_slots, _p(x), _p(_c(idx, np.int32)),
+                     _p(_c(slot_map, np.int32)), _p(pool_x), _p(pool_hdr))
+    return pool_x, pool_hdr
+
+
+def bucket(g: Geom, pool_hdr: np.ndarray, occ: np.ndarray):
+    recv_row = np.empty((g.n_slots,), np.int32)
+    bucket_slot = np.empty((g.E, g.C_r), np.int32)
+    arrivals = np.empty((g.E,), np.int32)
+    bucket_cnt = np.empty((g.E,), np.int32)
+    gc = g.c()
+    dropped = _load().orc_bucket(ctypes.byref(gc), _p(_c(pool_hdr, np.int32)),
+                                 _p(_c(occ, np.int32)), _p(recv_row), _p(bucket_slot),
+                                 _p(arrivals), _p(bucket_cnt))
+    return recv_row, bucket_slot, arrivals, bucket_cnt, int(dropped)
+
+
+def expert_pooled(g: Geom, pool_x, bucket_slot, bucket_cnt, scale):
+    n = pool_x.shape[0]
+    ret_x = np.empty_like(pool_x)
+    ret_hdr = np.empty((n,), np.int32)
+    gc = g.c()
+    _load().orc_expert_pooled(ctypes.byref(gc), n, _p(_c(pool_x, np.uint16)),
+                              _p(_c(bucket_slot, np.int32)), _p(_c(bucket_cnt, np.int32)),
+                              _p(_c(scale, np.float32)), _p(ret_x), _p(ret_hdr))
+    return ret_x, ret_hdr
+
+
+def expert_ragged(g: Geom, rows, row_hdr, scale):
+    n = rows.shape[0]
+    ret_x = np.empty_like(rows)
+    ret_hdr = np.empty((n,), np.int32)
+    gc = g.c()
+    _load().orc_expert_ragged(ctypes.byref(gc), n, _p(_c(rows, np.uint16)),
+                              _p(_c(row_hdr, np.int32)), _p(_c(scale, np.float32)),
+                              _p(ret_x), _p(ret_hdr))
+    return ret_x, ret_hdr
+
+
+def combine(g: Geom, ret_x, ret_hdr, slot_map, gates, with_mag: bool = False):
+    out = np.empty((g.T, g.D), np.float64)
+    gc = g.c()
+    args = (_p(_c(ret_x, np.uint16)), _p(_c(ret_hdr, np.int32)), _p(_c(slot_map, np.int32)),
+            _p(_c(gates, np.float64)))
+    _load().orc_combine(ctypes.byref(gc), *args, _p(out))
+    if not with_mag:
+        return out
+    mag = np.empty((g.T, g.D), np.float64)
+    _load().orc_combine_mag(ctypes.byref(gc), *args, _p(mag))
+    return out, mag
+
+
+def combine_tokens(g: Geom, x, idx, gates, slot_map, recv_row, scale, tokens):
+    tokens = _c(tokens, np.int64)
+    out = np.empty((tokens.size, g.D), np.float64)
+    mag = np.empty((tokens.size, g.D), np.float64)
+    gc = g.c()
+    _load().orc_combine_tokens(ctypes.byref(gc), _p(_c(x, np.uint16)), _p(_c(idx, np.int32)),
+                               _p(_c(gates, np.float64)), _p(_c(slot_map, np.int32)),
+                               _p(_c(recv_row, np.int32)), _p(_c(scale, np.float32)),
+                               _p(tokens), tokens.size, _p(out), _p(mag))
+    return out, mag
+
+
+def bf16_round(a: np.ndarray) -> np.ndarray:
+    a = _c(a, np.float32)
+    out = np.empty(a.shape, np.uint16)
+    _load().orc_bf16_round(_p(a), _p(out), a.size)
+    return out
+
+
+def expert_product(s: np.ndarray, x: np.ndarray) -> np.ndarray:
+    s, x = _c(s, np.float32), _c(x, np.uint16)
+    assert s.shape == x.shape
+    y = np.empty(x.shape, np.uint16)
+    _load().orc_expert_product(_p(s), _p(x), _p(y), x.size)
+    return y
+
+
+def run(w, logits: np.ndarray, x: np.ndarray, scale: np.ndarray, T: int | None = None,
+        with_mag: bool = False) -> dict:
+    """Whole path for workload ``w`` (optionally only its first ``T`` tokens,
+    i.e. the first T // T_s source shards).  Returns every intermediate."""
+    g = geom_for(w, T=T)
+    lg = logits[: g.T]
+    xx = x[: g.T]
+    r = {"geom": g}
+    r["idx"], r["gates"] = route(g, lg)
+    if w.mode == 0:
+        r["slot_map"], r["occ"], r["slot_tok"], r["sender_dropped"] = assign_pooled(g, r["idx"])
+        r["pool_x"], r["pool_hdr"] = pack(g, g.n_slots, xx, r["idx"], r["slot_map"])
+        (r["recv_row"], r["bucket_slot"], r["arrivals"], r["bucket_cnt"],
+         r["receiver_dropped"]) = bucket(g, r["pool_hdr"], r["occ"])
+        r["ret_x"], r["ret_hdr"] = expert_pooled(g, r["pool_x"], r["bucket_slot"],
+                                                 r["bucket_cnt"], scale)
+    else:
+        r["slot_map"], r["row_off"], r["row_cnt"], r["slot_tok"] = assign_ragged(g, r["idx"])
+        n_rows = g.T * g.k
+        r["pool_x"], r["pool_hdr"] = pack(g, n_rows, xx, r["idx"], r["slot_map"])
+        r["recv_row"] = (np.arange(n_rows, dtype=np.int64)
+                         - np.repeat(r["row_off"][:-1], r["row_cnt"])).astype(np.int32)
+        r["sender_dropped"] = r["receiver_dropped"] = 0
+        r["arrivals"] = r["bucket_cnt"] = r["row_cnt"]
+        r["ret_x"], r["ret_hdr"] = expert_ragged(g, r["pool_x"], r["pool_hdr"], scale)
+    res = combine(g, r["ret_x"], r["ret_hdr"], r["slot_map"], r["gates"], with_mag=with_mag)
+    if with_mag:
+        r["out"], r["mag"] = res
+    else:
+        r["out"] = res
+    r["kept"] = int(np.asarray(r["bucket_cnt"], np.int64).sum())
+    return r
