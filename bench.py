@@ -1,0 +1,380 @@
+"""Benchmark of the pooled-wave MoE dispatch/combine path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload rack]
+    python bench.py --impl reference ...        # the CPU oracle as the reference arm
+    torchrun --nproc-per-node N bench.py --gpus N ...
+
+One step = route -> dispatch (assign, pack, bucket) -> per-expert op ->
+combine -> drop statistics, on one synthetic batch already resident in HBM.
+The metric is routed assignments per second for dispatch + combine: T*k
+divided by the device time of route + assign + pack + bucket + combine, each
+timed with CUDA events on the launching stream inside the K timed steps (the
+per-expert op runs in every step but is timed apart, since it stands in for
+the expert network).  HBM GB/s and the fraction of the measured copy peak use
+the algorithmic bytes of those stages.
+
+Multi-GPU: every rank runs its own batch (seed = rank); the path needs no
+collective, so scaling is weak and the value is the sum over ranks of T*k
+divided by the slowest rank's time.
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed assignments/s and HBM GB/s (% of peak) for dispatch+combine; drop rate"
+UNIT = "assignments/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="rack")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
+    ap.add_argument("--cpu-sample-sources", type=int, default=16)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def alg_bytes(w, stats, C_s):
+    """Algorithmic bytes of route + dispatch + combine (what the method must
+    move; the exchange is an index relabel and moves nothing).  K_s = rows the
+    sender kept, K = rows the receiver kept."""
+    T, E, k, D = w.T, w.E, w.k, w.D
+    S = w.R * w.R * w.W * C_s if w.mode == 0 else T * k
+    K_s = T * k - stats.sender_dropped
+    K = stats.kept
+    route = 4 * T * E + 8 * T * k
+    assign = 4 * T * k + 4 * T * k                      # read idx, write slot_map
+    pack = 2 * T * D + 8 * T * k + S * (2 * D + 4)      # x rows, slot_map + idx, pool rows + headers
+    bucket = 8 * S                                      # read headers, write receiver rows
+    combine = 8 * T * k + 4 * K_s + 2 * D * K + 4 * T * D
+    return {"route": route, "assign": assign, "pack": pack, "bucket": bucket, "combine": combine,
+            "expert": 2 * D * K + 8 * S + S * (2 * D + 4)}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons during the timed region (reads only)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = [r.split(", ") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        os.unlink(self.path)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_from_profiles(kernel: str):
+    """DRAM bytes per launch for ``kernel`` from a committed ncu summary, if the
+    kernel source is unchanged since the capture (sha256 recorded there)."""
+    import hashlib
+    import re
+    prof = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
+    if not os.path.exists(prof):
+        return None
+    text = open(prof).read()
+    m_b = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
+    m_h = re.search(r"^source_sha256:\s*([0-9a-f]+)", text, re.M)
+    m_f = re.search(r"^source_file:\s*(\S+)", text, re.M)
+    if not (m_b and m_h and m_f):
+        return None
+    src = os.path.join(ROOT, m_f.group(1))
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != m_h.group(1):
+        return None
+    return float(m_b.group(1))
+
+
+def cpu_oracle_sample(w, n_src: int):
+    """Time the CPU oracle (single thread) on the first n_src source shards of
+    the batch: route, assignment, pack, bucketing, expert op and combine."""
+    import oracle
+    from combine_moe_pw_b200 import synth
+    T = n_src * (w.T // w.R) if w.mode == 0 else n_src * (w.T // w.R)
+    ws = w.with_(T=T)
+    lg, x, s = synth.logits(ws), synth.x_bf16(ws), synth.scales(w)
+    t0 = time.perf_counter()
+    if w.mode == 0:
+        oracle.run(w, lg, x, s, T=T)
+    else:
+        oracle.run(ws, lg, x, s)
+    dt = time.perf_counter() - t0
+    return T * w.k, dt
+
+
+def run_reference(a):
+    """Reference arm: the CPU oracle on the host cores, as it stands."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from combine_moe_pw_b200 import synth
+    w = synth.WORKLOADS[a.workload]
+    n_src = 1
+    for _ in range(a.warmup):
+        cpu_oracle_sample(w, n_src)
+    units, times = 0, []
+    for _ in range(a.steps):
+        u, dt = cpu_oracle_sample(w, n_src)
+        units += u
+        times.append(dt)
+    total = sum(times)
+    value = units / total
+    sample = (f"first {n_src} of {w.R} source shards ({n_src * (w.T // w.R)} tokens) of the "
+              f"{w.name} batch per step; whole oracle path (route..combine), one thread")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
+            "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": 1e3 * total / a.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    return {"workload": w.name, "tokens": w.T, "experts": w.E, "top_k": w.k, "width": w.D,
+            "ranks": w.R, "experts_per_rank": w.L, "waves": w.W,
+            "cf_send": w.cf_send_pct / 100 if w.cf_send_pct > 0 else None,
+            "cf_recv": w.cf_recv_pct / 100 if w.cf_recv_pct > 0 else None,
+            "mode": "pooled" if w.mode == 0 else "ragged",
+            "sequences": w.T // w.seq_len, "seq_len": w.seq_len,
+            "l2": "inputs larger than L2 (no flush)",
+            "metric_scope": "route + assign + pack + bucket + combine; expert op timed apart"}
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from combine_moe_pw_b200 import moe_pw as mp
+    from combine_moe_pw_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+
+    base = synth.WORKLOADS[a.workload]
+    w = base.with_(seed=base.seed + rank)
+    cfg = mp.Config.from_workload(w)
+    b = mp.Buffers(cfg, device=dev)
+    sizes = b.sizes
+    lg = synth.logits(w)
+    x = synth.x_bf16(w)
+    s = synth.scales(w)
+    b.logits.copy_(torch.from_numpy(lg))
+    b.x.copy_(torch.from_numpy(x.view(np.int16)))
+    b.scale.copy_(torch.from_numpy(s))
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    stages = ["route", "assign", "pack", "bucket", "expert", "combine"]
+
+    def step(evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record(stream)
+        mark(0)
+        b.route(stream)
+        mark(1)
+        b.assign(stream)
+        mark(2)
+        b.pack(stream)
+        mark(3)
+        b.bucket(stream)
+        mark(4)
+        b.expert(stream)
+        mark(5)
+        b.combine(stream)
+        mark(6)
+        return b.stats(stream)
+
+    for _ in range(max(a.warmup, 3)):
+        st = step()
+    launches_per_step = 8 if w.mode == 0 else 9
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(a.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for i in range(a.steps):
+        st = step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+
+    total_ms = start.elapsed_time(end)
+    per_stage = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(a.steps)]
+                 for j, n in enumerate(stages)}
+    dc_stages = ["route", "assign", "pack", "bucket", "combine"]
+    dc_ms = sum(sum(per_stage[n]) for n in dc_stages)  # over K steps
+    vals = torch.tensor([total_ms, dc_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, dc_ms = float(vals[0]), float(vals[1])
+
+    units = w.T * w.k * a.steps * world
+    value = units / (dc_ms / 1e3)
+    ab = alg_bytes(w, st, sizes.C_s)
+    b_alg = sum(ab[n] for n in dc_stages)
+    peak, peak_kind = measured_peaks()
+    gbs = b_alg * a.steps / (dc_ms / 1e3) / 1e9
+    stage_ms = {n: statistics.mean(v) for n, v in per_stage.items()}
+    dom = max(["pack", "combine"], key=lambda n: stage_ms[n])
+    kname = {"pack": "pack_kernel", "combine": "combine_kernel"}[dom]
+    achieved = ab[dom] / (stage_ms[dom] / 1e3) / 1e9
+    traffic = traffic_from_profiles(kname + "_" + a.workload)
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    e2e = None
+    if not a.no_e2e:
+        ke = a.e2e_steps or a.steps
+        h_lg = torch.from_numpy(lg).pin_memory()
+        h_x = torch.from_numpy(x.view(np.int16)).pin_memory()
+        h_s = torch.from_numpy(s).pin_memory()
+        h_out = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
+        h2d = h_lg.numel() * 4 + h_x.numel() * 2 + h_s.numel() * 4
+        d2h = h_out.numel() * 4 + mp.COUNTERS_BYTES
+
+        def e2e_step():
+            b.logits.copy_(h_lg, non_blocking=True)
+            b.x.copy_(h_x, non_blocking=True)
+            b.scale.copy_(h_s, non_blocking=True)
+            b.run_step(stream)
+            h_out.copy_(b.out, non_blocking=True)
+            return b.stats(stream)  # synchronises: the step's result is on the host
+
+        for _ in range(2):
+            e2e_step()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ev = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(ev, op=dist.ReduceOp.MAX)
+        e2e = {"value": w.T * w.k * ke * world / (float(ev[0]) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": float(ev[0]) / ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        u, dt = cpu_oracle_sample(base, a.cpu_sample_sources)
+        cpu = {"value": u / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"first {a.cpu_sample_sources} of {base.R} source shards "
+                         f"({a.cpu_sample_sources * (base.T // base.R)} tokens) of the {base.name} "
+                         f"batch, whole oracle path (route..combine), one thread, {dt:.1f} s"}
+
+    if rank == 0:
+        TK = w.T * w.k
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": a.steps, "warmup": max(a.warmup, 3),
+            "ms_per_step": total_ms / a.steps,
+            "ms_dispatch_combine_per_step": dc_ms / a.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "payload_dtype": "bf16", "data": "synthetic",
+            "config": config_of(w),
+            "hbm_gbs": gbs, "hbm_frac_of_peak": gbs / peak, "hbm_peak_gbs": peak,
+            "hbm_peak_kind": peak_kind,
+            "alg_bytes_per_step": b_alg,
+            "drop_rate": {"sender": st.sender_dropped / TK, "receiver": st.receiver_dropped / TK,
+                          "total": (st.sender_dropped + st.receiver_dropped) / TK},
+            "stage_ms": stage_ms,
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                         "alg_bytes_per_launch": ab[dom], "peak_kind": peak_kind},
+            "gpu_launches": launches_per_step * a.steps,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

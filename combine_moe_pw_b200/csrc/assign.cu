@@ -1,0 +1,310 @@
+// assign.cu - sender slot assignment (pooled) / expert row assignment (ragged).
+//
+// "Marin 开始公开训练 535B 参数 MoE 模型", section 二: one fixed pool per
+// (source, destination) and wave; the 1.10 sender factor caps each pool and
+// the overflow is dropped.  Section 四: the dropless ragged alternative.
+//
+// Both modes rank every assignment (t, j) among the earlier assignments of
+// its group that fall in the same bin, in flat (t, j) order:
+//   pooled: group = source shard s, bin = pool (d, w) = (e / L) * W + (e % L) / P,
+//           slot = (s * R*W + bin) * C_s + rank, kept iff rank < C_s;
+//   ragged: one group, bin = expert e, row = offset[e] + rank.
+// Work is split into chunks of consecutive tokens inside a group and done in
+// three deterministic passes (no order-giving atomics):
+//   1. count : per chunk, per-warp histograms in shared memory, summed per bin;
+//   2. scan  : per (group, bin), exclusive prefix over the group's chunks;
+//   3. rank  : per chunk, recount, per-warp bases = chunk base + earlier warps,
+//              then each warp walks its assignments 32 at a time: lanes with
+//              the same bin find each other with match.any and take ranks in
+//              lane order.
+// Ragged mode adds a one-block scan of the per-expert totals into offsets.
+#include "common.cuh"
+
+namespace moe_pw {
+
+namespace {
+
+constexpr int AW = 8;  // warps per block in count/rank
+
+struct RankArgs {
+    const int32_t *idx;
+    int32_t *slot_map;
+    int32_t *occ;
+    int32_t *counts;   // [n_chunks][NB], becomes the chunk bases after the scan
+    int32_t *totals;   // [n_groups][NB]
+    moe_pw_counters *ctr;
+    Geo g;
+};
+
+__device__ __forceinline__ int32_t bin_of_expert(const Geo &g, int32_t e)
+{
+    return g.mode == MOE_PW_POOLED ? (e / g.L) * g.W + (e % g.L) / g.P : e;
+}
+
+// Flat assignment range [a0, a1) of this block's chunk and its group.
+__device__ __forceinline__ void chunk_range(const Geo &g, int chunk, int64_t &a0, int64_t &a1,
+                                            int &group)
+{
+    group = chunk / g.chunks_per_group;
+    const int c = chunk - group * g.chunks_per_group;
+    const int64_t g0 = int64_t(group) * g.group_tokens;
+    const int64_t t0 = g0 + int64_t(c) * g.chunk_tokens;
+    int64_t t1 = t0 + g.chunk_tokens;
+    if (t1 > g0 + g.group_tokens) t1 = g0 + g.group_tokens;
+    a0 = t0 * g.k;
+    a1 = t1 * g.k;
+}
+
+// Shared-memory layout shared by count and rank.
+struct Smem {
+    int32_t *bin_tab;  // [E]
+    int32_t *hist;     // [AW][NB]
+    int32_t *off;      // [E + 1] (ragged rank pass)
+};
+
+__device__ __forceinline__ Smem carve(const Geo &g, int32_t *sm)
+{
+    Smem s;
+    s.bin_tab = sm;
+    s.hist = sm + g.E;
+    s.off = s.hist + AW * g.NB;
+    return s;
+}
+
+// Per-warp histogram of this warp's slice of the chunk.
+__device__ __forceinline__ void warp_hist(const RankArgs &p, const Smem &s, int64_t wa0,
+                                          int64_t wa1, int warp, int lane)
+{
+    int32_t *h = s.hist + warp * p.g.NB;
+    for (int64_t a = wa0; a < wa1; a += 32) {
+        const int64_t ai = a + lane;
+        int32_t b = -1;
+        if (ai < wa1) {
+            const int32_t e = p.idx[ai];
+            if (e >= 0 && e < p.g.E) b = s.bin_tab[e];
+        }
+        const unsigned same = __match_any_sync(FULL_MASK, b);
+        if (b >= 0 && lane == __ffs(same) - 1) h[b] += __popc(same);
+        __syncwarp();
+    }
+}
+
+__device__ __forceinline__ void setup(const RankArgs &p, const Smem &s)
+{
+    for (int e = threadIdx.x; e < p.g.E; e += blockDim.x) s.bin_tab[e] = bin_of_expert(p.g, e);
+    for (int i = threadIdx.x; i < AW * p.g.NB; i += blockDim.x) s.hist[i] = 0;
+}
+
+__global__ void __launch_bounds__(AW * 32) assign_count(RankArgs p)
+{
+    extern __shared__ int32_t sm[];
+    const Smem s = carve(p.g, sm);
+    setup(p, s);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int64_t a0, a1;
+    int group;
+    chunk_range(p.g, blockIdx.x, a0, a1, group);
+    const int64_t n = a1 - a0;
+    warp_hist(p, s, a0 + n * warp / AW, a0 + n * (warp + 1) / AW, warp, lane);
+    __syncthreads();
+    int32_t *out = p.counts + int64_t(blockIdx.x) * p.g.NB;
+    for (int b = threadIdx.x; b < p.g.NB; b += blockDim.x) {
+        int32_t sum = 0;
+        for (int w = 0; w < AW; ++w) sum += s.hist[w * p.g.NB + b];
+        out[b] = sum;
+    }
+}
+
+// Block (32 warps) per (group, 32-bin tile): exclusive scan over the group's
+// chunks, in place; totals, occupancy and sender drops.
+__global__ void __launch_bounds__(1024) assign_scan(RankArgs p)
+{
+    __shared__ int32_t part[32][33];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int group = blockIdx.y;
+    const int b = blockIdx.x * 32 + lane;
+    const int cpg = p.g.chunks_per_group;
+    const int c0 = cpg * warp / 32, c1 = cpg * (warp + 1) / 32;
+    int32_t *col = p.counts + int64_t(group) * cpg * p.g.NB + b;
+    int32_t sum = 0;
+    if (b < p.g.NB)
+        for (int c = c0; c < c1; ++c) sum += col[int64_t(c) * p.g.NB];
+    part[warp][lane] = sum;
+    __syncthreads();
+    if (warp == 0) {
+        int32_t run = 0;
+        for (int w = 0; w < 32; ++w) {
+            const int32_t v = part[w][lane];
+            part[w][lane] = run;
+            run += v;
+        }
+        if (b < p.g.NB) {
+            p.totals[int64_t(group) * p.g.NB + b] = run;
+            if (p.g.mode == MOE_PW_POOLED) {
+                const int64_t kept = run < p.g.C_s ? run : p.g.C_s;
+                p.occ[int64_t(group) * p.g.NB + b] = int32_t(kept);
+                if (run > kept) atomicAdd(&p.ctr->sender_dropped, (unsigned long long)(run - kept));
+                atomicMax(&p.ctr->max_occ, int32_t(kept));
+            }
+        }
+    }
+    __syncthreads();
+    if (b < p.g.NB) {
+        int32_t run = part[warp][lane];
+        for (int c = c0; c < c1; ++c) {
+            const int32_t v = col[int64_t(c) * p.g.NB];
+            col[int64_t(c) * p.g.NB] = run;
+            run += v;
+        }
+    }
+}
+
+// Ragged: occ[0..E] = exclusive scan of the per-expert totals (one block).
+__global__ void __launch_bounds__(1024) ragged_offsets(RankArgs p)
+{
+    __shared__ int32_t wsum[32];
+    const int E = p.g.E;
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int e0 = threadIdx.x * per;
+    int32_t local = 0;
+    for (int e = e0; e < e0 + per && e < E; ++e) local += p.totals[e];
+    // block exclusive scan of `local`
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int32_t incl = local;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t v = __shfl_up_sync(FULL_MASK, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = blockDim.x >> 5;
+        int32_t v = lane < nw ? wsum[lane] : 0;
+        int32_t inc = v;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t u = __shfl_up_sync(FULL_MASK, inc, o);
+            if (lane >= o) inc += u;
+        }
+        if (lane < nw) wsum[lane] = inc - v;
+    }
+    __syncthreads();
+    int32_t run = wsum[warp] + incl - local;
+    for (int e = e0; e < e0 + per && e < E; ++e) {
+        p.occ[e] = run;
+        run += p.totals[e];
+    }
+    if (threadIdx.x == blockDim.x - 1) p.occ[E] = run;
+}
+
+__global__ void __launch_bounds__(AW * 32) assign_rank(RankArgs p)
+{
+    extern __shared__ int32_t sm[];
+    const Smem s = carve(p.g, sm);
+    setup(p, s);
+    const bool ragged = p.g.mode == MOE_PW_RAGGED;
+    if (ragged)
+        for (int e = threadIdx.x; e <= p.g.E; e += blockDim.x) s.off[e] = p.occ[e];
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int64_t a0, a1;
+    int group;
+    chunk_range(p.g, blockIdx.x, a0, a1, group);
+    const int64_t n = a1 - a0;
+    const int64_t wa0 = a0 + n * warp / AW, wa1 = a0 + n * (warp + 1) / AW;
+    warp_hist(p, s, wa0, wa1, warp, lane);
+    __syncthreads();
+    // turn per-warp counts into per-warp starting ranks
+    const int32_t *base = p.counts + int64_t(blockIdx.x) * p.g.NB;
+    for (int b = threadIdx.x; b < p.g.NB; b += blockDim.x) {
+        int32_t run = base[b];
+        for (int w = 0; w < AW; ++w) {
+            const int32_t v = s.hist[w * p.g.NB + b];
+            s.hist[w * p.g.NB + b] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    int32_t *h = s.hist + warp * p.g.NB;
+    const int64_t pool_base = int64_t(group) * p.g.NB;
+    for (int64_t a = wa0; a < wa1; a += 32) {
+        const int64_t ai = a + lane;
+        int32_t b = -1;
+        if (ai < wa1) {
+            const int32_t e = p.idx[ai];
+            if (e >= 0 && e < p.g.E)
+                b = s.bin_tab[e];
+            else
+                set_error(p.ctr, MOE_PW_DEVERR_EXPERT_ID);
+        }
+        const unsigned same = __match_any_sync(FULL_MASK, b);
+        const int32_t r = (b >= 0 ? h[b] : 0) + __popc(same & lanemask_lt());
+        __syncwarp();
+        if (b >= 0 && lane == __ffs(same) - 1) h[b] += __popc(same);
+        __syncwarp();
+        if (ai < wa1) {
+            int32_t slot = -1;
+            if (b >= 0) {
+                if (ragged)
+                    slot = s.off[b] + r;
+                else if (r < p.g.C_s)
+                    slot = int32_t((pool_base + b) * p.g.C_s + r);
+            }
+            p.slot_map[ai] = slot;
+        }
+    }
+}
+
+size_t rank_smem_bytes(const Geo &g)
+{
+    return sizeof(int32_t) * (size_t(g.E) + size_t(AW) * g.NB + size_t(g.E) + 1);
+}
+
+}  // namespace
+
+cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, int32_t *occ,
+                          moe_pw_counters *ctr, void *ws, cudaStream_t st)
+{
+    cudaError_t err = cudaMemsetAsync(ctr, 0, sizeof(moe_pw_counters), st);
+    if (err != cudaSuccess) return err;
+    const int64_t occ_len = g.mode == MOE_PW_POOLED ? g.n_pools : int64_t(g.E) + 1;
+    if (g.T == 0) return cudaMemsetAsync(occ, 0, sizeof(int32_t) * occ_len, st);
+
+    RankArgs p;
+    p.idx = idx;
+    p.slot_map = slot_map;
+    p.occ = occ;
+    p.counts = static_cast<int32_t *>(ws);
+    p.totals = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + ws_counts_bytes(g));
+    p.ctr = ctr;
+    p.g = g;
+
+    const size_t smem = rank_smem_bytes(g);
+    static bool attr_done[64] = {};
+    int dev = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if (smem > 48 * 1024 && dev < 64 && !attr_done[dev]) {
+        DevInfo di;
+        if (dev_info(&di) != 0) return cudaErrorUnknown;
+        if ((err = cudaFuncSetAttribute(assign_count, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        di.smem_optin)) != cudaSuccess)
+            return err;
+        if ((err = cudaFuncSetAttribute(assign_rank, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        di.smem_optin)) != cudaSuccess)
+            return err;
+        attr_done[dev] = true;
+    }
+    assign_count<<<g.n_chunks, AW * 32, smem, st>>>(p);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    dim3 sgrid((g.NB + 31) / 32, g.n_groups);
+    assign_scan<<<sgrid, 1024, 0, st>>>(p);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (g.mode == MOE_PW_RAGGED) {
+        ragged_offsets<<<1, 1024, 0, st>>>(p);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    assign_rank<<<g.n_chunks, AW * 32, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace moe_pw

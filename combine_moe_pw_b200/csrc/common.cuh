@@ -1,0 +1,181 @@
+// common.cuh - internal declarations and device helpers of libmoe_pw.so.
+// Not part of the public ABI (include/moe_pw.h is).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "moe_pw.h"
+
+namespace moe_pw {
+
+constexpr unsigned FULL_MASK = 0xFFFFFFFFu;
+
+// Everything a kernel needs to know about the batch, derived on the host
+// from a validated moe_pw_config.
+struct Geo {
+    int64_t T;        // tokens
+    int32_t E, k, D, R, L, W, P;
+    int32_t mode;     // MOE_PW_POOLED / MOE_PW_RAGGED
+    int64_t T_s;      // tokens per source shard (pooled), T (ragged)
+    int64_t C_s, C_r; // capacities (pooled)
+    int64_t n_pools;  // R*R*W (pooled), 0 (ragged)
+    int64_t n_slots;  // pool rows
+    // ranking (assign) decomposition
+    int32_t NB;       // bins: pools per source (R*W) or experts (E)
+    int32_t n_groups; // sources (R) or 1
+    int64_t group_tokens;   // tokens per group
+    int64_t chunk_tokens;   // tokens per chunk
+    int32_t chunks_per_group;
+    int32_t n_chunks;
+};
+
+// Per-device attributes, cached on first use.
+struct DevInfo {
+    int sms;
+    int smem_optin;  // max dynamic shared memory per block (opt-in)
+};
+int dev_info(DevInfo *out);
+
+// Kernel launchers (asynchronous; return cudaError_t of the launch).
+cudaError_t launch_route(const Geo &g, const float *logits, int32_t *idx, float *gates,
+                         cudaStream_t st);
+cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, int32_t *occ,
+                          moe_pw_counters *ctr, void *ws, cudaStream_t st);
+cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
+                        const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
+                        int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st);
+cudaError_t launch_bucket(const Geo &g, const int32_t *pool_hdr, const int32_t *occ,
+                          int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,
+                          moe_pw_counters *ctr, cudaStream_t st);
+cudaError_t launch_expert(const Geo &g, const uint16_t *pool_x, const int32_t *pool_hdr,
+                          const int32_t *recv_row, const float *scale, uint16_t *ret_x,
+                          int32_t *ret_hdr, cudaStream_t st);
+cudaError_t launch_combine(const Geo &g, const uint16_t *ret_x, const int32_t *ret_hdr,
+                           const int32_t *slot_map, const float *gates, float *out,
+                           moe_pw_counters *ctr, cudaStream_t st);
+
+// Workspace layout of the ranking pass.
+inline int64_t align256(int64_t b) { return (b + 255) & ~int64_t(255); }
+inline int64_t ws_counts_bytes(const Geo &g) { return align256(4 * int64_t(g.n_chunks) * g.NB); }
+inline int64_t ws_totals_bytes(const Geo &g) { return align256(4 * int64_t(g.n_groups) * g.NB); }
+inline int64_t ws_bytes(const Geo &g) { return ws_counts_bytes(g) + ws_totals_bytes(g); }
+
+// ---------------------------------------------------------------------------
+// Device helpers: mbarrier and bulk (TMA) copies, inline PTX for sm_100a.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+// Make barrier initialisation and generic-proxy shared-memory writes visible
+// to the async proxy (TMA) before any bulk copy uses them.
+__device__ __forceinline__ void fence_init_and_proxy()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait on a barrier phase: gives up after `limit` polls (each poll
+// may itself suspend for a hardware time slice).  Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint32_t limit)
+{
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// Global -> shared bulk copy, completion counted on `bar` (bytes % 16 == 0,
+// both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32_t bytes,
+                                         uint64_t *bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst_smem)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// Shared -> global bulk copy in the calling thread's current bulk group.
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src_smem, uint32_t bytes,
+                                         uint64_t policy)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst),
+                 "r"(smem_addr(src_smem)), "r"(bytes), "l"(policy)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit()
+{
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until all of this thread's bulk groups have completed (writes performed).
+__device__ __forceinline__ void bulk_wait_all()
+{
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// L2 eviction policies for the bulk copies.
+__device__ __forceinline__ uint64_t policy_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void set_error(moe_pw_counters *ctr, int bits)
+{
+    atomicOr(&ctr->error, bits);
+}
+
+__device__ __forceinline__ unsigned lanemask_lt()
+{
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+}  // namespace moe_pw

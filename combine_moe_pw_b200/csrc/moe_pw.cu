@@ -1,0 +1,286 @@
+// moe_pw.cu - the C ABI of libmoe_pw.so: argument checks, sizes, launches.
+// The kernels live in route.cu, assign.cu, pack.cu, bucket.cu, expert.cu and
+// combine.cu; this file owns validation and the contract of include/moe_pw.h.
+#include <cstring>
+
+#include "common.cuh"
+
+namespace moe_pw {
+
+int dev_info(DevInfo *out)
+{
+    static DevInfo cache[64];
+    static bool have[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (dev >= 0 && dev < 64 && have[dev]) {
+        *out = cache[dev];
+        return 0;
+    }
+    DevInfo di;
+    if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return -1;
+    if (cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+        cudaSuccess)
+        return -1;
+    if (dev >= 0 && dev < 64) {
+        cache[dev] = di;
+        have[dev] = true;
+    }
+    *out = di;
+    return 0;
+}
+
+namespace {
+
+constexpr int64_t MAX_INT32 = 0x7FFFFFFF;
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Validate a config and derive the kernel geometry.
+int make_geo(const moe_pw_config *c, Geo *g)
+{
+    if (!c || !g) return MOE_PW_EINVAL;
+    if (c->T < 0 || c->R < 1 || c->L < 1 || c->W < 1 || c->P < 1 || c->k < 1 || c->D < 1)
+        return MOE_PW_EINVAL;
+    if (c->mode != MOE_PW_POOLED && c->mode != MOE_PW_RAGGED) return MOE_PW_EINVAL;
+    if (int64_t(c->W) * c->P != c->L) return MOE_PW_EINVAL;
+    if (int64_t(c->R) * c->L != c->E) return MOE_PW_EINVAL;
+    if (c->k > c->E) return MOE_PW_EINVAL;
+    if (c->T % c->R != 0) return MOE_PW_EINVAL;
+    if (c->k > 32 || c->E > 2048 || c->P > 32 || int64_t(c->R) * c->W > 2048)
+        return MOE_PW_EUNSUPPORTED;
+    if (c->D % 8 != 0 || c->D < 8 || c->D > 12288) return MOE_PW_EUNSUPPORTED;
+    if (c->T * c->k > MAX_INT32) return MOE_PW_EUNSUPPORTED;
+
+    std::memset(g, 0, sizeof(*g));
+    g->T = c->T;
+    g->E = c->E;
+    g->k = c->k;
+    g->D = c->D;
+    g->R = c->R;
+    g->L = c->L;
+    g->W = c->W;
+    g->P = c->P;
+    g->mode = c->mode;
+    const int64_t T_s = c->T / c->R;
+    if (c->mode == MOE_PW_POOLED) {
+        g->T_s = T_s;
+        const int64_t kp = c->k < c->P ? c->k : c->P;
+        g->C_s = c->cf_send_pct > 0
+                     ? ceil_div(int64_t(c->cf_send_pct) * T_s * c->k * c->P, int64_t(100) * c->E)
+                     : T_s * kp;
+        g->C_r = c->cf_recv_pct > 0
+                     ? ceil_div(int64_t(c->cf_recv_pct) * c->T * c->k, int64_t(100) * c->E)
+                     : c->T;
+        g->n_pools = int64_t(c->R) * c->R * c->W;
+        if (g->C_s > MAX_INT32 || g->C_r > MAX_INT32) return MOE_PW_EUNSUPPORTED;
+        g->n_slots = g->n_pools * g->C_s;
+        if (g->n_slots > MAX_INT32 || int64_t(c->E) * g->C_r > (int64_t(1) << 40))
+            return MOE_PW_EUNSUPPORTED;
+        g->NB = c->R * c->W;
+        g->n_groups = c->R;
+        g->group_tokens = T_s;
+    } else {
+        g->T_s = c->T;
+        g->n_pools = 0;
+        g->n_slots = c->T * c->k;
+        g->NB = c->E;
+        g->n_groups = 1;
+        g->group_tokens = c->T;
+    }
+    // ranking chunks: 256 tokens, never straddling a group
+    int64_t ct = 256;
+    if (g->group_tokens < ct) ct = g->group_tokens > 0 ? g->group_tokens : 1;
+    g->chunk_tokens = ct;
+    g->chunks_per_group = int32_t(ceil_div(g->group_tokens > 0 ? g->group_tokens : 1, ct));
+    const int64_t nch = int64_t(g->n_groups) * g->chunks_per_group;
+    if (nch > MAX_INT32) return MOE_PW_EUNSUPPORTED;
+    g->n_chunks = int32_t(nch);
+    return MOE_PW_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_PW_OK : MOE_PW_ECUDA; }
+
+}  // namespace
+}  // namespace moe_pw
+
+using namespace moe_pw;
+
+extern "C" {
+
+int moe_pw_version(void) { return 10000; }
+
+const char *moe_pw_strerror(int code)
+{
+    switch (code) {
+    case MOE_PW_OK: return "ok";
+    case MOE_PW_EINVAL: return "invalid argument or config";
+    case MOE_PW_EUNSUPPORTED: return "shape or alignment not supported by this build";
+    case MOE_PW_ECUDA: return "CUDA runtime or launch error";
+    case MOE_PW_EDEVICE: return "a kernel flagged a violation (see counters.error)";
+    case MOE_PW_ENOMEM: return "buffers exceed the memory budget";
+    default: return "unknown error code";
+    }
+}
+
+int moe_pw_plan(const moe_pw_config *cfg, int64_t budget_bytes, moe_pw_sizes *out)
+{
+    if (!out) return MOE_PW_EINVAL;
+    Geo g;
+    const int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    std::memset(out, 0, sizeof(*out));
+    const int64_t T = g.T, E = g.E, k = g.k, D = g.D;
+    out->C_s = g.mode == MOE_PW_POOLED ? g.C_s : 0;
+    out->C_r = g.mode == MOE_PW_POOLED ? g.C_r : 0;
+    out->n_pools = g.n_pools;
+    out->n_slots = g.n_slots;
+    out->occ_len = g.mode == MOE_PW_POOLED ? g.n_pools : E + 1;
+    out->bucket_len = g.mode == MOE_PW_POOLED ? E * g.C_r : 0;
+    out->workspace_bytes = ws_bytes(g);
+    const int64_t S = g.n_slots;
+    out->total_bytes = 4 * T * E          // logits
+                       + 8 * T * k        // idx, gates
+                       + 2 * T * D        // x
+                       + 4 * T * k        // slot_map
+                       + 4 * out->occ_len //
+                       + 2 * (2 * S * D)  // pool_x, ret_x
+                       + 3 * (4 * S)      // pool_hdr, recv_row, ret_hdr
+                       + 4 * out->bucket_len + 8 * E + 4 * E  // buckets, expert_counts, scale
+                       + 4 * T * D        // out
+                       + int64_t(sizeof(moe_pw_counters)) + out->workspace_bytes;
+    if (budget_bytes > 0 && out->total_bytes > budget_bytes) return MOE_PW_ENOMEM;
+    return MOE_PW_OK;
+}
+
+int moe_pw_route(const moe_pw_config *cfg, const float *logits, int32_t *idx, float *gates,
+                 cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.E % 4 != 0) return MOE_PW_EUNSUPPORTED;
+    if (g.T == 0) return MOE_PW_OK;
+    if (!logits || !idx || !gates) return MOE_PW_EINVAL;
+    if (!aligned(logits, 16) || !aligned(idx, 4) || !aligned(gates, 4)) return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_route(g, logits, idx, gates, stream));
+}
+
+int moe_pw_assign(const moe_pw_config *cfg, const int32_t *idx, int32_t *slot_map, int32_t *occ,
+                  moe_pw_counters *counters, void *workspace, size_t workspace_bytes,
+                  cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!counters || !occ) return MOE_PW_EINVAL;
+    if (g.T > 0 && (!idx || !slot_map || !workspace)) return MOE_PW_EINVAL;
+    if (g.T > 0 && int64_t(workspace_bytes) < ws_bytes(g)) return MOE_PW_EINVAL;
+    if (!aligned(counters, 8) || !aligned(occ, 4) || (g.T > 0 && (!aligned(idx, 4) ||
+        !aligned(slot_map, 4) || !aligned(workspace, 256))))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_assign(g, idx, slot_map, occ, counters, workspace, stream));
+}
+
+int moe_pw_pack(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
+                const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr,
+                moe_pw_counters *counters, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.n_slots == 0) return MOE_PW_OK;
+    if (!x || !idx || !slot_map || !occ || !pool_x || !pool_hdr || !counters) return MOE_PW_EINVAL;
+    if (!aligned(x, 16) || !aligned(pool_x, 16) || !aligned(idx, 4) || !aligned(slot_map, 4) ||
+        !aligned(occ, 4) || !aligned(pool_hdr, 4) || !aligned(counters, 8))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_pack(g, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream));
+}
+
+int moe_pw_bucket(const moe_pw_config *cfg, const int32_t *pool_hdr, const int32_t *occ,
+                  int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,
+                  moe_pw_counters *counters, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!counters || !expert_counts) return MOE_PW_EINVAL;
+    if (g.T > 0) {
+        if (!pool_hdr || !occ || !recv_row) return MOE_PW_EINVAL;
+        if (g.mode == MOE_PW_POOLED && !bucket_slot) return MOE_PW_EINVAL;
+    }
+    if (!aligned(counters, 8) || !aligned(expert_counts, 4)) return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_bucket(g, pool_hdr, occ, recv_row, bucket_slot, expert_counts, counters,
+                                 stream));
+}
+
+int moe_pw_dispatch(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
+                    int32_t *slot_map, int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr,
+                    int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,
+                    moe_pw_counters *counters, void *workspace, size_t workspace_bytes,
+                    cudaStream_t stream)
+{
+    int rc = moe_pw_assign(cfg, idx, slot_map, occ, counters, workspace, workspace_bytes, stream);
+    if (rc != MOE_PW_OK) return rc;
+    rc = moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream);
+    if (rc != MOE_PW_OK) return rc;
+    return moe_pw_bucket(cfg, pool_hdr, occ, recv_row, bucket_slot, expert_counts, counters,
+                         stream);
+}
+
+int moe_pw_expert(const moe_pw_config *cfg, const uint16_t *pool_x, const int32_t *pool_hdr,
+                  const int32_t *recv_row, const float *scale, uint16_t *ret_x, int32_t *ret_hdr,
+                  cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.n_slots == 0) return MOE_PW_OK;
+    if (!pool_x || !pool_hdr || !recv_row || !scale || !ret_x || !ret_hdr) return MOE_PW_EINVAL;
+    if (!aligned(pool_x, 16) || !aligned(ret_x, 16) || !aligned(pool_hdr, 4) ||
+        !aligned(recv_row, 4) || !aligned(scale, 4) || !aligned(ret_hdr, 4))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_expert(g, pool_x, pool_hdr, recv_row, scale, ret_x, ret_hdr, stream));
+}
+
+int moe_pw_combine(const moe_pw_config *cfg, const uint16_t *ret_x, const int32_t *ret_hdr,
+                   const int32_t *slot_map, const float *gates, float *out,
+                   moe_pw_counters *counters, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.T == 0) return MOE_PW_OK;
+    if (!ret_x || !ret_hdr || !slot_map || !gates || !out || !counters) return MOE_PW_EINVAL;
+    if (!aligned(ret_x, 16) || !aligned(out, 16) || !aligned(ret_hdr, 4) ||
+        !aligned(slot_map, 4) || !aligned(gates, 4) || !aligned(counters, 8))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_combine(g, ret_x, ret_hdr, slot_map, gates, out, counters, stream));
+}
+
+int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
+                 moe_pw_drop_stats *host_out, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!counters || !host_out) return MOE_PW_EINVAL;
+    moe_pw_counters c;
+    if (cudaMemcpyAsync(&c, counters, sizeof(c), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return MOE_PW_ECUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_PW_ECUDA;
+    host_out->assignments = g.T * g.k;
+    host_out->kept = int64_t(c.kept);
+    host_out->sender_dropped = int64_t(c.sender_dropped);
+    host_out->receiver_dropped = int64_t(c.receiver_dropped);
+    host_out->max_occ = c.max_occ;
+    host_out->max_fill = c.max_fill;
+    host_out->error = c.error;
+    host_out->reserved = 0;
+    return c.error != 0 ? MOE_PW_EDEVICE : MOE_PW_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,197 @@
+// pack.cu - copy each kept row into its pool slot(s) with TMA bulk copies.
+//
+// "Marin 开始公开训练 535B 参数 MoE 模型", section 二: the sender fills fixed
+// per-destination pools and the expert id travels with the row, so the
+// receiver needs no separate counts.  Empty slots get a zero row and header -1
+// (this library's reading), which makes the pools deterministic byte for byte.
+//
+// Design (HBM-bound permutation, no tensor cores):
+//   - persistent grid, up to MAX_PACK_WARPS independent pipelines per block
+//     (fewer for very wide rows, so every pipeline keeps >= LAG + 2 stages);
+//   - a warp owns a contiguous token range; for token t one lane issues a
+//     single cp.async.bulk load of the whole row x[t] (2*D bytes) into a
+//     shared-memory stage, tracked by an mbarrier;
+//   - when the row has landed, lane j (< k) issues the bulk store of that
+//     stage into slot slot_map[t][j] and writes the slot header: one HBM read
+//     of x[t] feeds up to k HBM writes, with no register traffic;
+//   - a stage is refilled once the stores reading it are done
+//     (cp.async.bulk.wait_group.read), LAG tokens later, so NS - LAG - 1 row
+//     loads and about LAG tokens of stores stay in flight per warp;
+//   - afterwards every warp zero-fills the empty tails (positions >= occ) of
+//     its share of the pools from a zeroed shared-memory row.
+// x is read once (evict_first); pool rows are written once (evict_first).
+#include "common.cuh"
+
+namespace moe_pw {
+
+namespace {
+
+constexpr int MAX_PACK_WARPS = 4;
+constexpr int LAG = 2;                    // store groups left in flight before a refill
+constexpr uint32_t WAIT_LIMIT = 1u << 24; // bounded mbarrier polls
+
+struct PackArgs {
+    const uint16_t *x;
+    const int32_t *idx;
+    const int32_t *slot_map;
+    const int32_t *occ;
+    uint16_t *pool_x;
+    int32_t *pool_hdr;
+    moe_pw_counters *ctr;
+    int64_t T;
+    int64_t n_slots;
+    int64_t n_pools;
+    int64_t C_s;
+    int32_t k;
+    int32_t D;
+    int32_t stages;
+    uint32_t rowbytes;
+};
+
+__global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int PACK_WARPS = blockDim.x >> 5;
+    const int NS = p.stages;
+    const uint32_t rb = p.rowbytes;
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+    unsigned char *zero = smem + ((PACK_WARPS * NS * sizeof(uint64_t) + 127) & ~size_t(127));
+    unsigned char *bufs = zero + rb;
+
+    for (uint32_t i = threadIdx.x; i < rb / 16; i += blockDim.x)
+        reinterpret_cast<uint4 *>(zero)[i] = make_uint4(0, 0, 0, 0);
+    if (lane == 0)
+        for (int s = 0; s < NS; ++s) mbar_init(&bars[warp * NS + s], 1);
+    fence_init_and_proxy();
+    __syncthreads();
+
+    const uint64_t pol_x = policy_evict_first();
+    const uint64_t pol_pool = policy_evict_first();
+    uint64_t *bar = bars + warp * NS;
+    unsigned char *buf = bufs + size_t(warp) * NS * rb;
+
+    const int64_t gw = int64_t(blockIdx.x) * PACK_WARPS + warp;
+    const int64_t GW = int64_t(gridDim.x) * PACK_WARPS;
+    const int64_t t0 = p.T * gw / GW, t1 = p.T * (gw + 1) / GW;
+    const int64_t n = t1 - t0;
+    const int64_t D = p.D;
+    const int k = p.k;
+
+    auto issue_load = [&](int64_t i) {
+        const int s = int(i % NS);
+        mbar_arrive_expect_tx(&bar[s], rb);
+        bulk_g2s(buf + size_t(s) * rb, p.x + (t0 + i) * D, rb, &bar[s], pol_x);
+    };
+
+    if (lane == 0)
+        for (int64_t i = 0; i < n && i < NS; ++i) issue_load(i);
+
+    // metadata of the next token, one (slot, expert) pair per lane j < k
+    int32_t nslot = -1, nexp = -1;
+    if (n > 0 && lane < k) {
+        nslot = p.slot_map[t0 * k + lane];
+        nexp = p.idx[t0 * k + lane];
+    }
+    bool ok = true;
+    for (int64_t i = 0; i < n; ++i) {
+        const int32_t slot = nslot, e = nexp;
+        if (i + 1 < n && lane < k) {
+            nslot = p.slot_map[(t0 + i + 1) * k + lane];
+            nexp = p.idx[(t0 + i + 1) * k + lane];
+        }
+        const int s = int(i % NS);
+        const uint32_t parity = uint32_t((i / NS) & 1);
+        const bool landed = mbar_wait_bounded(&bar[s], parity, WAIT_LIMIT);
+        if (!__all_sync(FULL_MASK, landed)) {
+            ok = false;
+            break;
+        }
+        if (slot >= p.n_slots) {
+            set_error(p.ctr, MOE_PW_DEVERR_SLOT);
+        } else if (slot >= 0) {
+            bulk_s2g(p.pool_x + int64_t(slot) * D, buf + size_t(s) * rb, rb, pol_pool);
+            p.pool_hdr[slot] = e;
+        }
+        bulk_commit();
+        if (i >= LAG) {
+            bulk_wait_read<LAG>();
+            __syncwarp();
+            const int64_t ii = i - LAG + NS;  // reuses the stage of token i - LAG
+            if (lane == 0 && ii < n) issue_load(ii);
+        }
+    }
+    if (!ok && lane == 0) set_error(p.ctr, MOE_PW_DEVERR_TIMEOUT);
+
+    // zero-fill the empty tail of each pool (pooled mode)
+    for (int64_t q = gw; q < p.n_pools; q += GW) {
+        int64_t filled = p.occ[q];
+        if (filled < 0) filled = 0;
+        if (filled > p.C_s) filled = p.C_s;
+        for (int64_t c = filled + lane; c < p.C_s; c += 32) {
+            const int64_t slot = q * p.C_s + c;
+            bulk_s2g(p.pool_x + slot * D, zero, rb, pol_pool);
+            p.pool_hdr[slot] = -1;
+        }
+        bulk_commit();
+        bulk_wait_read<8>();
+    }
+    bulk_wait_all();
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
+                        const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
+                        int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st)
+{
+    if (g.T == 0 && g.n_pools == 0) return cudaSuccess;
+    DevInfo di;
+    if (dev_info(&di) != 0) return cudaErrorUnknown;
+    PackArgs p;
+    p.x = x;
+    p.idx = idx;
+    p.slot_map = slot_map;
+    p.occ = occ;
+    p.pool_x = pool_x;
+    p.pool_hdr = pool_hdr;
+    p.ctr = ctr;
+    p.T = g.T;
+    p.n_slots = g.n_slots;
+    p.n_pools = g.n_pools;
+    p.C_s = g.C_s;
+    p.k = g.k;
+    p.D = g.D;
+    p.rowbytes = uint32_t(g.D) * 2u;
+
+    // warps and stages per warp: as many rows as fit next to the zero row,
+    // LAG + 2 .. 16 stages, dropping warps for very wide rows
+    const size_t budget = size_t(di.smem_optin) - 1024 - p.rowbytes;
+    int nw = MAX_PACK_WARPS;
+    while (nw > 1 && budget / (size_t(nw) * p.rowbytes) < size_t(LAG + 2)) --nw;
+    int stages = int(budget / (size_t(nw) * p.rowbytes));
+    if (stages > 16) stages = 16;
+    if (stages < LAG + 2) return cudaErrorInvalidValue;
+    p.stages = stages;
+    const int PACK_WARPS = nw;
+    const size_t bar_bytes = (PACK_WARPS * stages * sizeof(uint64_t) + 127) & ~size_t(127);
+    const size_t smem = bar_bytes + p.rowbytes + size_t(PACK_WARPS) * stages * p.rowbytes;
+
+    cudaError_t err = cudaFuncSetAttribute(pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           int(smem));
+    if (err != cudaSuccess) return err;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pack_kernel, PACK_WARPS * 32, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) per_sm = 1;
+    int64_t blocks = int64_t(di.sms) * per_sm;
+    const int64_t work = (g.T > g.n_pools ? g.T : g.n_pools);
+    const int64_t need = (work + PACK_WARPS - 1) / PACK_WARPS;
+    if (blocks > need) blocks = need;
+    if (blocks < 1) blocks = 1;
+    pack_kernel<<<unsigned(blocks), PACK_WARPS * 32, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace moe_pw

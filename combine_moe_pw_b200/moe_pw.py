@@ -1,0 +1,293 @@
+"""Thin Python binding of libmoe_pw.so (include/moe_pw.h), via ctypes.
+
+Each ``moe_pw_*`` function has the C entry point's name and arguments; it only
+turns torch tensors into device pointers, picks the current CUDA stream and
+raises ``MoePwError`` on a non-zero return code.  Every step of the path runs
+in the library's CUDA kernels; there is no fallback.  PyTorch provides device
+memory and streams.
+
+``Buffers`` allocates every array of the path for a config (plumbing) and
+``run_step`` chains route -> dispatch -> expert -> combine on one stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_pw.so")
+
+MOE_PW_OK, MOE_PW_EINVAL, MOE_PW_EUNSUPPORTED, MOE_PW_ECUDA, MOE_PW_EDEVICE, MOE_PW_ENOMEM = (
+    0, -1, -2, -3, -4, -5)
+MOE_PW_POOLED, MOE_PW_RAGGED = 0, 1
+DEVERR_EXPERT_ID, DEVERR_HEADER, DEVERR_TIMEOUT, DEVERR_SLOT = 1, 2, 4, 8
+
+
+class MoePwError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed: {code} ({msg})")
+        self.code = code
+
+
+class moe_pw_config(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("R", ctypes.c_int32), ("L", ctypes.c_int32),
+                ("W", ctypes.c_int32), ("P", ctypes.c_int32), ("cf_send_pct", ctypes.c_int32),
+                ("cf_recv_pct", ctypes.c_int32), ("mode", ctypes.c_int32)]
+
+
+class moe_pw_sizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("C_s", "C_r", "n_pools", "n_slots", "occ_len",
+                                              "bucket_len", "workspace_bytes", "total_bytes")]
+
+
+class moe_pw_counters(ctypes.Structure):
+    _fields_ = [("sender_dropped", ctypes.c_uint64), ("receiver_dropped", ctypes.c_uint64),
+                ("kept", ctypes.c_uint64), ("max_occ", ctypes.c_int32),
+                ("max_fill", ctypes.c_int32), ("error", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+class moe_pw_drop_stats(ctypes.Structure):
+    _fields_ = [("assignments", ctypes.c_int64), ("kept", ctypes.c_int64),
+                ("sender_dropped", ctypes.c_int64), ("receiver_dropped", ctypes.c_int64),
+                ("max_occ", ctypes.c_int32), ("max_fill", ctypes.c_int32),
+                ("error", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+# name -> argument types (after the config pointer); every function returns int
+_VP, _SZ, _I64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64
+_CFG = ctypes.POINTER(moe_pw_config)
+SIGNATURES = {
+    "moe_pw_version": [],
+    "moe_pw_strerror": [ctypes.c_int],
+    "moe_pw_plan": [_CFG, _I64, ctypes.POINTER(moe_pw_sizes)],
+    "moe_pw_route": [_CFG, _VP, _VP, _VP, _VP],
+    "moe_pw_assign": [_CFG, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "moe_pw_pack": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_bucket": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_dispatch": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "moe_pw_expert": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_combine": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_stats": [_CFG, _VP, ctypes.POINTER(moe_pw_drop_stats), _VP],
+}
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libmoe_pw.so.  Raises if it has not been built: there is no
+    fallback implementation of any step."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing; build it with "
+                              "`python -m combine_moe_pw_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(path)
+        for name, args in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_char_p if name == "moe_pw_strerror" else ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _check(name: str, rc: int):
+    if rc != MOE_PW_OK:
+        raise MoePwError(name, rc, load_library().moe_pw_strerror(rc).decode())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+@dataclass(frozen=True)
+class Config:
+    """Python mirror of ``moe_pw_config``."""
+
+    T: int
+    E: int
+    k: int
+    D: int
+    R: int
+    L: int
+    W: int
+    P: int
+    cf_send_pct: int = 110
+    cf_recv_pct: int = 115
+    mode: int = MOE_PW_POOLED
+
+    @classmethod
+    def from_workload(cls, w) -> "Config":
+        return cls(T=w.T, E=w.E, k=w.k, D=w.D, R=w.R, L=w.L, W=w.W, P=w.P,
+                   cf_send_pct=w.cf_send_pct, cf_recv_pct=w.cf_recv_pct, mode=w.mode)
+
+    def c(self) -> moe_pw_config:
+        return moe_pw_config(self.T, self.E, self.k, self.D, self.R, self.L, self.W, self.P,
+                             self.cf_send_pct, self.cf_recv_pct, self.mode)
+
+
+def _cfg(cfg) -> moe_pw_config:
+    return cfg.c() if isinstance(cfg, Config) else cfg
+
+
+def moe_pw_version() -> int:
+    return load_library().moe_pw_version()
+
+
+def moe_pw_plan(cfg, budget_bytes: int = 0) -> moe_pw_sizes:
+    out = moe_pw_sizes()
+    c = _cfg(cfg)
+    _check("moe_pw_plan", load_library().moe_pw_plan(ctypes.byref(c), budget_bytes,
+                                                     ctypes.byref(out)))
+    return out
+
+
+def moe_pw_route(cfg, logits, idx, gates, stream=None):
+    c = _cfg(cfg)
+    _check("moe_pw_route", load_library().moe_pw_route(
+        ctypes.byref(c), _ptr(logits), _ptr(idx), _ptr(gates), _stream(stream)))
+
+
+def moe_pw_assign(cfg, idx, slot_map, occ, counters, workspace, workspace_bytes=None, stream=None):
+    c = _cfg(cfg)
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check("moe_pw_assign", load_library().moe_pw_assign(
+        ctypes.byref(c), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(counters), _ptr(workspace),
+        wsb, _stream(stream)))
+
+
+def moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream=None):
+    c = _cfg(cfg)
+    _check("moe_pw_pack", load_library().moe_pw_pack(
+        ctypes.byref(c), _ptr(x), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(pool_x),
+        _ptr(pool_hdr), _ptr(counters), _stream(stream)))
+
+
+def moe_pw_bucket(cfg, pool_hdr, occ, recv_row, bucket_slot, expert_counts, counters, stream=None):
+    c = _cfg(cfg)
+    _check("moe_pw_bucket", load_library().moe_pw_bucket(
+        ctypes.byref(c), _ptr(pool_hdr), _ptr(occ), _ptr(recv_row), _ptr(bucket_slot),
+        _ptr(expert_counts), _ptr(counters), _stream(stream)))
+
+
+def moe_pw_dispatch(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, recv_row, bucket_slot,
+                    expert_counts, counters, workspace, workspace_bytes=None, stream=None):
+    c = _cfg(cfg)
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check("moe_pw_dispatch", load_library().moe_pw_dispatch(
+        ctypes.byref(c), _ptr(x), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(pool_x),
+        _ptr(pool_hdr), _ptr(recv_row), _ptr(bucket_slot), _ptr(expert_counts), _ptr(counters),
+        _ptr(workspace), wsb, _stream(stream)))
+
+
+def moe_pw_expert(cfg, pool_x, pool_hdr, recv_row, scale, ret_x, ret_hdr, stream=None):
+    c = _cfg(cfg)
+    _check("moe_pw_expert", load_library().moe_pw_expert(
+        ctypes.byref(c), _ptr(pool_x), _ptr(pool_hdr), _ptr(recv_row), _ptr(scale), _ptr(ret_x),
+        _ptr(ret_hdr), _stream(stream)))
+
+
+def moe_pw_combine(cfg, ret_x, ret_hdr, slot_map, gates, out, counters, stream=None):
+    c = _cfg(cfg)
+    _check("moe_pw_combine", load_library().moe_pw_combine(
+        ctypes.byref(c), _ptr(ret_x), _ptr(ret_hdr), _ptr(slot_map), _ptr(gates), _ptr(out),
+        _ptr(counters), _stream(stream)))
+
+
+def moe_pw_stats(cfg, counters, stream=None, raise_on_device_error: bool = True) -> moe_pw_drop_stats:
+    c = _cfg(cfg)
+    out = moe_pw_drop_stats()
+    rc = load_library().moe_pw_stats(ctypes.byref(c), _ptr(counters), ctypes.byref(out),
+                                     _stream(stream))
+    if rc == MOE_PW_EDEVICE and not raise_on_device_error:
+        return out
+    _check("moe_pw_stats", rc)
+    return out
+
+
+COUNTERS_BYTES = ctypes.sizeof(moe_pw_counters)
+
+
+class Buffers:
+    """Every device array of the path for one config, allocated with torch.
+
+    Layouts follow include/moe_pw.h.  bf16 arrays are stored as int16 tensors
+    holding the raw bits (``.view(torch.bfloat16)`` gives the values)."""
+
+    def __init__(self, cfg: Config, device="cuda", budget_bytes: int = 0):
+        self.cfg = cfg
+        self.sizes = s = moe_pw_plan(cfg, budget_bytes)
+        dev = torch.device(device)
+        T, E, k, D = cfg.T, cfg.E, cfg.k, cfg.D
+        i32, f32, i16 = torch.int32, torch.float32, torch.int16
+        self.logits = torch.empty((T, E), dtype=f32, device=dev)
+        self.x = torch.empty((T, D), dtype=i16, device=dev)
+        self.scale = torch.empty((E,), dtype=f32, device=dev)
+        self.idx = torch.empty((T, k), dtype=i32, device=dev)
+        self.gates = torch.empty((T, k), dtype=f32, device=dev)
+        self.slot_map = torch.empty((T, k), dtype=i32, device=dev)
+        self.occ = torch.empty((max(s.occ_len, 1),), dtype=i32, device=dev)
+        self.pool_x = torch.empty((s.n_slots, D), dtype=i16, device=dev)
+        self.pool_hdr = torch.empty((s.n_slots,), dtype=i32, device=dev)
+        self.recv_row = torch.empty((s.n_slots,), dtype=i32, device=dev)
+        self.bucket_slot = torch.empty((max(s.bucket_len, 1),), dtype=i32, device=dev)
+        self.expert_counts = torch.empty((2, E), dtype=i32, device=dev)
+        self.ret_x = torch.empty((s.n_slots, D), dtype=i16, device=dev)
+        self.ret_hdr = torch.empty((s.n_slots,), dtype=i32, device=dev)
+        self.out = torch.empty((T, D), dtype=f32, device=dev)
+        self.counters = torch.zeros((COUNTERS_BYTES // 8,), dtype=torch.int64, device=dev)
+        self.workspace = torch.empty((max(s.workspace_bytes, 256),), dtype=torch.uint8, device=dev)
+
+    def route(self, stream=None):
+        moe_pw_route(self.cfg, self.logits, self.idx, self.gates, stream)
+
+    def dispatch(self, stream=None):
+        moe_pw_dispatch(self.cfg, self.x, self.idx, self.slot_map, self.occ, self.pool_x,
+                        self.pool_hdr, self.recv_row, self.bucket_slot, self.expert_counts,
+                        self.counters, self.workspace, stream=stream)
+
+    def assign(self, stream=None):
+        moe_pw_assign(self.cfg, self.idx, self.slot_map, self.occ, self.counters, self.workspace,
+                      stream=stream)
+
+    def pack(self, stream=None):
+        moe_pw_pack(self.cfg, self.x, self.idx, self.slot_map, self.occ, self.pool_x,
+                    self.pool_hdr, self.counters, stream)
+
+    def bucket(self, stream=None):
+        moe_pw_bucket(self.cfg, self.pool_hdr, self.occ, self.recv_row, self.bucket_slot,
+                      self.expert_counts, self.counters, stream)
+
+    def expert(self, stream=None):
+        moe_pw_expert(self.cfg, self.pool_x, self.pool_hdr, self.recv_row, self.scale,
+                      self.ret_x, self.ret_hdr, stream)
+
+    def combine(self, stream=None):
+        moe_pw_combine(self.cfg, self.ret_x, self.ret_hdr, self.slot_map, self.gates, self.out,
+                       self.counters, stream)
+
+    def stats(self, stream=None, raise_on_device_error: bool = True) -> moe_pw_drop_stats:
+        return moe_pw_stats(self.cfg, self.counters, stream, raise_on_device_error)
+
+    def run_step(self, stream=None):
+        """route -> dispatch (assign, pack, bucket) -> expert -> combine."""
+        self.route(stream)
+        self.dispatch(stream)
+        self.expert(stream)
+        self.combine(stream)

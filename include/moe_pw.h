@@ -1,0 +1,259 @@
+/*
+ * moe_pw.h - C ABI of libmoe_pw.so: capacity-limited pooled-wave MoE token
+ * dispatch and combine on one NVIDIA B200 (sm_100a).
+ *
+ * The method is the expert-parallel transport of the Marin 535B-A23B model,
+ * described in "Marin 开始公开训练 535B 参数 MoE 模型" (lamjinlab blog),
+ * section 二 (how the sparse model is organised):
+ *   - a router picks k = 8 of E = 384 routed experts per token;
+ *   - experts sit on R = 64 expert-parallel ranks, L = 6 per rank;
+ *   - the sender builds one fixed pool per destination rank, not one buffer
+ *     per expert, and sends it in W = 3 waves of identical shape;
+ *   - the expert id travels inside the row payload, so no token counts or
+ *     routing metadata are exchanged;
+ *   - a sender factor 1.10 caps what one source sends one destination and a
+ *     receiver factor 1.15 caps the rows one local expert accepts; assignments
+ *     over either fixed buffer are dropped and the two drops are counted apart.
+ * Section 四 of the same page adds that a dropped assignment does not lose
+ * the token and names a dropless ragged all-to-all as an alternative; the
+ * huxiu article "535B大模型“直播”训练三个月" (MoE / token dropping section) notes
+ * that results come back through a second all-to-all.
+ *
+ * Here the R ranks are logical shards of one batch on one GPU: the exchange is
+ * a relabelling of pool indices in HBM (destination d reads pool (s, d, w)
+ * where source s wrote it), so nothing crosses a device boundary.
+ *
+ * Conventions that the pages leave open (and this library fixes):
+ *   - token t belongs to source s = t / (T / R); expert e lives on rank
+ *     d = e / L as local expert e % L; wave w carries local experts
+ *     {P*w, ..., P*w + P - 1} (P = L / W);
+ *   - top-k order is (logit descending, expert id ascending): equal logits go
+ *     to the lower id (float comparison: -0.0 equals +0.0); gates are the
+ *     softmax over the k chosen logits, max-subtracted, summed in j order;
+ *   - sender order: assignments (t, j) of a source in lexicographic order; the
+ *     slot of (t, j) in pool (s, d, w) is the number of earlier ones in that
+ *     pool; kept iff slot < C_s;
+ *   - receiver order: per (d, w), sources ascending, then slots ascending; the
+ *     row of an arrival is the number of earlier arrivals for its expert; kept
+ *     iff row < C_r;
+ *   - capacities C_s = ceil(cf_s% * (T/R) * k * P / (100 * E)),
+ *     C_r = ceil(cf_r% * T * k / (100 * E)); a factor <= 0 is unbounded
+ *     (C_s = (T/R) * min(k, P), C_r = T);
+ *   - empty slots hold an all-zero row and header -1;
+ *   - per-expert op (stand-in for the expert network): y = s_e * x in fp32,
+ *     rounded to bf16 nearest-even; the return pools share the dispatch pools'
+ *     slot ids; slots the receiver did not keep return zeros and header -1;
+ *   - combine: out[t] = sum over surviving j of g_j * y_j in fp32, j
+ *     ascending, one fmaf per term from +0; no renormalisation over drops.
+ *
+ * Data layout (all row-major, element types as named):
+ *   logits  f32  [T, E]
+ *   idx     i32  [T, k]          gates f32 [T, k]
+ *   x       bf16 [T, D]          (raw bits as uint16_t)
+ *   slot_map i32 [T, k]          flat slot id of (t, j), or -1 if sender-dropped
+ *   occ     i32  pooled: [R(src), R(dst), W] rows kept per pool
+ *                ragged: [E + 1] row offsets of each expert (exclusive scan)
+ *   pool_x  bf16 [n_slots, D]    pooled: slot = ((s*R + d)*W + w)*C_s + c
+ *   pool_hdr i32 [n_slots]       global expert id, or -1
+ *   recv_row i32 [n_slots]       row of the slot in its expert bucket, or -1
+ *   bucket_slot i32 [E, C_r]     slot of each bucket row, or -1 (pooled only)
+ *   expert_counts i32 [2, E]     arrivals[e], then kept[e] = min(arrivals, C_r)
+ *   scale   f32  [E]
+ *   ret_x   bf16 [n_slots, D]    ret_hdr i32 [n_slots]
+ *   out     f32  [T, D]
+ * In ragged mode n_slots = T * k rows, grouped by expert (ascending), token
+ * order inside an expert; slot_map holds row ids and nothing is dropped.
+ *
+ * Ownership: the caller allocates every buffer (device memory unless stated)
+ * and keeps it alive until the stream work completes.  The library allocates
+ * nothing and keeps no state between calls except a per-device cache of
+ * attributes; calls are reentrant.
+ *
+ * Alignment: logits, x, pool_x, ret_x and out 16-byte aligned; every other
+ * array 4-byte aligned; the workspace 256-byte aligned.
+ *
+ * Errors: every call returns MOE_PW_OK (0) or a negative code and never
+ * aborts, traps or throws.  Device-side violations (an expert id out of range
+ * in idx, a header outside its pool's experts, a bounded wait that ran out)
+ * set counters->error; moe_pw_stats reports them as MOE_PW_EDEVICE.
+ * All calls except moe_pw_plan and moe_pw_stats are asynchronous on `stream`.
+ */
+#ifndef MOE_PW_H
+#define MOE_PW_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_PW_OK 0
+#define MOE_PW_EINVAL (-1)        /* null pointer, bad config, inconsistent sizes */
+#define MOE_PW_EUNSUPPORTED (-2)  /* shape or alignment this build does not handle */
+#define MOE_PW_ECUDA (-3)         /* a CUDA runtime call or a launch failed */
+#define MOE_PW_EDEVICE (-4)       /* a kernel flagged a violation (moe_pw_stats) */
+#define MOE_PW_ENOMEM (-5)        /* buffers exceed the caller's budget (moe_pw_plan) */
+
+#define MOE_PW_POOLED 0
+#define MOE_PW_RAGGED 1
+
+/* counters->error bits */
+#define MOE_PW_DEVERR_EXPERT_ID 1   /* idx entry outside [0, E) */
+#define MOE_PW_DEVERR_HEADER 2      /* pool header outside its (d, w) experts */
+#define MOE_PW_DEVERR_TIMEOUT 4     /* a bounded wait gave up */
+#define MOE_PW_DEVERR_SLOT 8        /* slot_map entry outside [-1, n_slots) */
+
+/* Problem description.  Limits of this build: 1 <= k <= 32, k <= E,
+ * E == R * L, L == W * P, E <= 2048 (and E % 4 == 0 for moe_pw_route),
+ * T % R == 0, 8 <= D <= 12288 with D % 8 == 0, R * W <= 2048. */
+typedef struct moe_pw_config {
+    int64_t T;            /* tokens in the batch (>= 0) */
+    int32_t E;            /* routed experts */
+    int32_t k;            /* experts chosen per token */
+    int32_t D;            /* latent width, bf16 elements */
+    int32_t R;            /* expert-parallel ranks (logical) */
+    int32_t L;            /* experts per rank */
+    int32_t W;            /* waves per (source, destination) */
+    int32_t P;            /* experts per wave */
+    int32_t cf_send_pct;  /* sender capacity factor, percent (110); <= 0 unbounded */
+    int32_t cf_recv_pct;  /* receiver capacity factor, percent (115); <= 0 unbounded */
+    int32_t mode;         /* MOE_PW_POOLED or MOE_PW_RAGGED */
+} moe_pw_config;
+
+/* Sizes derived from a config by moe_pw_plan.  Element counts unless "bytes". */
+typedef struct moe_pw_sizes {
+    int64_t C_s;            /* sender capacity per (s, d, w) pool (pooled) */
+    int64_t C_r;            /* receiver capacity per expert (pooled) */
+    int64_t n_pools;        /* R * R * W (pooled), 0 (ragged) */
+    int64_t n_slots;        /* rows of pool_x / ret_x */
+    int64_t occ_len;        /* int32 entries of occ */
+    int64_t bucket_len;     /* int32 entries of bucket_slot (0 in ragged mode) */
+    int64_t workspace_bytes;/* scratch for moe_pw_assign / moe_pw_dispatch */
+    int64_t total_bytes;    /* every buffer of the path, logits to out */
+} moe_pw_sizes;
+
+/* Device-side counters, written by the kernels.  moe_pw_assign zeroes them. */
+typedef struct moe_pw_counters {
+    unsigned long long sender_dropped;
+    unsigned long long receiver_dropped;
+    unsigned long long kept;
+    int32_t max_occ;     /* largest pool occupancy */
+    int32_t max_fill;    /* largest per-expert kept count */
+    int32_t error;       /* MOE_PW_DEVERR_* bits */
+    int32_t reserved;
+} moe_pw_counters;
+
+/* Host copy of the counters, filled by moe_pw_stats. */
+typedef struct moe_pw_drop_stats {
+    int64_t assignments;       /* T * k */
+    int64_t kept;              /* rows every expert accepted */
+    int64_t sender_dropped;
+    int64_t receiver_dropped;
+    int32_t max_occ;
+    int32_t max_fill;
+    int32_t error;
+    int32_t reserved;
+} moe_pw_drop_stats;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int moe_pw_version(void);
+
+/* Text for a return code (static storage). */
+const char *moe_pw_strerror(int code);
+
+/*
+ * Host-only.  Validates `cfg` and fills `out` with capacities and buffer
+ * sizes.  budget_bytes > 0 makes the call fail with MOE_PW_ENOMEM when the
+ * path's buffers (out->total_bytes) exceed it: the pages record a fixed
+ * expert-cell design whose memory estimate failed allocation, and a caller
+ * can refuse such a config before allocating.  Never touches the GPU.
+ */
+int moe_pw_plan(const moe_pw_config *cfg, int64_t budget_bytes, moe_pw_sizes *out);
+
+/*
+ * Route (section 二: the router picks k experts per token).  One warp per
+ * token selects the k largest logits (ties to the lower id) and writes their
+ * ids to idx and their softmax gates to gates.  Logits must be finite.
+ */
+int moe_pw_route(const moe_pw_config *cfg, const float *logits, int32_t *idx, float *gates,
+                 cudaStream_t stream);
+
+/*
+ * Sender slot assignment (section 二: fixed per-destination pools, sender
+ * factor).  Zeroes *counters, then writes slot_map and occ and counts sender
+ * drops.  Ranks come from per-chunk histograms and a prefix scan over chunks,
+ * so the result is deterministic.  Ragged mode: slot_map receives row ids and
+ * occ the E + 1 expert row offsets.  workspace: device scratch of at least
+ * moe_pw_sizes.workspace_bytes, 256-byte aligned; its contents on entry do
+ * not matter.
+ */
+int moe_pw_assign(const moe_pw_config *cfg, const int32_t *idx, int32_t *slot_map,
+                  int32_t *occ, moe_pw_counters *counters, void *workspace,
+                  size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Pack (section 二: expert id in the payload).  Copies each kept row x[t] into
+ * its slot with TMA bulk copies through shared memory (one read of x[t], up to
+ * k writes), writes the expert id into the slot header, and fills the empty
+ * tail of every pool (positions >= occ) with zeros and header -1.  Ragged
+ * mode: rows only, no empty slots.  A slot_map entry >= n_slots is skipped
+ * and flagged in counters->error (which moe_pw_assign zeroed).
+ */
+int moe_pw_pack(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
+                const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
+                int32_t *pool_hdr, moe_pw_counters *counters, cudaStream_t stream);
+
+/*
+ * Exchange + receiver bucketing (section 二: receiver factor; huxiu: first
+ * all-to-all).  For every (d, w) walks the pools (s, d, w), s ascending, over
+ * positions c < occ, and ranks each arrival within its expert.  Writes
+ * recv_row, bucket_slot (pooled; may be NULL in ragged mode) and
+ * expert_counts, and adds receiver drops and kept rows to *counters.
+ */
+int moe_pw_bucket(const moe_pw_config *cfg, const int32_t *pool_hdr, const int32_t *occ,
+                  int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,
+                  moe_pw_counters *counters, cudaStream_t stream);
+
+/* moe_pw_assign, moe_pw_pack and moe_pw_bucket in one call. */
+int moe_pw_dispatch(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
+                    int32_t *slot_map, int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr,
+                    int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,
+                    moe_pw_counters *counters, void *workspace, size_t workspace_bytes,
+                    cudaStream_t stream);
+
+/*
+ * Per-expert op and return layout (stand-in for the expert network; huxiu:
+ * results return by a second all-to-all).  For every slot: if the receiver
+ * kept it (recv_row >= 0), ret_x = bf16_rn(scale[e] * pool_x) and ret_hdr = e;
+ * otherwise ret_x = 0 and ret_hdr = -1.
+ */
+int moe_pw_expert(const moe_pw_config *cfg, const uint16_t *pool_x, const int32_t *pool_hdr,
+                  const int32_t *recv_row, const float *scale, uint16_t *ret_x,
+                  int32_t *ret_hdr, cudaStream_t stream);
+
+/*
+ * Combine (section 四: a dropped assignment leaves the token, so its term is
+ * simply absent).  out[t] = sum_j g_j * float(ret_x[slot_map[t][j]]) over
+ * j with slot >= 0 and ret_hdr[slot] >= 0, fp32, j ascending, fmaf from +0.
+ * A slot_map entry >= n_slots is skipped and flagged in counters->error.
+ */
+int moe_pw_combine(const moe_pw_config *cfg, const uint16_t *ret_x, const int32_t *ret_hdr,
+                   const int32_t *slot_map, const float *gates, float *out,
+                   moe_pw_counters *counters, cudaStream_t stream);
+
+/*
+ * Drop statistics (section 二: the two kinds of drop are reported apart).
+ * Copies *counters (device) to *host_out (host memory) and synchronises the
+ * stream.  Returns MOE_PW_EDEVICE when a kernel flagged a violation (the
+ * stats are still filled).
+ */
+int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
+                 moe_pw_drop_stats *host_out, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_PW_H */

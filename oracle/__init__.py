@@ -96,6 +96,7 @@ def _configure(lib):
     lib.orc_assign_pooled.argtypes = [gp, vp, vp, vp, vp]
     lib.orc_assign_pooled.restype = i64
     lib.orc_pack.argtypes = [gp, i64, vp, vp, vp, vp, vp]
+    lib.orc_pack_headers.argtypes = [gp, i64, vp, vp, vp]
     lib.orc_bucket.argtypes = [gp, vp, vp, vp, vp, vp, vp]
     lib.orc_bucket.restype = i64
     lib.orc_assign_ragged.argtypes = [gp, vp, vp, vp, vp, vp]
@@ -203,6 +204,14 @@ def pack(g: Geom, n_slots: int, x: np.ndarray, idx: np.ndarray, slot_map: np.nda
     return pool_x, pool_hdr
 
 
+def pack_headers(g: Geom, n_slots: int, idx: np.ndarray, slot_map: np.ndarray) -> np.ndarray:
+    pool_hdr = np.empty((n_slots,), np.int32)
+    gc = g.c()
+    _load().orc_pack_headers(ctypes.byref(gc), n_slots, _p(_c(idx, np.int32)),
+                             _p(_c(slot_map, np.int32)), _p(pool_hdr))
+    return pool_hdr
+
+
 def bucket(g: Geom, pool_hdr: np.ndarray, occ: np.ndarray):
     recv_row = np.empty((g.n_slots,), np.int32)
     bucket_slot = np.empty((g.E, g.C_r), np.int32)
@@ -260,6 +269,30 @@ def combine_tokens(g: Geom, x, idx, gates, slot_map, recv_row, scale, tokens):
                                _p(_c(recv_row, np.int32)), _p(_c(scale, np.float32)),
                                _p(tokens), tokens.size, _p(out), _p(mag))
     return out, mag
+
+
+def run_headers(w, logits: np.ndarray) -> dict:
+    """The integer part of the path (route, assignment, headers, bucketing)
+    plus the gates, without materialising any pool rows.  Rows are checked
+    per slot / per token with ``combine_tokens`` and ``expert_product``."""
+    g = geom_for(w)
+    r = {"geom": g}
+    r["idx"], r["gates"] = route(g, logits)
+    if w.mode == 0:
+        r["slot_map"], r["occ"], r["slot_tok"], r["sender_dropped"] = assign_pooled(g, r["idx"])
+        r["pool_hdr"] = pack_headers(g, g.n_slots, r["idx"], r["slot_map"])
+        (r["recv_row"], r["bucket_slot"], r["arrivals"], r["bucket_cnt"],
+         r["receiver_dropped"]) = bucket(g, r["pool_hdr"], r["occ"])
+    else:
+        r["slot_map"], r["row_off"], r["row_cnt"], r["slot_tok"] = assign_ragged(g, r["idx"])
+        n_rows = g.T * g.k
+        r["pool_hdr"] = pack_headers(g, n_rows, r["idx"], r["slot_map"])
+        r["recv_row"] = (np.arange(n_rows, dtype=np.int64)
+                         - np.repeat(r["row_off"][:-1], r["row_cnt"])).astype(np.int32)
+        r["sender_dropped"] = r["receiver_dropped"] = 0
+        r["arrivals"] = r["bucket_cnt"] = r["row_cnt"]
+    r["kept"] = int(np.asarray(r["bucket_cnt"], np.int64).sum())
+    return r
 
 
 def bf16_round(a: np.ndarray) -> np.ndarray:

@@ -223,6 +223,19 @@ void orc_pack(const orc_geom *g, int64_t n_slots, const uint16_t *x, const int32
     }
 }
 
+/* The header half of the pack alone (same definition, rows left out), for
+ * batches whose pools are too large to materialise on the host. */
+void orc_pack_headers(const orc_geom *g, int64_t n_slots, const int32_t *idx,
+                      const int32_t *slot_map, int32_t *pool_hdr)
+{
+    for (int64_t q = 0; q < n_slots; ++q) pool_hdr[q] = -1;
+    for (int64_t t = 0; t < g->T; ++t)
+        for (int32_t j = 0; j < g->k; ++j) {
+            const int64_t slot = slot_map[t * g->k + j];
+            if (slot >= 0) pool_hdr[slot] = idx[t * g->k + j];
+        }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Exchange + receiver bucketing (pooled).                                   */
 /* ------------------------------------------------------------------------ */

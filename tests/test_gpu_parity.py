@@ -1,0 +1,307 @@
+"""GPU path against the CPU oracle, element by element, through the C ABI.
+
+Bar: bit-exact for every integer/byte output (top-k ids, slot maps, pool
+occupancy, pool rows and headers, receiver rows, buckets, per-expert counts,
+returned rows and headers, drop counts); the fp32 gates within 1e-6 relative;
+the fp32 combine within 1e-6 of sum_j g_j |y_j| (the combine's own scale, so
+cancelling terms do not make the bound meaningless; where that scale is 0 the
+output must be exactly 0).
+
+Small cases run the whole oracle.  Full-size cases (the pages' shapes) run
+the oracle's integer path completely and check rows on sampled slots and the
+combine on sampled tokens, in the same launch configuration bench.py times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_moe_pw_b200 import moe_pw as mp
+from combine_moe_pw_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+GATE_RTOL = 1e-6
+COMBINE_TOL = 1e-6
+
+
+def _inputs(w, logits=None):
+    lg = synth.logits(w) if logits is None else logits
+    return lg, synth.x_bf16(w), synth.scales(w)
+
+
+def run_gpu(w, lg, x, s, sub_steps=False):
+    cfg = mp.Config.from_workload(w)
+    b = mp.Buffers(cfg)
+    b.logits.copy_(torch.from_numpy(lg))
+    b.x.copy_(torch.from_numpy(x.view(np.int16)))
+    b.scale.copy_(torch.from_numpy(s))
+    if sub_steps:
+        b.route()
+        b.assign()
+        b.pack()
+        b.bucket()
+        b.expert()
+        b.combine()
+    else:
+        b.run_step()
+    st = b.stats(raise_on_device_error=False)
+    torch.cuda.synchronize()
+    return b, st
+
+
+def _np(t):
+    return t.cpu().numpy()
+
+
+def _u16(t):
+    return t.cpu().numpy().view(np.uint16)
+
+
+def check_gates(g_gpu, g_ref):
+    rel = np.abs(g_gpu.astype(np.float64) - g_ref) / g_ref
+    assert rel.max() <= GATE_RTOL, f"gate rel err {rel.max():.3e}"
+
+
+def check_combine(out_gpu, ref, mag):
+    diff = np.abs(out_gpu.astype(np.float64) - ref)
+    zero = mag == 0
+    assert not diff[zero].any(), "output must be exactly 0 where every term is 0"
+    err = (diff[~zero] / mag[~zero]).max() if (~zero).any() else 0.0
+    assert err <= COMBINE_TOL, f"combine err {err:.3e}"
+    return err
+
+
+def check_full(w, lg, x, s, b, st):
+    """Every output against the whole oracle."""
+    r = oracle.run(w, lg, x, s, with_mag=True)
+    g = r["geom"]
+    np.testing.assert_array_equal(_np(b.idx), r["idx"])
+    check_gates(_np(b.gates), r["gates"])
+    np.testing.assert_array_equal(_np(b.slot_map), r["slot_map"])
+    if w.mode == synth.MODE_POOLED:
+        np.testing.assert_array_equal(_np(b.occ)[: g.n_pools], r["occ"].reshape(-1))
+        np.testing.assert_array_equal(_np(b.bucket_slot)[: w.E * g.C_r], r["bucket_slot"].reshape(-1))
+    else:
+        np.testing.assert_array_equal(_np(b.occ)[: w.E + 1], r["row_off"])
+    np.testing.assert_array_equal(_u16(b.pool_x), r["pool_x"])
+    np.testing.assert_array_equal(_np(b.pool_hdr), r["pool_hdr"])
+    np.testing.assert_array_equal(_np(b.recv_row), r["recv_row"])
+    ec = _np(b.expert_counts)
+    np.testing.assert_array_equal(ec[0], r["arrivals"])
+    np.testing.assert_array_equal(ec[1], r["bucket_cnt"])
+    np.testing.assert_array_equal(_u16(b.ret_x), r["ret_x"])
+    np.testing.assert_array_equal(_np(b.ret_hdr), r["ret_hdr"])
+    err = check_combine(_np(b.out), r["out"], r["mag"])
+    assert st.error == 0
+    assert (st.sender_dropped, st.receiver_dropped, st.kept) == (
+        r["sender_dropped"], r["receiver_dropped"], r["kept"])
+    assert st.assignments == w.T * w.k
+    assert st.kept + st.sender_dropped + st.receiver_dropped == w.T * w.k
+    return r, err
+
+
+def check_sampled(w, lg, x, s, b, st, n_tok=1024, n_slot=8192, seed=0):
+    """Integer path in full, rows and combine on samples (oracle per slot /
+    per token)."""
+    r = oracle.run_headers(w, lg)
+    g = r["geom"]
+    np.testing.assert_array_equal(_np(b.idx), r["idx"])
+    check_gates(_np(b.gates), r["gates"])
+    np.testing.assert_array_equal(_np(b.slot_map), r["slot_map"])
+    if w.mode == synth.MODE_POOLED:
+        np.testing.assert_array_equal(_np(b.occ)[: g.n_pools], r["occ"].reshape(-1))
+        np.testing.assert_array_equal(_np(b.bucket_slot)[: w.E * g.C_r], r["bucket_slot"].reshape(-1))
+    else:
+        np.testing.assert_array_equal(_np(b.occ)[: w.E + 1], r["row_off"])
+    np.testing.assert_array_equal(_np(b.pool_hdr), r["pool_hdr"])
+    np.testing.assert_array_equal(_np(b.recv_row), r["recv_row"])
+    ec = _np(b.expert_counts)
+    np.testing.assert_array_equal(ec[0], r["arrivals"])
+    np.testing.assert_array_equal(ec[1], r["bucket_cnt"])
+    assert (st.sender_dropped, st.receiver_dropped, st.kept, st.error) == (
+        r["sender_dropped"], r["receiver_dropped"], r["kept"], 0)
+
+    rng = np.random.default_rng(seed)
+    n_slots = r["pool_hdr"].size
+    slots = np.unique(np.concatenate([rng.integers(0, n_slots, n_slot), [0, n_slots - 1]]))
+    st_idx = torch.from_numpy(slots).to(b.pool_x.device)
+    pool_rows = _u16(b.pool_x.index_select(0, st_idx))
+    ret_rows = _u16(b.ret_x.index_select(0, st_idx))
+    tok = r["slot_tok"][slots]
+    full = tok >= 0
+    exp_pool = np.zeros_like(pool_rows)
+    exp_pool[full] = x[tok[full]]
+    np.testing.assert_array_equal(pool_rows, exp_pool)
+    kept = r["recv_row"][slots] >= 0
+    exp_ret = np.zeros_like(ret_rows)
+    e = r["pool_hdr"][slots][kept]
+    exp_ret[kept] = oracle.expert_product(np.repeat(s[e][:, None], w.D, axis=1), x[tok[kept]])
+    np.testing.assert_array_equal(ret_rows, exp_ret)
+    np.testing.assert_array_equal(_np(b.ret_hdr)[slots], np.where(kept, r["pool_hdr"][slots], -1))
+
+    toks = np.unique(np.concatenate([rng.integers(0, w.T, n_tok), [0, w.T - 1]]))
+    ref, mag = oracle.combine_tokens(g, x, r["idx"], r["gates"], r["slot_map"], r["recv_row"], s,
+                                     toks)
+    out = _np(b.out[torch.from_numpy(toks).to(b.out.device)])
+    return r, check_combine(out, ref, mag)
+
+
+# ---------------------------------------------------------------------------
+# small cases, whole oracle
+# ---------------------------------------------------------------------------
+
+TINY = synth.WORKLOADS["tiny"]
+
+SMALL_CASES = {
+    "tiny": TINY,
+    "tiny_ragged": TINY.with_(mode=synth.MODE_RAGGED, cf_send_pct=0, cf_recv_pct=0),
+    "tiny_ragged_zipf": TINY.with_(mode=synth.MODE_RAGGED, cf_send_pct=0, cf_recv_pct=0,
+                                   logit_kind=synth.LOGIT_ZIPF),
+    "tiny_unbounded": TINY.with_(cf_send_pct=0, cf_recv_pct=0),
+    "tiny_tight": TINY.with_(cf_send_pct=60, cf_recv_pct=70),
+    "tiny_zipf": TINY.with_(logit_kind=synth.LOGIT_ZIPF),
+    "tiny_seqbias": TINY.with_(logit_kind=synth.LOGIT_SEQBIAS),
+    "k1": TINY.with_(k=1),
+    "k4": TINY.with_(k=4),
+    "k16": TINY.with_(k=16),
+    "k32": TINY.with_(k=32),
+    "min_width": TINY.with_(D=8),
+    "odd_width": TINY.with_(D=136),
+    "max_width": TINY.with_(T=256, D=12288),
+    "single_pool": TINY.with_(R=1, L=16, W=1, P=16, T=512, cf_send_pct=30),
+    "ragged_tail": TINY.with_(T=8 * 37, seq_len=37),
+    "ragged_tail_ragged": TINY.with_(T=8 * 37, seq_len=37, mode=synth.MODE_RAGGED,
+                                     cf_send_pct=0, cf_recv_pct=0),
+    "many_chunks": TINY.with_(T=8 * 1000 + 0, seq_len=1000, D=64),
+    "wide_E": synth.Workload("wide_E", T=64 * 24, R=64, L=16, W=4, P=4, k=8, D=64, seq_len=24,
+                             logit_kind=synth.LOGIT_SEQBIAS),
+    "E2048": synth.Workload("E2048", T=256 * 8, R=256, L=8, W=4, P=2, k=8, D=32, seq_len=64,
+                            logit_kind=synth.LOGIT_IID),
+    "pages_ranks_small": synth.Workload("pages_ranks_small", T=64 * 64, R=64, L=6, W=3, P=2, k=8,
+                                        D=256, seq_len=1024, logit_kind=synth.LOGIT_SEQBIAS),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL_CASES))
+def test_small_full_parity(name):
+    w = SMALL_CASES[name]
+    lg, x, s = _inputs(w)
+    b, st = run_gpu(w, lg, x, s)
+    check_full(w, lg, x, s, b, st)
+
+
+def test_ties_quantised_logits():
+    lg, x, s = _inputs(TINY)
+    lg = (np.round(lg * 2) / 2).astype(np.float32)  # many exact ties
+    lg[::7, 5] = -0.0
+    lg[::7, 9] = 0.0
+    b, st = run_gpu(TINY, lg, x, s)
+    check_full(TINY, lg, x, s, b, st)
+
+
+def test_all_equal_logits_closed_form():
+    lg, x, s = _inputs(TINY)
+    lg = np.full_like(lg, 0.25)
+    b, st = run_gpu(TINY, lg, x, s)
+    np.testing.assert_array_equal(_np(b.idx), np.tile(np.arange(8, dtype=np.int32), (TINY.T, 1)))
+    assert np.all(_np(b.gates) == np.float32(0.125))  # exp(0)/8 exactly
+    check_full(TINY, lg, x, s, b, st)
+
+
+def test_identity_experts_return_x():
+    """Unbounded capacity and s_e = 1: out = x * sum_j g_j, within a few fp32 ulp of x."""
+    w = TINY.with_(cf_send_pct=0, cf_recv_pct=0)
+    lg, x, _ = _inputs(w)
+    s = np.ones(w.E, np.float32)
+    b, st = run_gpu(w, lg, x, s)
+    assert st.sender_dropped == st.receiver_dropped == 0
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    np.testing.assert_allclose(_np(b.out), xf, rtol=8 * 2.0 ** -23, atol=0)
+
+
+def test_sub_steps_equal_dispatch():
+    lg, x, s = _inputs(TINY)
+    b1, st1 = run_gpu(TINY, lg, x, s)
+    b2, st2 = run_gpu(TINY, lg, x, s, sub_steps=True)
+    for name in ["idx", "gates", "slot_map", "occ", "pool_x", "pool_hdr", "recv_row",
+                 "bucket_slot", "expert_counts", "ret_x", "ret_hdr", "out"]:
+        assert torch.equal(getattr(b1, name), getattr(b2, name)), name
+
+
+def test_deterministic_repeat():
+    """Two runs, one on a side stream, give the same bytes everywhere."""
+    w = synth.WORKLOADS["tiny"].with_(T=8 * 2048, seq_len=2048, D=256)
+    lg, x, s = _inputs(w)
+    b1, _ = run_gpu(w, lg, x, s)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        b2, _ = run_gpu(w, lg, x, s)
+    side.synchronize()
+    for name in ["idx", "gates", "slot_map", "occ", "pool_x", "pool_hdr", "recv_row",
+                 "bucket_slot", "expert_counts", "ret_x", "ret_hdr", "out"]:
+        assert torch.equal(getattr(b1, name), getattr(b2, name)), name
+
+
+def test_empty_batch():
+    for mode in (synth.MODE_POOLED, synth.MODE_RAGGED):
+        w = TINY.with_(T=0, mode=mode)
+        cfg = mp.Config.from_workload(w)
+        b = mp.Buffers(cfg)
+        b.expert_counts.fill_(7)
+        b.run_step()
+        st = b.stats()
+        assert (st.assignments, st.kept, st.sender_dropped, st.receiver_dropped) == (0, 0, 0, 0)
+        assert int(b.expert_counts.abs().sum()) == 0
+
+
+def test_bad_expert_ids_are_flagged_not_faulted():
+    """idx entries outside [0, E) are caught by the assignment kernels'
+    bounds checks: the assignment gets no slot and the error bit is set."""
+    lg, x, s = _inputs(TINY)
+    cfg = mp.Config.from_workload(TINY)
+    b = mp.Buffers(cfg)
+    b.logits.copy_(torch.from_numpy(lg))
+    b.x.copy_(torch.from_numpy(x.view(np.int16)))
+    b.route()
+    b.idx[5, 3] = -7
+    b.idx[100, 0] = TINY.E + 3
+    b.assign()
+    b.pack()
+    b.bucket()
+    st = b.stats(raise_on_device_error=False)
+    assert st.error & mp.DEVERR_EXPERT_ID
+    assert int(b.slot_map[5, 3]) == -1 and int(b.slot_map[100, 0]) == -1
+    with pytest.raises(mp.MoePwError) as ei:
+        b.stats()
+    assert ei.value.code == mp.MOE_PW_EDEVICE
+
+
+def test_bad_slot_in_combine_is_flagged():
+    lg, x, s = _inputs(TINY)
+    b, st = run_gpu(TINY, lg, x, s)
+    ref = b.out.clone()
+    b.slot_map[3, 2] = int(b.pool_hdr.numel()) + 5
+    b.combine()
+    st = b.stats(raise_on_device_error=False)
+    assert st.error & mp.DEVERR_SLOT
+    assert torch.equal(b.out[:3], ref[:3]) and torch.equal(b.out[4:], ref[4:])
+
+
+# ---------------------------------------------------------------------------
+# the pages' shapes, bench launch configuration, sampled rows
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["layer", "rack", "long", "ragged"])
+def test_full_size_sampled_parity(name):
+    w = synth.WORKLOADS[name]
+    lg, x, s = _inputs(w)
+    b, st = run_gpu(w, lg, x, s)
+    r, err = check_sampled(w, lg, x, s, b, st)
+    if name == "long":  # fewer, longer sequences -> worse balance than the rack batch
+        rr = oracle.run_headers(synth.WORKLOADS["rack"], synth.logits(synth.WORKLOADS["rack"]))
+        assert r["sender_dropped"] + r["receiver_dropped"] > rr["sender_dropped"] + rr["receiver_dropped"]
+    if name == "ragged":
+        assert r["kept"] == w.T * w.k
+    del b
+    torch.cuda.empty_cache()
