@@ -2,6 +2,7 @@
 // The kernels live in route.cu, assign.cu, pack.cu, bucket.cu, expert.cu and
 // combine.cu; this file owns validation and the contract of include/moe_pw.h.
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -284,3 +285,61 @@ int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of moe_pw_assign.
+//
+// Some callers cannot hand this library a workspace: a plugin whose host
+// process owns all device memory and exposes no allocator to it, or a
+// latency-critical loop that must never call cudaMalloc/cudaFree (both can
+// synchronise the whole device).  For them, moe_pw_assign_noalloc keeps the
+// ranking scratch in a fixed array compiled into the library instead.
+// ---------------------------------------------------------------------------
+
+namespace moe_pw {
+namespace {
+
+// Fixed scratch of the allocation-free assign: 4 MiB on every device that
+// loads this library, held until the process exits.
+constexpr size_t NOALLOC_SCRATCH_BYTES = MOE_PW_NOALLOC_SCRATCH_BYTES;
+__device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch, looked up once per device with that
+// device current (in host code the symbol's name is only a host-side handle).
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[64];
+
+int noalloc_scratch(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_PW_ECUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_PW_ECUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return MOE_PW_OK;
+}
+
+}  // namespace
+}  // namespace moe_pw
+
+extern "C" int moe_pw_assign_noalloc(const moe_pw_config *cfg, const int32_t *idx,
+                                     int32_t *slot_map, int32_t *occ, moe_pw_counters *counters,
+                                     cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!counters || !occ) return MOE_PW_EINVAL;
+    if (g.T > 0 && (!idx || !slot_map)) return MOE_PW_EINVAL;
+    if (ws_bytes(g) > int64_t(NOALLOC_SCRATCH_BYTES)) return MOE_PW_ENOMEM;
+    if (!aligned(counters, 8) || !aligned(occ, 4) ||
+        (g.T > 0 && (!aligned(idx, 4) || !aligned(slot_map, 4))))
+        return MOE_PW_EUNSUPPORTED;
+    void *scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch)) != MOE_PW_OK) return rc;
+    return cuda_rc(launch_assign(g, idx, slot_map, occ, counters, scratch, stream));
+}

@@ -67,6 +67,7 @@ SIGNATURES = {
     "moe_pw_plan": [_CFG, _I64, ctypes.POINTER(moe_pw_sizes)],
     "moe_pw_route": [_CFG, _VP, _VP, _VP, _VP],
     "moe_pw_assign": [_CFG, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "moe_pw_assign_noalloc": [_CFG, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_pack": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_bucket": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_dispatch": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
@@ -170,6 +171,17 @@ def moe_pw_assign(cfg, idx, slot_map, occ, counters, workspace, workspace_bytes=
     _check("moe_pw_assign", load_library().moe_pw_assign(
         ctypes.byref(c), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(counters), _ptr(workspace),
         wsb, _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20  # MOE_PW_NOALLOC_SCRATCH_BYTES
+
+
+def moe_pw_assign_noalloc(cfg, idx, slot_map, occ, counters, stream=None):
+    """moe_pw_assign without a workspace argument: the library's built-in
+    scratch array is used (see include/moe_pw.h for its limits)."""
+    c = _cfg(cfg)
+    _check("moe_pw_assign_noalloc", load_library().moe_pw_assign_noalloc(
+        ctypes.byref(c), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(counters), _stream(stream)))
 
 
 def moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream=None):

@@ -216,6 +216,35 @@ int moe_pw_bucket(const moe_pw_config *cfg, const int32_t *pool_hdr, const int32
                   int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,
                   moe_pw_counters *counters, cudaStream_t stream);
 
+/*
+ * Allocation-free moe_pw_assign.  (The pages have no counterpart: this is an
+ * interface convenience of this library, not part of the method.)
+ *
+ * For callers that cannot allocate device memory for a workspace: a plugin
+ * whose host process owns every device allocation and gives it no allocator,
+ * or a latency-critical loop that must never call cudaMalloc/cudaFree, which
+ * can synchronise the whole device.  Same inputs, outputs and results as
+ * moe_pw_assign, but the ranking scratch is a fixed array of
+ * MOE_PW_NOALLOC_SCRATCH_BYTES compiled into the library: every GPU that
+ * loads the library holds it until the process exits.  This call allocates
+ * nothing and calls no allocating routine.
+ *   - A batch whose ranking needs more scratch than that (workspace_bytes of
+ *     moe_pw_plan above the limit) is refused with MOE_PW_ENOMEM before any
+ *     launch; the rack-scale batch (262,144 tokens, 64 ranks, 3 waves) needs
+ *     under 1 MiB.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents; nothing in it needs to start at zero (each call writes every
+ *     entry it reads).  Calls whose kernels overlap on the GPU, such as calls
+ *     on two streams without ordering between them, race on the array and
+ *     give wrong slots: order them on one stream or with events.
+ */
+#define MOE_PW_NOALLOC_SCRATCH_BYTES (4u << 20)
+int moe_pw_assign_noalloc(const moe_pw_config *cfg, const int32_t *idx, int32_t *slot_map,
+                          int32_t *occ, moe_pw_counters *counters, cudaStream_t stream);
+
 /* moe_pw_assign, moe_pw_pack and moe_pw_bucket in one call. */
 int moe_pw_dispatch(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
                     int32_t *slot_map, int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr,
