@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
     ap.add_argument("--cpu-sample-sources", type=int, default=16)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the batch's token count (profiling a smaller case)")
     return ap.parse_args()
 
 
@@ -225,6 +227,8 @@ def main():
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
 
     base = synth.WORKLOADS[a.workload]
+    if a.tokens:
+        base = base.with_(T=a.tokens, seq_len=min(base.seq_len, a.tokens // base.R * base.R))
     w = base.with_(seed=base.seed + rank)
     cfg = mp.Config.from_workload(w)
     b = mp.Buffers(cfg, device=dev)
