@@ -7,10 +7,14 @@
 //
 // Layout: lane l holds float4 number l + 32*v of the row (v < NV), i.e. the
 // logits of experts 4*(l + 32*v) + c.  Each logit becomes an order-preserving
-// unsigned key (0 marks "taken or absent").  A selection round is one
-// warp-wide max of the keys (redux.sync) followed by a warp-wide min of the
-// expert ids holding that key, which settles ties toward the lower id.  The
-// next token's row is loaded while the current one is being selected.
+// unsigned key (0 marks "taken or absent").
+// Selection: tau = the k-th largest of the 32 lane maxima bounds the top k
+// from below; the logits >= tau (typically ~k of them) are compacted into
+// shared memory and ranked exactly by (key descending, id ascending).  When
+// more than 32 logits pass (many equal values), k exact rounds run instead:
+// a warp-wide max of the keys (redux.sync), then a warp-wide min of the ids
+// holding it.  The next token's row is loaded while the current one is
+// being selected.
 #include "common.cuh"
 
 namespace moe_pw {
@@ -44,13 +48,19 @@ __device__ __forceinline__ void load_row(const float *__restrict__ logits, int64
     }
 }
 
+constexpr int ROUTE_WARPS = 8;
+
 template <int NV>
-__global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ logits,
-                                                    int32_t *__restrict__ idx,
-                                                    float *__restrict__ gates, int64_t T,
-                                                    int E, int k)
+__global__ void __launch_bounds__(ROUTE_WARPS * 32) route_kernel(const float *__restrict__ logits,
+                                                                 int32_t *__restrict__ idx,
+                                                                 float *__restrict__ gates,
+                                                                 int64_t T, int E, int k)
 {
+    // per warp: candidate list and the selected (key, id) pairs in rank order
+    __shared__ uint2 cand_sm[ROUTE_WARPS][32];
+    __shared__ uint2 sel_sm[ROUTE_WARPS][32];
     const int lane = threadIdx.x & 31;
+    const int wib = threadIdx.x >> 5;
     const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarp = (int64_t(gridDim.x) * blockDim.x) >> 5;
     const int E4 = E >> 2;
@@ -71,33 +81,85 @@ __global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ lo
             key[v][2] = in ? order_key(cur[v].z) : 0u;
             key[v][3] = in ? order_key(cur[v].w) : 0u;
         }
+        uint32_t lm = 0;
+#pragma unroll
+        for (int v = 0; v < NV; ++v)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) lm = max(lm, key[v][c]);
+
+        // tau = k-th largest lane maximum: at least k logits are >= tau, so
+        // every one of the top k is >= tau.  Usually few logits pass.
+        uint32_t rem = lm, tau = 0;
+        for (int j = 0; j < k; ++j) {
+            tau = __reduce_max_sync(FULL_MASK, rem);
+            if (rem == tau) rem = 0u;
+        }
+        int cnt = 0;
+#pragma unroll
+        for (int v = 0; v < NV; ++v)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) cnt += key[v][c] >= tau;
+        const int C = tau ? int(__reduce_add_sync(FULL_MASK, unsigned(cnt))) : 1 << 30;
 
         uint32_t sel_key = 0;
         int32_t sel_idx = 0;
-        for (int j = 0; j < k; ++j) {
-            uint32_t lm = 0;
+        if (C <= 32) {
+            // compact the candidates (lane order, then element order) ...
+            int pos = cnt;
 #pragma unroll
-            for (int v = 0; v < NV; ++v)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) lm = max(lm, key[v][c]);
-            const uint32_t m = __reduce_max_sync(FULL_MASK, lm);
-            // lowest expert id in this lane whose key equals the maximum
-            int32_t cand = 0x7FFFFFFF;
-#pragma unroll
-            for (int v = NV - 1; v >= 0; --v)
-#pragma unroll
-                for (int c = 3; c >= 0; --c)
-                    if (key[v][c] == m) cand = base + 128 * v + c;
-            const int32_t gi = __reduce_min_sync(FULL_MASK, cand);
-            const int32_t rel = gi - base;  // equals 128*v + c only in the owning lane
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(FULL_MASK, pos, o);
+                if (lane >= o) pos += u;
+            }
+            pos -= cnt;
 #pragma unroll
             for (int v = 0; v < NV; ++v)
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    if (rel == 128 * v + c) key[v][c] = 0u;
-            if (lane == j) {
-                sel_key = m;
-                sel_idx = gi;
+                    if (key[v][c] >= tau) cand_sm[wib][pos++] = make_uint2(key[v][c], base + 128 * v + c);
+            __syncwarp();
+            // ... and rank each one by (key descending, id ascending)
+            uint2 me = make_uint2(0u, 0u);
+            if (lane < C) me = cand_sm[wib][lane];
+            int rank = 0;
+            for (int i = 0; i < C; ++i) {
+                const uint2 o = cand_sm[wib][i];
+                rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+            }
+            if (lane < C && rank < k) sel_sm[wib][rank] = me;
+            __syncwarp();
+            if (lane < k) {
+                sel_key = sel_sm[wib][lane].x;
+                sel_idx = int32_t(sel_sm[wib][lane].y);
+            }
+            __syncwarp();
+        } else {
+            // many equal logits: k exact rounds over every logit
+            for (int j = 0; j < k; ++j) {
+                uint32_t mx = 0;
+#pragma unroll
+                for (int v = 0; v < NV; ++v)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) mx = max(mx, key[v][c]);
+                const uint32_t m = __reduce_max_sync(FULL_MASK, mx);
+                // lowest expert id in this lane whose key equals the maximum
+                int32_t cand = 0x7FFFFFFF;
+#pragma unroll
+                for (int v = NV - 1; v >= 0; --v)
+#pragma unroll
+                    for (int c = 3; c >= 0; --c)
+                        if (key[v][c] == m) cand = base + 128 * v + c;
+                const int32_t gi = __reduce_min_sync(FULL_MASK, cand);
+                const int32_t rel = gi - base;  // equals 128*v + c only in the owning lane
+#pragma unroll
+                for (int v = 0; v < NV; ++v)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        if (rel == 128 * v + c) key[v][c] = 0u;
+                if (lane == j) {
+                    sel_key = m;
+                    sel_idx = gi;
+                }
             }
         }
 
@@ -123,10 +185,10 @@ cudaError_t launch_nv(const Geo &g, const float *logits, int32_t *idx, float *ga
     DevInfo di;
     if (dev_info(&di) != 0) return cudaErrorUnknown;
     const int64_t warps_needed = g.T;
-    int64_t blocks = (warps_needed + 7) / 8;
+    int64_t blocks = (warps_needed + ROUTE_WARPS - 1) / ROUTE_WARPS;
     const int64_t cap = int64_t(di.sms) * 8;  // 64 resident warps per SM
     if (blocks > cap) blocks = cap;
-    route_kernel<NV><<<unsigned(blocks), 256, 0, st>>>(logits, idx, gates, g.T, g.E, g.k);
+    route_kernel<NV><<<unsigned(blocks), ROUTE_WARPS * 32, 0, st>>>(logits, idx, gates, g.T, g.E, g.k);
     return cudaGetLastError();
 }
 
