@@ -55,6 +55,26 @@ def parse():
     return ap.parse_args()
 
 
+def rank_workload(base, rank: int):
+    """Each rank runs its own independent batch: same shape, seed offset by rank."""
+    return base.with_(seed=base.seed + rank)
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of per-rank timings (all ranks call it in the same order)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def throughput(units_per_rank_step: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job rate: units of all ranks over the slowest rank's time."""
+    return units_per_rank_step * steps * world / (ms / 1e3)
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -229,7 +249,7 @@ def main():
     base = synth.WORKLOADS[a.workload]
     if a.tokens:
         base = base.with_(T=a.tokens, seq_len=min(base.seq_len, a.tokens // base.R * base.R))
-    w = base.with_(seed=base.seed + rank)
+    w = rank_workload(base, rank)
     cfg = mp.Config.from_workload(w)
     b = mp.Buffers(cfg, device=dev)
     sizes = b.sizes
@@ -288,13 +308,8 @@ def main():
                  for j, n in enumerate(stages)}
     dc_stages = ["route", "assign", "pack", "bucket", "combine"]
     dc_ms = sum(sum(per_stage[n]) for n in dc_stages)  # over K steps
-    vals = torch.tensor([total_ms, dc_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, dc_ms = float(vals[0]), float(vals[1])
-
-    units = w.T * w.k * a.steps * world
-    value = units / (dc_ms / 1e3)
+    total_ms, dc_ms = max_over_ranks([total_ms, dc_ms], world, dev)
+    value = throughput(w.T * w.k, a.steps, world, dc_ms)
     ab = alg_bytes(w, st, sizes.C_s)
     b_alg = sum(ab[n] for n in dc_stages)
     peak, peak_kind = measured_peaks()
@@ -335,12 +350,10 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        ev = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(ev, op=dist.ReduceOp.MAX)
-        e2e = {"value": w.T * w.k * ke * world / (float(ev[0]) / 1e3), "unit": UNIT,
+        (e_ms,) = max_over_ranks([e0.elapsed_time(e1)], world, dev)
+        e2e = {"value": throughput(w.T * w.k, ke, world, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": float(ev[0]) / ke}
+               "ms_per_step": e_ms / ke}
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:

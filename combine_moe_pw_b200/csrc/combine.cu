@@ -17,7 +17,21 @@ namespace moe_pw {
 
 namespace {
 
-constexpr int U = 2;  // chunks per lane per iteration
+#ifndef MOE_PW_COMBINE_U
+#define MOE_PW_COMBINE_U 2
+#endif
+#ifndef MOE_PW_COMBINE_MINB
+#define MOE_PW_COMBINE_MINB 0  // 0: let the compiler pick the register budget
+#endif
+#ifndef MOE_PW_COMBINE_BLOCKS_PER_SM
+#define MOE_PW_COMBINE_BLOCKS_PER_SM 8
+#endif
+#if MOE_PW_COMBINE_MINB > 0
+#define MOE_PW_COMBINE_BOUNDS __launch_bounds__(256, MOE_PW_COMBINE_MINB)
+#else
+#define MOE_PW_COMBINE_BOUNDS __launch_bounds__(256)
+#endif
+constexpr int U = MOE_PW_COMBINE_U;  // chunks per lane per iteration
 
 __device__ __forceinline__ void fma_row(float (&acc)[8], float gj, const uint4 &v)
 {
@@ -32,7 +46,7 @@ __device__ __forceinline__ void fma_row(float (&acc)[8], float gj, const uint4 &
 }
 
 template <int KMAX>
-__global__ void __launch_bounds__(256) combine_kernel(const uint4 *__restrict__ ret_x,
+__global__ void MOE_PW_COMBINE_BOUNDS combine_kernel(const uint4 *__restrict__ ret_x,
                                                       const int32_t *__restrict__ ret_hdr,
                                                       const int32_t *__restrict__ slot_map,
                                                       const float *__restrict__ gates,
@@ -112,7 +126,8 @@ cudaError_t launch_k(const Geo &g, const uint16_t *ret_x, const int32_t *ret_hdr
     DevInfo di;
     if (dev_info(&di) != 0) return cudaErrorUnknown;
     int64_t blocks = (g.T + 7) / 8;
-    if (blocks > int64_t(di.sms) * 8) blocks = int64_t(di.sms) * 8;
+    if (blocks > int64_t(di.sms) * MOE_PW_COMBINE_BLOCKS_PER_SM)
+        blocks = int64_t(di.sms) * MOE_PW_COMBINE_BLOCKS_PER_SM;
     combine_kernel<KMAX><<<unsigned(blocks), 256, 0, st>>>(
         reinterpret_cast<const uint4 *>(ret_x), ret_hdr, slot_map, gates,
         reinterpret_cast<float4 *>(out), g.T, g.k, g.D / 8, g.n_slots, ctr);
