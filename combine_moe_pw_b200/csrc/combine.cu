@@ -6,6 +6,10 @@
 // not renormalised: "Marin 开始公开训练 535B 参数 MoE 模型", section 四 -- a
 // dropped assignment leaves the token to the shared experts.
 //
+// With gates == nullptr every gate is 1: fmaf(1, y, acc) is the exact sum,
+// which makes the same kernel the pack's backward (dx = sum of the slots'
+// gradient rows).
+//
 // One warp per token.  Lanes j < k read (slot, gate, ret_hdr) once and the
 // warp broadcasts them into registers; then each lane owns 16-byte chunks of
 // the row (8 bf16), issues the loads of all k rows for two chunks before
@@ -62,7 +66,7 @@ __global__ void MOE_PW_COMBINE_BOUNDS combine_kernel(const uint4 *__restrict__ r
         float my_gate = 0.0f;
         if (lane < k) {
             my_slot = slot_map[t * k + lane];
-            my_gate = gates[t * k + lane];
+            my_gate = gates ? gates[t * k + lane] : 1.0f;
             if (my_slot >= n_slots) {
                 set_error(ctr, MOE_PW_DEVERR_SLOT);
                 my_slot = -1;

@@ -55,6 +55,12 @@ cudaError_t launch_combine(const Geo &g, const uint16_t *ret_x, const int32_t *r
                            const int32_t *slot_map, const float *gates, float *out,
                            moe_pw_counters *ctr, cudaStream_t st);
 
+cudaError_t launch_combine_backward(const Geo &g, const float *dout, const uint16_t *ret_x,
+                                    const int32_t *ret_hdr, const int32_t *slot_map,
+                                    const int32_t *idx, const float *gates, uint16_t *d_ret,
+                                    float *dgates, float *dlogits, moe_pw_counters *ctr,
+                                    cudaStream_t st);
+
 // Workspace layout of the ranking pass.
 inline int64_t align256(int64_t b) { return (b + 255) & ~int64_t(255); }
 inline int64_t ws_counts_bytes(const Geo &g) { return align256(4 * int64_t(g.n_chunks) * g.NB); }

@@ -262,6 +262,43 @@ int moe_pw_combine(const moe_pw_config *cfg, const uint16_t *ret_x, const int32_
     return cuda_rc(launch_combine(g, ret_x, ret_hdr, slot_map, gates, out, counters, stream));
 }
 
+int moe_pw_combine_backward(const moe_pw_config *cfg, const float *dout, const uint16_t *ret_x,
+                            const int32_t *ret_hdr, const int32_t *slot_map, const int32_t *idx,
+                            const float *gates, uint16_t *d_ret, float *dgates, float *dlogits,
+                            moe_pw_counters *counters, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.T == 0 && g.n_slots == 0) return MOE_PW_OK;
+    if (!ret_hdr || !d_ret || !counters) return MOE_PW_EINVAL;
+    if (g.T > 0 && (!dout || !ret_x || !slot_map || !idx || !gates)) return MOE_PW_EINVAL;
+    if (!aligned(d_ret, 16) || !aligned(ret_hdr, 4) || !aligned(counters, 8) ||
+        (g.T > 0 && (!aligned(dout, 16) || !aligned(ret_x, 16) || !aligned(slot_map, 4) ||
+                     !aligned(idx, 4) || !aligned(gates, 4))) ||
+        (dgates && !aligned(dgates, 4)) || (dlogits && !aligned(dlogits, 4)))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_combine_backward(g, dout, ret_x, ret_hdr, slot_map, idx, gates, d_ret,
+                                           dgates, dlogits, counters, stream));
+}
+
+int moe_pw_dispatch_backward(const moe_pw_config *cfg, const uint16_t *d_pool,
+                             const int32_t *recv_row, const int32_t *slot_map, float *dx,
+                             moe_pw_counters *counters, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.T == 0) return MOE_PW_OK;
+    if (!d_pool || !recv_row || !slot_map || !dx || !counters) return MOE_PW_EINVAL;
+    if (!aligned(d_pool, 16) || !aligned(dx, 16) || !aligned(recv_row, 4) ||
+        !aligned(slot_map, 4) || !aligned(counters, 8))
+        return MOE_PW_EUNSUPPORTED;
+    // the combine kernel with unit gates; recv_row >= 0 marks the slots whose
+    // gradient rows are live (the others were zeroed by the expert backward)
+    return cuda_rc(launch_combine(g, d_pool, recv_row, slot_map, nullptr, dx, counters, stream));
+}
+
 int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
                  moe_pw_drop_stats *host_out, cudaStream_t stream)
 {

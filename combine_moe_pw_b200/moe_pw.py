@@ -73,6 +73,8 @@ SIGNATURES = {
     "moe_pw_dispatch": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_expert": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_combine": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_combine_backward": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_dispatch_backward": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_stats": [_CFG, _VP, ctypes.POINTER(moe_pw_drop_stats), _VP],
 }
 
@@ -222,6 +224,21 @@ def moe_pw_combine(cfg, ret_x, ret_hdr, slot_map, gates, out, counters, stream=N
         _ptr(counters), _stream(stream)))
 
 
+def moe_pw_combine_backward(cfg, dout, ret_x, ret_hdr, slot_map, idx, gates, d_ret, dgates,
+                            dlogits, counters, stream=None):
+    c = _cfg(cfg)
+    _check("moe_pw_combine_backward", load_library().moe_pw_combine_backward(
+        ctypes.byref(c), _ptr(dout), _ptr(ret_x), _ptr(ret_hdr), _ptr(slot_map), _ptr(idx),
+        _ptr(gates), _ptr(d_ret), _ptr(dgates), _ptr(dlogits), _ptr(counters), _stream(stream)))
+
+
+def moe_pw_dispatch_backward(cfg, d_pool, recv_row, slot_map, dx, counters, stream=None):
+    c = _cfg(cfg)
+    _check("moe_pw_dispatch_backward", load_library().moe_pw_dispatch_backward(
+        ctypes.byref(c), _ptr(d_pool), _ptr(recv_row), _ptr(slot_map), _ptr(dx), _ptr(counters),
+        _stream(stream)))
+
+
 def moe_pw_stats(cfg, counters, stream=None, raise_on_device_error: bool = True) -> moe_pw_drop_stats:
     c = _cfg(cfg)
     out = moe_pw_drop_stats()
@@ -296,6 +313,30 @@ class Buffers:
 
     def stats(self, stream=None, raise_on_device_error: bool = True) -> moe_pw_drop_stats:
         return moe_pw_stats(self.cfg, self.counters, stream, raise_on_device_error)
+
+    def alloc_backward(self):
+        """Gradient buffers: dout (input), d_ret / d_pool (gradient pools),
+        dgates, dlogits, dx."""
+        dev, T, E, k, D = self.out.device, self.cfg.T, self.cfg.E, self.cfg.k, self.cfg.D
+        n = self.sizes.n_slots
+        self.dout = torch.empty((T, D), dtype=torch.float32, device=dev)
+        self.d_ret = torch.empty((n, D), dtype=torch.int16, device=dev)
+        self.d_pool = torch.empty((n, D), dtype=torch.int16, device=dev)
+        self.d_pool_hdr = torch.empty((n,), dtype=torch.int32, device=dev)
+        self.dgates = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.dlogits = torch.empty((T, E), dtype=torch.float32, device=dev)
+        self.dx = torch.empty((T, D), dtype=torch.float32, device=dev)
+
+    def run_backward(self, stream=None):
+        """combine backward -> expert backward (the same scale op on the
+        gradient pool) -> pack backward."""
+        moe_pw_combine_backward(self.cfg, self.dout, self.ret_x, self.ret_hdr, self.slot_map,
+                                self.idx, self.gates, self.d_ret, self.dgates, self.dlogits,
+                                self.counters, stream)
+        moe_pw_expert(self.cfg, self.d_ret, self.pool_hdr, self.recv_row, self.scale,
+                      self.d_pool, self.d_pool_hdr, stream)
+        moe_pw_dispatch_backward(self.cfg, self.d_pool, self.recv_row, self.slot_map, self.dx,
+                                 self.counters, stream)
 
     def run_step(self, stream=None):
         """route -> dispatch (assign, pack, bucket) -> expert -> combine."""

@@ -101,6 +101,7 @@ def _load():
         lib.synth_logits.argtypes = [ctypes.c_int, i64, i32, i64, f64, u64, vp]
         lib.synth_x_bf16.argtypes = [i64, i32, u64, vp]
         lib.synth_scales.argtypes = [i32, f64, f64, u64, vp]
+        lib.synth_dout_f32.argtypes = [i64, i32, u64, vp]
         lib.synth_u64.argtypes = [u64, u64, u64]
         lib.synth_u64.restype = u64
         lib.synth_normal.argtypes = [u64, u64, u64]
@@ -130,6 +131,15 @@ def x_bf16(w: Workload, out: np.ndarray | None = None) -> np.ndarray:
     assert out.dtype == np.uint16 and out.shape == (w.T, w.D)
     if _load().synth_x_bf16(w.T, w.D, w.seed, _ptr(out)) != 0:
         raise ValueError(f"synth_x_bf16 failed for {w}")
+    return out
+
+
+def dout(w: Workload, out: np.ndarray | None = None) -> np.ndarray:
+    """Upstream gradient dL/dout for the backward, fp32 [T, D] ~ N(0, 1)."""
+    out = np.empty((w.T, w.D), np.float32) if out is None else out
+    assert out.dtype == np.float32 and out.shape == (w.T, w.D)
+    if _load().synth_dout_f32(w.T, w.D, w.seed, _ptr(out)) != 0:
+        raise ValueError("synth_dout_f32 failed")
     return out
 
 

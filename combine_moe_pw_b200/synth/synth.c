@@ -60,7 +60,7 @@ static inline uint16_t f32_bits_to_bf16(float f)
 }
 
 /* stream ids */
-enum { ST_LOGIT = 1, ST_SEQBIAS = 2, ST_X = 3, ST_SCALE = 4, ST_PERM = 5 };
+enum { ST_LOGIT = 1, ST_SEQBIAS = 2, ST_X = 3, ST_SCALE = 4, ST_PERM = 5, ST_DOUT = 6 };
 
 /*
  * Router logits, row-major [T, E] fp32.
@@ -117,6 +117,17 @@ int synth_x_bf16(int64_t T, int32_t D, uint64_t seed, uint16_t *out)
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i)
         out[i] = f32_bits_to_bf16((float)draw_normal(kx, (uint64_t)i));
+    return 0;
+}
+
+/* Upstream gradient dL/dout, row-major [T, D] fp32: N(0,1) rounded to fp32. */
+int synth_dout_f32(int64_t T, int32_t D, uint64_t seed, float *out)
+{
+    if (T < 0 || D <= 0 || !out) return -1;
+    const uint64_t kd = stream_key(seed, ST_DOUT);
+    const int64_t n = T * (int64_t)D;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = (float)draw_normal(kd, (uint64_t)i);
     return 0;
 }
 

@@ -273,6 +273,37 @@ int moe_pw_combine(const moe_pw_config *cfg, const uint16_t *ret_x, const int32_
                    moe_pw_counters *counters, cudaStream_t stream);
 
 /*
+ * Backward of the combine.  The pages train this model ("Marin 开始公开训练 535B
+ * 参数 MoE 模型", section 一) but give no backward; this is the derivative of the
+ * forward definitions above.  Given dout = dL/dout (f32 [T, D]):
+ *   d_ret (bf16 [n_slots, D], the gradient pool, same slot ids as ret_x):
+ *     for every surviving (t, j) (slot >= 0, ret_hdr[slot] >= 0)
+ *     d_ret[slot] = bf16_rn(g_j * dout[t]) with the product in fp32; every
+ *     other slot is zeroed (a fixed pool, like the forward's);
+ *   dgates (f32 [T, k], may be NULL): <dout[t], y_j> for surviving (t, j),
+ *     else 0 (fp32, each lane's share in chunk order, then a fixed xor tree);
+ *   dlogits (f32 [T, E], may be NULL): the top-k softmax backward,
+ *     dlogits[t][idx[t][j]] = g_j * (dgate_j - sum_i g_i dgate_i), all other
+ *     logits 0 (top-k selection is piecewise constant in the logits).
+ * The stand-in expert op's backward is moe_pw_expert applied to d_ret (the
+ * same scale op, its bf16 rounding passed straight through), giving d_pool.
+ */
+int moe_pw_combine_backward(const moe_pw_config *cfg, const float *dout, const uint16_t *ret_x,
+                            const int32_t *ret_hdr, const int32_t *slot_map, const int32_t *idx,
+                            const float *gates, uint16_t *d_ret, float *dgates, float *dlogits,
+                            moe_pw_counters *counters, cudaStream_t stream);
+
+/*
+ * Backward of the pack: x[t] was copied into the slot of each (t, j) the
+ * sender kept, so dx[t] = sum over those j of d_pool[slot] (f32 [T, D], j
+ * ascending, exact fp32 adds from +0).  Slots the receiver dropped
+ * (recv_row < 0) carry zero gradient and are skipped.
+ */
+int moe_pw_dispatch_backward(const moe_pw_config *cfg, const uint16_t *d_pool,
+                             const int32_t *recv_row, const int32_t *slot_map, float *dx,
+                             moe_pw_counters *counters, cudaStream_t stream);
+
+/*
  * Drop statistics (section 二: the two kinds of drop are reported apart).
  * Copies *counters (device) to *host_out (host memory) and synchronises the
  * stream.  Returns MOE_PW_EDEVICE when a kernel flagged a violation (the

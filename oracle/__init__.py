@@ -105,6 +105,8 @@ def _configure(lib):
     lib.orc_combine.argtypes = [gp, vp, vp, vp, vp, vp]
     lib.orc_combine_tokens.argtypes = [gp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp]
     lib.orc_combine_mag.argtypes = [gp, vp, vp, vp, vp, vp]
+    lib.orc_combine_backward.argtypes = [gp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.orc_dispatch_backward.argtypes = [gp, vp, vp, vp, vp]
     lib.orc_bf16_round.argtypes = [vp, vp, i64]
     lib.orc_expert_product.argtypes = [vp, vp, vp, i64]
     return lib
@@ -293,6 +295,45 @@ def run_headers(w, logits: np.ndarray) -> dict:
         r["arrivals"] = r["bucket_cnt"] = r["row_cnt"]
     r["kept"] = int(np.asarray(r["bucket_cnt"], np.int64).sum())
     return r
+
+
+def combine_backward(g: Geom, dout, ret_x, ret_hdr, slot_map, idx, gates):
+    """(d_ret bf16 bits [n_slots, D], dgate f64 [T, k], dlogits f64 [T, E])."""
+    n = ret_x.shape[0]
+    d_ret = np.empty((n, g.D), np.uint16)
+    dgate = np.empty((g.T, g.k), np.float64)
+    dlogits = np.empty((g.T, g.E), np.float64)
+    gc = g.c()
+    _load().orc_combine_backward(ctypes.byref(gc), n, _p(_c(dout, np.float32)),
+                                 _p(_c(ret_x, np.uint16)), _p(_c(ret_hdr, np.int32)),
+                                 _p(_c(slot_map, np.int32)), _p(_c(idx, np.int32)),
+                                 _p(_c(gates, np.float64)), _p(d_ret), _p(dgate), _p(dlogits))
+    return d_ret, dgate, dlogits
+
+
+def dispatch_backward(g: Geom, d_pool, recv_row, slot_map):
+    """dx f64 [T, D]."""
+    dx = np.empty((g.T, g.D), np.float64)
+    gc = g.c()
+    _load().orc_dispatch_backward(ctypes.byref(gc), _p(_c(d_pool, np.uint16)),
+                                  _p(_c(recv_row, np.int32)), _p(_c(slot_map, np.int32)), _p(dx))
+    return dx
+
+
+def run_backward(w, r: dict, dout: np.ndarray, scale: np.ndarray) -> dict:
+    """Backward of ``run``'s forward for a given dL/dout: combine backward,
+    the expert op's backward (the same scale op on the gradient pool, the
+    bf16 rounding passed straight through) and the pack transpose."""
+    g = r["geom"]
+    b = {}
+    b["d_ret"], b["dgate"], b["dlogits"] = combine_backward(
+        g, dout, r["ret_x"], r["ret_hdr"], r["slot_map"], r["idx"], r["gates"])
+    if w.mode == 0:
+        b["d_pool"], _ = expert_pooled(g, b["d_ret"], r["bucket_slot"], r["bucket_cnt"], scale)
+    else:
+        b["d_pool"], _ = expert_ragged(g, b["d_ret"], r["pool_hdr"], scale)
+    b["dx"] = dispatch_backward(g, b["d_pool"], r["recv_row"], r["slot_map"])
+    return b
 
 
 def bf16_round(a: np.ndarray) -> np.ndarray:

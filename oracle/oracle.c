@@ -474,3 +474,76 @@ void orc_expert_product(const float *s, const uint16_t *x, uint16_t *y, int64_t 
 {
     for (int64_t i = 0; i < n; ++i) y[i] = f32_to_bf16_rne(s[i] * bf16_to_f32(x[i]));
 }
+
+/* ------------------------------------------------------------------------ */
+/* Backward of combine and dispatch.                                         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The pages train this model ("Marin 开始公开训练 535B 参数 MoE 模型", section 一),
+ * so the path also needs its gradient.  The pages describe no backward; these
+ * are the derivatives of the forward definitions above (READING: gradients
+ * travel in the same fixed pools, bf16 like the forward payload).
+ *
+ * Given dout = dL/dout [T, D] (fp32):
+ *   surviving (t, j) (slot >= 0 and ret_hdr[slot] >= 0):
+ *     d_ret[slot] = bf16(g_j * dout[t])   product in fp32 (it decides a bf16
+ *                                         code), gate rounded to fp32 first
+ *     dgate[t][j] = <dout[t], y_j>        y_j = returned row, in double
+ *   every other slot of d_ret: zero (a fixed pool, like the forward)
+ *   dgate of a dropped (t, j): 0
+ *   softmax over the chosen logits: dl_j = g_j * (dgate_j - sum_i g_i dgate_i),
+ *   dlogits[t][idx[t][j]] = dl_j, every other logit 0 (top-k is piecewise
+ *   constant in the logits).
+ */
+void orc_combine_backward(const orc_geom *g, int64_t n_slots, const float *dout,
+                          const uint16_t *ret_x, const int32_t *ret_hdr, const int32_t *slot_map,
+                          const int32_t *idx, const double *gates, uint16_t *d_ret,
+                          double *dgate, double *dlogits)
+{
+    const int64_t D = g->D;
+    const int32_t k = g->k, E = g->E;
+    for (int64_t q = 0; q < n_slots * D; ++q) d_ret[q] = 0;
+    for (int64_t t = 0; t < g->T; ++t) {
+        const float *dt = dout + t * D;
+        double *dl = dlogits + t * E;
+        for (int32_t e = 0; e < E; ++e) dl[e] = 0.0;
+        double weighted = 0.0;
+        for (int32_t j = 0; j < k; ++j) {
+            const int64_t slot = slot_map[t * k + j];
+            double dg = 0.0;
+            if (slot >= 0 && ret_hdr[slot] >= 0) {
+                const float gj = (float)gates[t * k + j];
+                for (int64_t i = 0; i < D; ++i) {
+                    d_ret[slot * D + i] = f32_to_bf16_rne(gj * dt[i]);
+                    dg += (double)dt[i] * (double)bf16_to_f32(ret_x[slot * D + i]);
+                }
+            }
+            dgate[t * k + j] = dg;
+            weighted += gates[t * k + j] * dg;
+        }
+        for (int32_t j = 0; j < k; ++j)
+            dl[idx[t * k + j]] = gates[t * k + j] * (dgate[t * k + j] - weighted);
+    }
+}
+
+/*
+ * Pack transpose: x[t] was copied into the slot of every (t, j) the sender
+ * kept, so dx[t] = sum over those j of d_pool[slot], in double.  Slots the
+ * receiver dropped carry a zero gradient (the expert op's backward writes
+ * zeros there), so they are left out.
+ */
+void orc_dispatch_backward(const orc_geom *g, const uint16_t *d_pool, const int32_t *recv_row,
+                           const int32_t *slot_map, double *dx)
+{
+    const int64_t D = g->D;
+    for (int64_t t = 0; t < g->T; ++t) {
+        double *o = dx + t * D;
+        for (int64_t i = 0; i < D; ++i) o[i] = 0.0;
+        for (int32_t j = 0; j < g->k; ++j) {
+            const int64_t slot = slot_map[t * g->k + j];
+            if (slot < 0 || recv_row[slot] < 0) continue;
+            for (int64_t i = 0; i < D; ++i) o[i] += (double)bf16_to_f32(d_pool[slot * D + i]);
+        }
+    }
+}

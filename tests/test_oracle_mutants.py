@@ -13,6 +13,7 @@ import pytest
 import oracle
 from combine_moe_pw_b200 import synth
 
+import test_oracle_backward as tb
 import test_oracle_combine as tc
 import test_oracle_dispatch as td
 import test_oracle_route as tr
@@ -41,7 +42,23 @@ def _tiny_run():
     return oracle.run(w, lg, x, s, with_mag=True)
 
 
+def _bw_case():
+    w, lg, x, s = _tiny()
+    r = oracle.run(w, lg, x, s)
+    dout = synth.dout(w)
+    return w, lg, x, s, r, dout, oracle.run_backward(w, r, dout, s)
+
+
 MUTANTS = [
+    ("softmax_backward_sign", "gates[t * k + j] * (dgate[t * k + j] - weighted)",
+     "gates[t * k + j] * (weighted - dgate[t * k + j])",
+     lambda: tb.test_backward_with_exact_rows(_bw_case())),
+    ("grad_row_without_gate", "d_ret[slot * D + i] = f32_to_bf16_rne(gj * dt[i]);",
+     "d_ret[slot * D + i] = f32_to_bf16_rne(dt[i]);",
+     lambda: tb.test_backward_matches_autograd(_bw_case())),
+    ("dispatch_backward_skips_last_choice", "for (int32_t j = 0; j < g->k; ++j) {\n            const int64_t slot = slot_map[t * g->k + j];\n            if (slot < 0 || recv_row[slot] < 0) continue;",
+     "for (int32_t j = 0; j + 1 < g->k; ++j) {\n            const int64_t slot = slot_map[t * g->k + j];\n            if (slot < 0 || recv_row[slot] < 0) continue;",
+     lambda: tb.test_backward_matches_autograd(_bw_case())),
     ("ties_to_higher_index", "l[e] > l[best]", "l[e] >= l[best]",
      lambda: tr.test_topk_matches_full_sort(48, 8)),
     ("gate_sum_skips_first", "den += ex[j];", "if (j) den += ex[j];",
