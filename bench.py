@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
     ap.add_argument("--cpu-sample-sources", type=int, default=16)
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward timing (reported apart from the metric)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the batch's token count (profiling a smaller case)")
     return ap.parse_args()
@@ -81,6 +83,18 @@ def measured_peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def backward_bytes(w, stats, C_s):
+    """Algorithmic bytes of the backward stages (K = rows the receiver kept)."""
+    T, E, k, D = w.T, w.E, w.k, w.D
+    S = w.R * w.R * w.W * C_s if w.mode == 0 else T * k
+    K = stats.kept
+    combine_bwd = (4 * T * D + 2 * D * K + 2 * D * K + 2 * D * (S - K) + 4 * S + 12 * T * k
+                   + 4 * T * E + 4 * T * k)
+    expert_bwd = 2 * D * K + 8 * S + S * (2 * D + 4)
+    dispatch_bwd = 2 * D * K + 4 * T * D + 4 * T * k + 4 * K
+    return {"combine_bwd": combine_bwd, "expert_bwd": expert_bwd, "dispatch_bwd": dispatch_bwd}
 
 
 def alg_bytes(w, stats, C_s):
@@ -320,6 +334,51 @@ def main():
     achieved = ab[dom] / (stage_ms[dom] / 1e3) / 1e9
     traffic = traffic_from_profiles(kname + "_" + a.workload)
 
+    # backward (gradient of dispatch/combine), timed in its own loop
+    bwd = None
+    if not a.no_backward:
+        b.alloc_backward()
+        b.dout.copy_(torch.from_numpy(synth.dout(w)))
+        names = ["combine_bwd", "expert_bwd", "dispatch_bwd"]
+
+        def bstep(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            mp.moe_pw_combine_backward(cfg, b.dout, b.ret_x, b.ret_hdr, b.slot_map, b.idx,
+                                       b.gates, b.d_ret, b.dgates, b.dlogits, b.counters, stream)
+            if ev is not None:
+                ev[1].record(stream)
+            mp.moe_pw_expert(cfg, b.d_ret, b.pool_hdr, b.recv_row, b.scale, b.d_pool,
+                             b.d_pool_hdr, stream)
+            if ev is not None:
+                ev[2].record(stream)
+            mp.moe_pw_dispatch_backward(cfg, b.d_pool, b.recv_row, b.slot_map, b.dx, b.counters,
+                                        stream)
+            if ev is not None:
+                ev[3].record(stream)
+
+        for _ in range(3):
+            bstep()
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(a.steps):
+            bstep(bev[i])
+        torch.cuda.synchronize(dev)
+        bms = {n: statistics.mean(bev[i][j].elapsed_time(bev[i][j + 1]) for i in range(a.steps))
+               for j, n in enumerate(names)}
+        bb = backward_bytes(w, st, sizes.C_s)
+        tot_ms = max_over_ranks([sum(bms.values())], world, dev)[0]
+        bwd = {"ms_per_step": tot_ms, "stage_ms": bms,
+               "value": throughput(w.T * w.k, 1, world, tot_ms), "unit": UNIT,
+               "hbm_gbs": sum(bb.values()) / (tot_ms / 1e3) / 1e9,
+               "hbm_frac_of_peak": sum(bb.values()) / (tot_ms / 1e3) / 1e9 / measured_peaks()[0],
+               "alg_bytes_per_step": sum(bb.values()),
+               "stage_gbs": {n: bb[n] / (bms[n] / 1e3) / 1e9 for n in names}}
+        del b.d_ret, b.d_pool
+        torch.cuda.empty_cache()
+
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
     if not a.no_e2e:
@@ -383,6 +442,7 @@ def main():
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "alg_bytes_per_launch": ab[dom], "peak_kind": peak_kind},
             "gpu_launches": launches_per_step * a.steps,
+            "backward": bwd,
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,

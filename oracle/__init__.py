@@ -107,6 +107,7 @@ def _configure(lib):
     lib.orc_combine_mag.argtypes = [gp, vp, vp, vp, vp, vp]
     lib.orc_combine_backward.argtypes = [gp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.orc_dispatch_backward.argtypes = [gp, vp, vp, vp, vp]
+    lib.orc_backward_tokens.argtypes = [gp, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp]
     lib.orc_bf16_round.argtypes = [vp, vp, i64]
     lib.orc_expert_product.argtypes = [vp, vp, vp, i64]
     return lib
@@ -318,6 +319,24 @@ def dispatch_backward(g: Geom, d_pool, recv_row, slot_map):
     _load().orc_dispatch_backward(ctypes.byref(gc), _p(_c(d_pool, np.uint16)),
                                   _p(_c(recv_row, np.int32)), _p(_c(slot_map, np.int32)), _p(dx))
     return dx
+
+
+def backward_tokens(g: Geom, x, idx, gates, slot_map, recv_row, scale, dout, tokens):
+    """Per-token backward (see orc_backward_tokens): d_ret rows [n, k, D] bf16
+    bits, dgate [n, k], dlogits [n, E], dx [n, D]."""
+    tokens = _c(tokens, np.int64)
+    n = tokens.size
+    d_ret = np.empty((n, g.k, g.D), np.uint16)
+    dgate = np.empty((n, g.k), np.float64)
+    dlogits = np.empty((n, g.E), np.float64)
+    dx = np.empty((n, g.D), np.float64)
+    gc = g.c()
+    _load().orc_backward_tokens(ctypes.byref(gc), _p(_c(x, np.uint16)), _p(_c(idx, np.int32)),
+                                _p(_c(gates, np.float64)), _p(_c(slot_map, np.int32)),
+                                _p(_c(recv_row, np.int32)), _p(_c(scale, np.float32)),
+                                _p(_c(dout, np.float32)), _p(tokens), n, _p(d_ret), _p(dgate),
+                                _p(dlogits), _p(dx))
+    return d_ret, dgate, dlogits, dx
 
 
 def run_backward(w, r: dict, dout: np.ndarray, scale: np.ndarray) -> dict:

@@ -547,3 +547,55 @@ void orc_dispatch_backward(const orc_geom *g, const uint16_t *d_pool, const int3
         }
     }
 }
+
+/*
+ * The whole backward for a list of tokens only (the same definitions,
+ * written per token for batches whose pools are too large for the host):
+ * for each listed token t and each j it survived with (slot >= 0 and
+ * recv_row[slot] >= 0), y_j = bf16(s_e * x[t]) and
+ *   d_ret row  = bf16(g_j * dout[t])            (fp32 product, gate in fp32)
+ *   dgate_j    = <dout[t], y_j>                  (double)
+ *   d_pool row = bf16(s_e * d_ret row)           (expert op backward)
+ *   dx[t]      = sum_j d_pool row                (double)
+ * and dlogits row t as in orc_combine_backward.  Outputs are per listed token:
+ * d_ret_rows [n, k, D] (zero for dropped j), dgate [n, k], dlogits [n, E],
+ * dx [n, D].
+ */
+void orc_backward_tokens(const orc_geom *g, const uint16_t *x, const int32_t *idx,
+                         const double *gates, const int32_t *slot_map, const int32_t *recv_row,
+                         const float *scale, const float *dout, const int64_t *tokens,
+                         int64_t n_tokens, uint16_t *d_ret_rows, double *dgate, double *dlogits,
+                         double *dx)
+{
+    const int64_t D = g->D;
+    const int32_t k = g->k, E = g->E;
+    for (int64_t n = 0; n < n_tokens; ++n) {
+        const int64_t t = tokens[n];
+        const float *dt = dout + t * D;
+        double *o = dx + n * D, *dl = dlogits + n * E;
+        for (int64_t i = 0; i < D; ++i) o[i] = 0.0;
+        for (int32_t e = 0; e < E; ++e) dl[e] = 0.0;
+        double weighted = 0.0;
+        for (int32_t j = 0; j < k; ++j) {
+            uint16_t *gr = d_ret_rows + (n * k + j) * D;
+            const int64_t slot = slot_map[t * k + j];
+            double dg = 0.0;
+            if (slot >= 0 && recv_row[slot] >= 0) {
+                const int32_t e = idx[t * k + j];
+                const float gj = (float)gates[t * k + j];
+                for (int64_t i = 0; i < D; ++i) {
+                    const float y = bf16_to_f32(f32_to_bf16_rne(scale[e] * bf16_to_f32(x[t * D + i])));
+                    dg += (double)dt[i] * (double)y;
+                    gr[i] = f32_to_bf16_rne(gj * dt[i]);
+                    o[i] += (double)bf16_to_f32(f32_to_bf16_rne(scale[e] * bf16_to_f32(gr[i])));
+                }
+            } else {
+                for (int64_t i = 0; i < D; ++i) gr[i] = 0;
+            }
+            dgate[n * k + j] = dg;
+            weighted += gates[t * k + j] * dg;
+        }
+        for (int32_t j = 0; j < k; ++j)
+            dl[idx[t * k + j]] = gates[t * k + j] * (dgate[n * k + j] - weighted);
+    }
+}

@@ -120,3 +120,55 @@ def test_backward_deterministic():
     b2, *_ = run_both(w)
     for n in ["d_ret", "dgates", "dlogits", "d_pool", "dx"]:
         assert torch.equal(getattr(b1, n), getattr(b2, n)), n
+
+
+@pytest.mark.parametrize("name", ["rack", "ragged"])
+def test_backward_full_size_sampled(name):
+    """The pages' shapes in the bench's launch configuration; the oracle's
+    integer path in full, the backward on sampled tokens."""
+    w = synth.WORKLOADS[name]
+    lg, x, s, dout = synth.logits(w), synth.x_bf16(w), synth.scales(w), synth.dout(w)
+    b = mp.Buffers(mp.Config.from_workload(w))
+    b.logits.copy_(torch.from_numpy(lg))
+    b.x.copy_(torch.from_numpy(x.view(np.int16)))
+    b.scale.copy_(torch.from_numpy(s))
+    b.run_step()
+    b.alloc_backward()
+    b.dout.copy_(torch.from_numpy(dout))
+    b.run_backward()
+    assert b.stats(raise_on_device_error=False).error == 0
+    r = oracle.run_headers(w, lg)
+    rng = np.random.default_rng(3)
+    toks = np.unique(np.concatenate([rng.integers(0, w.T, 512), [0, w.T - 1]]))
+    d_ret, dgate, dlog, dx = oracle.backward_tokens(r["geom"], x, r["idx"], r["gates"],
+                                                    r["slot_map"], r["recv_row"], s, dout, toks)
+    tt = torch.from_numpy(toks).cuda()
+    sm = r["slot_map"][toks]
+    live = (sm >= 0) & (r["recv_row"][np.where(sm >= 0, sm, 0)] >= 0)
+    # y rows and magnitudes for the tolerances
+    e = r["idx"][toks]
+    y = _f32(oracle.expert_product(np.repeat(s[e].reshape(-1, 1), w.D, axis=1),
+                                   np.repeat(x[toks], w.k, axis=0))).reshape(toks.size, w.k, w.D)
+    M = (np.abs(dout[toks].astype(np.float64))[:, None, :] * np.abs(y)).sum(axis=2) * live
+    g = r["gates"][toks]
+    dg = b.dgates[tt].cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(dg - dgate) <= 1e-5 * M + 1e-30)
+    dl = b.dlogits[tt].cpu().numpy().astype(np.float64)
+    ii = e.astype(np.int64)
+    tol = 2e-5 * g * (M + (g * M).sum(axis=1, keepdims=True)) + 1e-30
+    assert np.all(np.abs(np.take_along_axis(dl, ii, 1) - np.take_along_axis(dlog, ii, 1)) <= tol)
+    off = np.ones_like(dl, bool)
+    np.put_along_axis(off, ii, False, axis=1)
+    assert not dl[off].any()
+    slots = torch.from_numpy(np.where(live, sm, 0).reshape(-1).astype(np.int64)).cuda()
+    got = _f32(b.d_ret.index_select(0, slots).cpu().numpy().view(np.uint16)).reshape(
+        toks.size, w.k, w.D)
+    ref = _f32(d_ret)
+    assert np.all(np.abs(got - ref)[live] <= _ulp_bf16(ref)[live])
+    gdx = b.dx[tt].cpu().numpy().astype(np.float64)
+    mag = (np.abs(ref) * s[e][:, :, None] * live[:, :, None]).sum(axis=1) * (1 + 2.0 ** -7)
+    err = np.abs(gdx - dx)
+    assert np.all(err <= 2.0 ** -7 * mag + 1e-30)
+    assert (err > 1e-6 * mag + 1e-30).mean() < 1e-3
+    del b
+    torch.cuda.empty_cache()

@@ -120,3 +120,20 @@ def test_ragged_backward_equals_unbounded_pooled():
     np.testing.assert_array_equal(bp["dx"], br["dx"])
     np.testing.assert_array_equal(bp["dlogits"], br["dlogits"])
     np.testing.assert_array_equal(bp["dgate"], br["dgate"])
+
+
+def test_backward_tokens_equals_full_backward(case):
+    w, lg, x, s, r, dout, b = case
+    toks = np.array([0, 3, 255, 256, 1500, 2047])
+    d_ret, dgate, dlogits, dx = oracle.backward_tokens(r["geom"], x, r["idx"], r["gates"],
+                                                       r["slot_map"], r["recv_row"], s, dout, toks)
+    np.testing.assert_array_equal(dgate, b["dgate"][toks])
+    np.testing.assert_array_equal(dlogits, b["dlogits"][toks])
+    np.testing.assert_array_equal(dx, b["dx"][toks])
+    sm = r["slot_map"][toks]
+    for n in range(toks.size):
+        for j in range(w.k):
+            if sm[n, j] >= 0 and r["recv_row"][sm[n, j]] >= 0:
+                np.testing.assert_array_equal(d_ret[n, j], b["d_ret"][sm[n, j]])
+            else:
+                assert not d_ret[n, j].any()
