@@ -61,6 +61,11 @@ cudaError_t launch_combine_backward(const Geo &g, const float *dout, const uint1
                                     float *dgates, float *dlogits, moe_pw_counters *ctr,
                                     cudaStream_t st);
 
+cudaError_t launch_gemm(const uint16_t *A, const uint16_t *Bt, int64_t M, int32_t N, int32_t K,
+                        int32_t mode, uint16_t *C, int64_t ldc, const int32_t *slot_map,
+                        const int32_t *idx, int32_t topk, uint16_t *pool_x, int32_t *pool_hdr,
+                        int64_t n_slots, moe_pw_counters *ctr, cudaStream_t st);
+
 // Workspace layout of the ranking pass.
 inline int64_t align256(int64_t b) { return (b + 255) & ~int64_t(255); }
 inline int64_t ws_counts_bytes(const Geo &g) { return align256(4 * int64_t(g.n_chunks) * g.NB); }
@@ -95,6 +100,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
                  "r"(bytes)
                  : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)

@@ -299,6 +299,48 @@ int moe_pw_dispatch_backward(const moe_pw_config *cfg, const uint16_t *d_pool,
     return cuda_rc(launch_combine(g, d_pool, recv_row, slot_map, nullptr, dx, counters, stream));
 }
 
+int moe_pw_project(const uint16_t *A, const uint16_t *Bt, uint16_t *C, int64_t M, int32_t N,
+                   int32_t K, moe_pw_counters *counters, cudaStream_t stream)
+{
+    if (M < 0 || N < 0 || K < 1 || M > MAX_INT32) return MOE_PW_EINVAL;
+    if (M == 0 || N == 0) return MOE_PW_OK;
+    if (!A || !Bt || !C || !counters) return MOE_PW_EINVAL;
+    if (K % 8 != 0 || N % 8 != 0) return MOE_PW_EUNSUPPORTED;
+    if (!aligned(A, 16) || !aligned(Bt, 16) || !aligned(C, 16) || !aligned(counters, 8))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_gemm(A, Bt, M, N, K, 0, C, N, nullptr, nullptr, 0, nullptr, nullptr, 0,
+                               counters, stream));
+}
+
+int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint16_t *w_down_t,
+                        int32_t model_width, const int32_t *idx, const int32_t *slot_map,
+                        const int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr,
+                        moe_pw_counters *counters, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (model_width < 8 || model_width % 8 != 0) return MOE_PW_EUNSUPPORTED;
+    if (g.n_slots == 0) return MOE_PW_OK;
+    if (!h || !w_down_t || !idx || !slot_map || !occ || !pool_x || !pool_hdr || !counters)
+        return MOE_PW_EINVAL;
+    if (!aligned(h, 16) || !aligned(w_down_t, 16) || !aligned(pool_x, 16) || !aligned(idx, 4) ||
+        !aligned(slot_map, 4) || !aligned(occ, 4) || !aligned(pool_hdr, 4) ||
+        !aligned(counters, 8))
+        return MOE_PW_EUNSUPPORTED;
+    // rows of the kept slots straight from the GEMM epilogue ...
+    cudaError_t e = launch_gemm(h, w_down_t, g.T, g.D, model_width, 1, nullptr, 0, slot_map, idx,
+                                g.k, pool_x, pool_hdr, g.n_slots, counters, stream);
+    if (e != cudaSuccess) return MOE_PW_ECUDA;
+    // ... and the empty pool tails zero-filled by the pack kernel's second phase
+    if (g.mode == MOE_PW_POOLED) {
+        Geo tails = g;
+        tails.T = 0;
+        e = launch_pack(tails, nullptr, idx, slot_map, occ, pool_x, pool_hdr, counters, stream);
+    }
+    return cuda_rc(e);
+}
+
 int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
                  moe_pw_drop_stats *host_out, cudaStream_t stream)
 {

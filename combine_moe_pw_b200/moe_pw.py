@@ -75,6 +75,8 @@ SIGNATURES = {
     "moe_pw_combine": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_combine_backward": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_dispatch_backward": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_project": [_VP, _VP, _VP, _I64, ctypes.c_int32, ctypes.c_int32, _VP, _VP],
+    "moe_pw_project_pack": [_CFG, _VP, _VP, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_stats": [_CFG, _VP, ctypes.POINTER(moe_pw_drop_stats), _VP],
 }
 
@@ -237,6 +239,21 @@ def moe_pw_dispatch_backward(cfg, d_pool, recv_row, slot_map, dx, counters, stre
     _check("moe_pw_dispatch_backward", load_library().moe_pw_dispatch_backward(
         ctypes.byref(c), _ptr(d_pool), _ptr(recv_row), _ptr(slot_map), _ptr(dx), _ptr(counters),
         _stream(stream)))
+
+
+def moe_pw_project(A, Bt, C, M: int, N: int, K: int, counters, stream=None):
+    """C = bf16(A @ Bt^T) on the tensor cores (bf16 operands, fp32 accumulation)."""
+    _check("moe_pw_project", load_library().moe_pw_project(
+        _ptr(A), _ptr(Bt), _ptr(C), M, N, K, _ptr(counters), _stream(stream)))
+
+
+def moe_pw_project_pack(cfg, h, w_down_t, model_width: int, idx, slot_map, occ, pool_x, pool_hdr,
+                        counters, stream=None):
+    """Down-projection fused with the pack (see include/moe_pw.h)."""
+    c = _cfg(cfg)
+    _check("moe_pw_project_pack", load_library().moe_pw_project_pack(
+        ctypes.byref(c), _ptr(h), _ptr(w_down_t), model_width, _ptr(idx), _ptr(slot_map),
+        _ptr(occ), _ptr(pool_x), _ptr(pool_hdr), _ptr(counters), _stream(stream)))
 
 
 def moe_pw_stats(cfg, counters, stream=None, raise_on_device_error: bool = True) -> moe_pw_drop_stats:

@@ -102,6 +102,7 @@ def _load():
         lib.synth_x_bf16.argtypes = [i64, i32, u64, vp]
         lib.synth_scales.argtypes = [i32, f64, f64, u64, vp]
         lib.synth_dout_f32.argtypes = [i64, i32, u64, vp]
+        lib.synth_matrix_bf16.argtypes = [i64, i64, f64, u64, u64, vp]
         lib.synth_u64.argtypes = [u64, u64, u64]
         lib.synth_u64.restype = u64
         lib.synth_normal.argtypes = [u64, u64, u64]
@@ -141,6 +142,30 @@ def dout(w: Workload, out: np.ndarray | None = None) -> np.ndarray:
     if _load().synth_dout_f32(w.T, w.D, w.seed, _ptr(out)) != 0:
         raise ValueError("synth_dout_f32 failed")
     return out
+
+
+# named matrices for the latent projections (stream ids >= 16)
+STREAM_H, STREAM_W_DOWN, STREAM_W_UP = 16, 17, 18
+MODEL_WIDTH = 6144  # model state width of the pages' layer (latent = half of it)
+
+
+def matrix_bf16(rows: int, cols: int, std: float, stream: int, seed: int = 0) -> np.ndarray:
+    """bf16 bits [rows, cols] ~ N(0, std^2) from a named stream."""
+    out = np.empty((rows, cols), np.uint16)
+    if _load().synth_matrix_bf16(rows, cols, std, seed, stream, _ptr(out)) != 0:
+        raise ValueError("synth_matrix_bf16 failed")
+    return out
+
+
+def projection_inputs(w: Workload, model_width: int = MODEL_WIDTH):
+    """Model-width activations h [T, Dm] ~ N(0,1) and random-init projection
+    weights, both stored K-major for the GEMM: w_down_t [D, Dm] (h @ w_down_t^T
+    gives the latent) and w_up_t [Dm, D] (latent @ w_up_t^T gives model width),
+    each ~ N(0, 1/fan_in)."""
+    h = matrix_bf16(w.T, model_width, 1.0, STREAM_H, w.seed)
+    w_down_t = matrix_bf16(w.D, model_width, model_width ** -0.5, STREAM_W_DOWN, w.seed)
+    w_up_t = matrix_bf16(model_width, w.D, w.D ** -0.5, STREAM_W_UP, w.seed)
+    return h, w_down_t, w_up_t
 
 
 def scales(w: Workload) -> np.ndarray:

@@ -61,6 +61,7 @@ static inline uint16_t f32_bits_to_bf16(float f)
 
 /* stream ids */
 enum { ST_LOGIT = 1, ST_SEQBIAS = 2, ST_X = 3, ST_SCALE = 4, ST_PERM = 5, ST_DOUT = 6 };
+/* streams >= 16 are free for named matrices (activations, projection weights) */
 
 /*
  * Router logits, row-major [T, E] fp32.
@@ -128,6 +129,20 @@ int synth_dout_f32(int64_t T, int32_t D, uint64_t seed, float *out)
     const int64_t n = T * (int64_t)D;
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) out[i] = (float)draw_normal(kd, (uint64_t)i);
+    return 0;
+}
+
+/* A named bf16 matrix [rows, cols]: N(0, std^2) rounded to fp32, then to bf16
+ * (activations and synthetic random-init projection weights). */
+int synth_matrix_bf16(int64_t rows, int64_t cols, double std, uint64_t seed, uint64_t stream,
+                      uint16_t *out)
+{
+    if (rows < 0 || cols <= 0 || !out || stream < 16) return -1;
+    const uint64_t km = stream_key(seed, stream);
+    const int64_t n = rows * cols;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = f32_bits_to_bf16((float)(std * draw_normal(km, (uint64_t)i)));
     return 0;
 }
 

@@ -304,6 +304,31 @@ int moe_pw_dispatch_backward(const moe_pw_config *cfg, const uint16_t *d_pool,
                              moe_pw_counters *counters, cudaStream_t stream);
 
 /*
+ * Latent projection on the tensor cores (section 二: the routed activations are
+ * compressed from the 6144-wide model state to 3072 before the exchange and
+ * projected back afterwards).  C[m][n] = bf16_rn(sum_k A[m][k] * Bt[n][k]),
+ * fp32 accumulation in TMEM (tcgen05.mma, bf16 operands).  A: bf16 [M, K]
+ * row-major, Bt: bf16 [N, K] row-major (one row per output column), C: bf16
+ * [M, N].  K % 8 == 0, N % 8 == 0, all three 16-byte aligned.  counters
+ * receives MOE_PW_DEVERR_TIMEOUT if a bounded wait gives up.
+ */
+int moe_pw_project(const uint16_t *A, const uint16_t *Bt, uint16_t *C, int64_t M, int32_t N,
+                   int32_t K, moe_pw_counters *counters, cudaStream_t stream);
+
+/*
+ * Down-projection fused with the pack: pool_x[slot] = bf16(h[t] @ w_down_t^T)
+ * for every (t, j) the sender kept (slot_map from moe_pw_assign), written by
+ * the GEMM epilogue directly into the pool slots, headers as in moe_pw_pack,
+ * and the empty pool tails zero-filled: the same pools moe_pw_pack builds
+ * from x = bf16(h @ w_down_t^T), without materialising x.
+ * h: bf16 [T, model_width]; w_down_t: bf16 [D, model_width].
+ */
+int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint16_t *w_down_t,
+                        int32_t model_width, const int32_t *idx, const int32_t *slot_map,
+                        const int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr,
+                        moe_pw_counters *counters, cudaStream_t stream);
+
+/*
  * Drop statistics (section 二: the two kinds of drop are reported apart).
  * Copies *counters (device) to *host_out (host memory) and synchronises the
  * stream.  Returns MOE_PW_EDEVICE when a kernel flagged a violation (the

@@ -108,6 +108,7 @@ def _configure(lib):
     lib.orc_combine_backward.argtypes = [gp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.orc_dispatch_backward.argtypes = [gp, vp, vp, vp, vp]
     lib.orc_backward_tokens.argtypes = [gp, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp]
+    lib.orc_project.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp]
     lib.orc_bf16_round.argtypes = [vp, vp, i64]
     lib.orc_expert_product.argtypes = [vp, vp, vp, i64]
     return lib
@@ -353,6 +354,21 @@ def run_backward(w, r: dict, dout: np.ndarray, scale: np.ndarray) -> dict:
         b["d_pool"], _ = expert_ragged(g, b["d_ret"], r["pool_hdr"], scale)
     b["dx"] = dispatch_backward(g, b["d_pool"], r["recv_row"], r["slot_map"])
     return b
+
+
+def project(A: np.ndarray, Bt: np.ndarray, exact: bool = False):
+    """C = bf16(A @ Bt^T) (bf16 bits); with exact=True also the double sums
+    and sum |terms|."""
+    A, Bt = _c(A, np.uint16), _c(Bt, np.uint16)
+    M, K = A.shape
+    N = Bt.shape[0]
+    assert Bt.shape[1] == K
+    C = np.empty((M, N), np.uint16)
+    Ce = np.empty((M, N), np.float64) if exact else None
+    mag = np.empty((M, N), np.float64) if exact else None
+    _load().orc_project(_p(A), _p(Bt), M, N, K, _p(C), _p(Ce) if exact else None,
+                        _p(mag) if exact else None)
+    return (C, Ce, mag) if exact else C
 
 
 def bf16_round(a: np.ndarray) -> np.ndarray:

@@ -599,3 +599,36 @@ void orc_backward_tokens(const orc_geom *g, const uint16_t *x, const int32_t *id
             dl[idx[t * k + j]] = gates[t * k + j] * (dgate[n * k + j] - weighted);
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Latent projections.                                                       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * "Marin 开始公开训练 535B 参数 MoE 模型", section 二: before the routed
+ * activations cross GPUs a latent projection halves their width (6144 ->
+ * 3072), and the outputs are projected back before they meet the shared
+ * experts.  READING: a plain matrix product with bf16 operands,
+ *   C[m][n] = bf16( sum_k A[m][k] * Bt[n][k] ),
+ * the sum in double, rounded to fp32 and then to bf16 nearest-even (the
+ * device accumulates in fp32).  Bt is stored row n = output column n.
+ * Also returns, per element, sum_k |A[m][k] * Bt[n][k]| (the accumulation
+ * error is measured against it).
+ */
+void orc_project(const uint16_t *A, const uint16_t *Bt, int64_t M, int64_t N, int64_t K,
+                 uint16_t *C, double *Cexact, double *mag)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, am = 0.0;
+            for (int64_t kk = 0; kk < K; ++kk) {
+                const double p = (double)bf16_to_f32(A[m * K + kk]) * (double)bf16_to_f32(Bt[n * K + kk]);
+                acc += p;
+                am += fabs(p);
+            }
+            C[m * N + n] = f32_to_bf16_rne((float)acc);
+            if (Cexact) Cexact[m * N + n] = acc;
+            if (mag) mag[m * N + n] = am;
+        }
+    }
+}

@@ -1,0 +1,130 @@
+"""Latent projection on the tensor cores (tcgen05) against the CPU oracle.
+
+Tolerance (derived): the device accumulates K bf16 products in fp32 and
+rounds to bf16; the oracle sums in double.  |gpu - exact| <= 2^-8 |exact| (bf16
+rounding, one ulp margin) + 2^-20 * sum_k |a_k b_k| (fp32 accumulation: K
+roundings of partial sums, K <= 6144 < 2^13 gives K * 2^-24 < 2^-11 of the
+magnitude; the bound leaves room), and the bf16 codes must agree on almost
+every element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_moe_pw_b200 import moe_pw as mp
+from combine_moe_pw_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _f64(u16):
+    return (u16.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _ctr():
+    return torch.zeros((mp.COUNTERS_BYTES // 8,), dtype=torch.int64, device="cuda")
+
+
+def gpu_project(A, Bt):
+    M, K = A.shape
+    N = Bt.shape[0]
+    a = torch.from_numpy(A.view(np.int16)).cuda()
+    b = torch.from_numpy(Bt.view(np.int16)).cuda()
+    c = torch.full((M, N), 0x7FC0, dtype=torch.int16, device="cuda")  # NaN poison
+    ctr = _ctr()
+    mp.moe_pw_project(a, b, c, M, N, K, ctr)
+    torch.cuda.synchronize()
+    assert mp.moe_pw_stats(mp.Config(T=0, E=8, k=1, D=8, R=1, L=8, W=1, P=8), ctr).error == 0
+    return c.cpu().numpy().view(np.uint16), ctr
+
+
+def check_project(A, Bt, C):
+    Cr, Ce, mag = oracle.project(A, Bt, exact=True)
+    got = _f64(C)
+    assert np.all(np.isfinite(got))
+    assert np.all(np.abs(got - Ce) <= 2.0 ** -8 * np.abs(Ce) + 2.0 ** -20 * mag + 1e-30)
+    assert (C != Cr).mean() < 0.02
+
+
+def test_single_tile():
+    A = synth.matrix_bf16(128, 64, 1.0, 30)
+    Bt = synth.matrix_bf16(256, 64, 0.125, 31)
+    C, ctr = gpu_project(A, Bt)
+    check_project(A, Bt, C)
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 512, 128), (300, 264, 200), (1, 8, 8), (129, 264, 4096),
+                                   (640, 3072, 256), (512, 768, 1024)])
+def test_shapes(M, N, K):
+    A = synth.matrix_bf16(M, K, 1.0, 32)
+    Bt = synth.matrix_bf16(N, K, K ** -0.5, 33)
+    C, ctr = gpu_project(A, Bt)
+    check_project(A, Bt, C)
+
+
+def test_identity_weights_copy_rows():
+    K = 256
+    A = synth.matrix_bf16(384, K, 1.0, 34)
+    eye = torch.eye(K, dtype=torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    C, _ = gpu_project(A, eye)
+    np.testing.assert_array_equal(C, A)
+
+
+def _pack_inputs(w, Dm):
+    lg = synth.logits(w)
+    h, wd, _ = synth.projection_inputs(w, Dm)
+    return lg, h, wd
+
+
+@pytest.mark.parametrize("name,Dm", [("tiny", 256), ("pages_small", 1024)])
+def test_project_pack_matches_two_step_and_oracle(name, Dm):
+    w = (synth.WORKLOADS["tiny"] if name == "tiny" else
+         synth.Workload("pages_small", T=64 * 64, R=64, L=6, W=3, P=2, k=8, D=512, seq_len=1024,
+                        logit_kind=synth.LOGIT_SEQBIAS))
+    lg, h, wd = _pack_inputs(w, Dm)
+    cfg = mp.Config.from_workload(w)
+    b = mp.Buffers(cfg)
+    b.logits.copy_(torch.from_numpy(lg))
+    hd = torch.from_numpy(h.view(np.int16)).cuda()
+    wdd = torch.from_numpy(wd.view(np.int16)).cuda()
+    b.route()
+    b.assign()
+    # two-step: x = project(h), then pack
+    mp.moe_pw_project(hd, wdd, b.x, w.T, w.D, Dm, b.counters)
+    b.pack()
+    ref_pool = b.pool_x.clone()
+    ref_hdr = b.pool_hdr.clone()
+    x_gpu = b.x.cpu().numpy().view(np.uint16)
+    # fused
+    b.pool_x.fill_(0x1234)
+    b.pool_hdr.fill_(-7)
+    mp.moe_pw_project_pack(cfg, hd, wdd, Dm, b.idx, b.slot_map, b.occ, b.pool_x, b.pool_hdr,
+                           b.counters)
+    st = b.stats()
+    assert st.error == 0
+    assert torch.equal(b.pool_x, ref_pool) and torch.equal(b.pool_hdr, ref_hdr)
+    # the projection itself against the oracle, and the pools against an
+    # oracle pack of the GPU's x (integer work: bit-exact)
+    check_project(h, wd, x_gpu)
+    r = oracle.run_headers(w, lg)
+    np.testing.assert_array_equal(b.pool_hdr.cpu().numpy(), r["pool_hdr"])
+    pool = b.pool_x.cpu().numpy().view(np.uint16)
+    full = r["slot_tok"] >= 0
+    np.testing.assert_array_equal(pool[full], x_gpu[r["slot_tok"][full]])
+    assert not pool[~full].any()
+
+
+def test_down_projection_full_size_sampled():
+    """Rack batch: h [262144, 6144] x w_down^T -> [262144, 3072], rows sampled."""
+    w = synth.WORKLOADS["rack"]
+    h, wd, _ = synth.projection_inputs(w)
+    hd = torch.from_numpy(h.view(np.int16)).cuda()
+    wdd = torch.from_numpy(wd.view(np.int16)).cuda()
+    c = torch.empty((w.T, w.D), dtype=torch.int16, device="cuda")
+    ctr = _ctr()
+    mp.moe_pw_project(hd, wdd, c, w.T, w.D, h.shape[1], ctr)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([np.random.default_rng(5).integers(0, w.T, 24), [0, w.T - 1]]))
+    C = c[torch.from_numpy(rows).cuda()].cpu().numpy().view(np.uint16)
+    check_project(h[rows], wd, C)
