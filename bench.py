@@ -52,9 +52,76 @@ def parse():
     ap.add_argument("--cpu-sample-sources", type=int, default=16)
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward timing (reported apart from the metric)")
+    ap.add_argument("--no-projection", action="store_true",
+                    help="skip the latent-projection timing (reported apart from the metric)")
+    ap.add_argument("--projection-only", action="store_true",
+                    help="time only the tensor-core projections (profiling)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the batch's token count (profiling a smaller case)")
     return ap.parse_args()
+
+
+def measured_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return float(json.load(open(p))["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def time_projection(w, dev, stream, steps: int, b=None):
+    """The latent projections on the tensor cores: down (model width 6144 ->
+    latent), up (latent -> model width), and the down-projection fused with the
+    pack against project-then-pack.  Inputs are seeded random activations and
+    random-init weights already in HBM."""
+    import torch
+    from combine_moe_pw_b200 import moe_pw as mp
+    from combine_moe_pw_b200 import synth
+    T, D, Dm = w.T, w.D, synth.MODEL_WIDTH
+    g = torch.Generator(device=dev).manual_seed(w.seed)
+    h = torch.randn(T, Dm, device=dev, generator=g).to(torch.bfloat16).view(torch.int16)
+    wd = (torch.randn(D, Dm, device=dev, generator=g) * Dm ** -0.5).to(torch.bfloat16).view(torch.int16)
+    wu = (torch.randn(Dm, D, device=dev, generator=g) * D ** -0.5).to(torch.bfloat16).view(torch.int16)
+    xl = torch.empty(T, D, dtype=torch.int16, device=dev)
+    y = torch.empty(T, Dm, dtype=torch.int16, device=dev)
+    ctr = torch.zeros(mp.COUNTERS_BYTES // 8, dtype=torch.int64, device=dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        torch.cuda.synchronize(dev)
+        for e0, e1 in evs:
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+
+    flops = 2.0 * T * D * Dm
+    peak, kind = measured_tflops()
+    out = {"model_width": Dm, "latent_width": D, "tokens": T, "flops_per_gemm": flops,
+           "peak_tflops": peak, "peak_kind": kind}
+    ms = timed(lambda: mp.moe_pw_project(h, wd, xl, T, D, Dm, ctr, stream))
+    out["down_ms"] = ms
+    out["down_tflops"] = flops / ms / 1e9
+    ms = timed(lambda: mp.moe_pw_project(xl, wu, y, T, Dm, D, ctr, stream))
+    out["up_ms"] = ms
+    out["up_tflops"] = flops / ms / 1e9
+    out["down_frac"] = out["down_tflops"] / peak
+    out["up_frac"] = out["up_tflops"] / peak
+    if b is not None:
+        cfg = b.cfg
+        out["project_pack_ms"] = timed(lambda: mp.moe_pw_project_pack(
+            cfg, h, wd, Dm, b.idx, b.slot_map, b.occ, b.pool_x, b.pool_hdr, b.counters, stream))
+
+        def two_step():
+            mp.moe_pw_project(h, wd, b.x, T, D, Dm, b.counters, stream)
+            b.pack(stream)
+        out["project_then_pack_ms"] = timed(two_step)
+    del h, wd, wu, xl, y
+    torch.cuda.empty_cache()
+    return out
 
 
 def rank_workload(base, rank: int):
@@ -275,6 +342,13 @@ def main():
     b.scale.copy_(torch.from_numpy(s))
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
+    if a.projection_only:
+        b.route(stream)
+        b.assign(stream)
+        proj = time_projection(w, dev, stream, a.steps, b)
+        if rank == 0:
+            print(json.dumps({"projection": proj}), flush=True)
+        return
 
     stages = ["route", "assign", "pack", "bucket", "expert", "combine"]
 
@@ -379,6 +453,10 @@ def main():
         del b.d_ret, b.d_pool
         torch.cuda.empty_cache()
 
+    proj = None
+    if not a.no_projection:
+        proj = time_projection(w, dev, stream, min(a.steps, 10), b)
+
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
     if not a.no_e2e:
@@ -443,6 +521,7 @@ def main():
                          "alg_bytes_per_launch": ab[dom], "peak_kind": peak_kind},
             "gpu_launches": launches_per_step * a.steps,
             "backward": bwd,
+            "projection": proj,
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,

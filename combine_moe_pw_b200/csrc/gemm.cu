@@ -18,7 +18,9 @@
 //               thread, commits each stage back to the producer and each
 //               finished tile to the epilogue
 //   warps 2..5  epilogue: tcgen05.ld the accumulator (warp w reads TMEM
-//               lanes 32*(w%4)...), round to bf16 and store; the two
+//               lanes 32*(w%4)...), round to bf16 into a padded shared-memory
+//               copy of its 32 rows, release the accumulator, then write each
+//               row segment as one coalesced 512-byte warp store; the two
 //               accumulators let the epilogue of tile i overlap the MMAs of
 //               tile i+1
 // Tiles are visited n-fastest so the 12 column tiles of one row block run
@@ -29,9 +31,10 @@
 // Epilogue modes:
 //   ROWS     C row-major [M, ldc]
 //   SCATTER  project-and-pack: row m (token t) is written straight into the
-//            pool slot of every (t, j) the sender kept (slot_map), 512 bytes
-//            of the row per column tile, and the tile at column 0 writes the
-//            slot header; the latent rows are never materialised.
+//            pool slot of every (t, j) the sender kept (slot_map), one
+//            coalesced 512-byte store per slot and column tile, and the tile
+//            at column 0 writes the slot header; the latent rows are never
+//            materialised.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -44,12 +47,23 @@ namespace moe_pw {
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+#ifndef MOE_PW_GEMM_STAGES
+#define MOE_PW_GEMM_STAGES 4
+#endif
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = MOE_PW_GEMM_STAGES;
 constexpr uint32_t A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint32_t GEMM_WAIT_LIMIT = 1u << 24;
-constexpr size_t SMEM_BYTES = size_t(STAGES) * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+// epilogue staging: per epilogue warp 32 rows x half a tile (128 bf16 =
+// 256 bytes); the 16-byte chunk c of row r is stored at chunk c ^ (r & 7), so
+// both the per-row writes and the per-chunk reads spread over the banks
+constexpr int HALF = BN / 2;
+constexpr int SLOTS_IN_REGS = 8;  // choices per token whose slots the epilogue keeps in registers
+constexpr uint32_t ROW_PITCH = HALF * 2;
+constexpr uint32_t STAGING_BYTES = 4 * 32 * ROW_PITCH;
+constexpr size_t SMEM_BYTES =
+    size_t(STAGES) * STAGE_BYTES + STAGING_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
 enum Mode { ROWS = 0, SCATTER = 1 };
 
@@ -104,7 +118,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     // stage buffers need 1024-byte alignment for the 128-byte swizzle atoms
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Shared *sh = reinterpret_cast<Shared *>(smem + size_t(STAGES) * STAGE_BYTES);
+    uint8_t *staging = smem + size_t(STAGES) * STAGE_BYTES;
+    Shared *sh = reinterpret_cast<Shared *>(staging + STAGING_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const int m_tiles = (p.M + BM - 1) / BM, n_tiles = (p.N + BN - 1) / BN;
@@ -188,55 +203,111 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
     } else {
-        // epilogue: TMEM lane quarter of this warp
+        // epilogue: TMEM lane quarter of this warp; each thread owns one row
         const int q = warp & 3;
-        const int row = q * 32 + lane;
+        uint8_t *stage_rows = staging + size_t(warp - 2) * 32 * ROW_PITCH;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             const int m_blk = tile / n_tiles, n_blk = tile - m_blk * n_tiles;
-            const bool ok = wait_or_abort(&sh->tfull[acc], acc_phase, sh, p.ctr);
-            if (!__all_sync(FULL_MASK, ok)) break;
-            umma::fence_after_sync();
-            const int64_t m = int64_t(m_blk) * BM + row;
-            const int n0 = n_blk * BN;
-            const bool row_ok = m < p.M;
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t v[32];
-                umma::tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), v);
-                uint4 out[4];
+            // SCATTER: the slots of this thread's own row, fetched before the
+            // accumulator is read so the store loop needs no global loads
+            int32_t row_slot[SLOTS_IN_REGS];
+            {
+                const int64_t my_m = int64_t(m_blk) * BM + q * 32 + lane;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    out[i].x = pack_bf16(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
-                    out[i].y = pack_bf16(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-                    out[i].z = pack_bf16(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-                    out[i].w = pack_bf16(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
-                }
-                if (!row_ok) continue;
-                const int nc = n0 + c * 32;
-                if (p.mode == ROWS) {
-                    uint16_t *dst = p.C + m * p.ldc + nc;
+                for (int j = 0; j < SLOTS_IN_REGS; ++j) row_slot[j] = -1;
+                if (p.mode == SCATTER && my_m < p.M && p.topk <= SLOTS_IN_REGS) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        if (nc + 8 * i + 8 <= p.N) reinterpret_cast<uint4 *>(dst)[i] = out[i];
-                } else {
-                    for (int j = 0; j < p.topk; ++j) {
-                        const int32_t slot = p.slot_map[m * p.topk + j];
-                        if (slot < 0) continue;
-                        if (slot >= p.n_slots) {
+                    for (int j = 0; j < SLOTS_IN_REGS; ++j) {
+                        if (j >= p.topk) break;
+                        int32_t sl = p.slot_map[my_m * p.topk + j];
+                        if (sl >= p.n_slots) {
                             set_error(p.ctr, MOE_PW_DEVERR_SLOT);
-                            continue;
+                            sl = -1;
                         }
-                        uint16_t *dst = p.pool_x + int64_t(slot) * p.N + nc;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            if (nc + 8 * i + 8 <= p.N) __stcs(reinterpret_cast<uint4 *>(dst) + i, out[i]);
-                        if (nc == 0) p.pool_hdr[slot] = p.idx[m * p.topk + j];
+                        row_slot[j] = sl;
+                        if (sl >= 0 && n_blk == 0) p.pool_hdr[sl] = p.idx[my_m * p.topk + j];
                     }
                 }
             }
-            umma::fence_before_sync();
-            mbar_arrive(&sh->tempty[acc]);
+            const bool ok = wait_or_abort(&sh->tfull[acc], acc_phase, sh, p.ctr);
+            if (!__all_sync(FULL_MASK, ok)) break;
+            umma::fence_after_sync();
+            const int n0 = n_blk * BN;
+            const int hw = lane >> 4, l16 = lane & 15;
+            for (int h = 0; h < 2; ++h) {
+                // 1. TMEM -> bf16 -> this thread's row (half h) in shared memory
+                uint8_t *my_row = stage_rows + size_t(lane) * ROW_PITCH;
+#pragma unroll 1
+                for (int c = 0; c < HALF / 32; ++c) {
+                    uint32_t v[32];
+                    umma::tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) +
+                                        uint32_t(acc * BN + h * HALF + c * 32),
+                                    v);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint4 o;
+                        o.x = pack_bf16(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+                        o.y = pack_bf16(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+                        o.z = pack_bf16(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+                        o.w = pack_bf16(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+                        const int chunk = (c * 4 + i) ^ (lane & 7);
+                        reinterpret_cast<uint4 *>(my_row)[chunk] = o;
+                    }
+                }
+                if (h == 1) {
+                    // 2. the accumulator is free for the next tile's MMAs
+                    umma::fence_before_sync();
+                    mbar_arrive(&sh->tempty[acc]);
+                }
+                __syncwarp();
+                // 3. each half-warp writes one 256-byte row segment per store:
+                //    rows r + hw, chunk l16 (ROWS), or that segment into every
+                //    kept slot of the row (SCATTER)
+                const int ncol = n0 + h * HALF + 8 * l16;
+                const bool col_ok = ncol + 8 <= p.N;
+                for (int r = 0; r < 32; r += 2) {
+                    const int row = r + hw;
+                    const int64_t m = int64_t(m_blk) * BM + q * 32 + row;
+                    const bool row_ok = m < p.M;
+                    const uint4 val = reinterpret_cast<const uint4 *>(
+                        stage_rows + size_t(row) * ROW_PITCH)[l16 ^ (row & 7)];
+                    if (p.mode == ROWS) {
+                        if (row_ok && col_ok) reinterpret_cast<uint4 *>(p.C + m * p.ldc + ncol)[0] = val;
+                        continue;
+                    }
+                    if (p.topk <= SLOTS_IN_REGS) {
+#pragma unroll
+                        for (int j = 0; j < SLOTS_IN_REGS; ++j) {
+                            const int32_t slot = __shfl_sync(FULL_MASK, row_slot[j], row);
+                            if (j < p.topk && slot >= 0 && col_ok)
+                                __stcs(reinterpret_cast<uint4 *>(p.pool_x + int64_t(slot) * p.N + ncol), val);
+                        }
+                        continue;
+                    }
+                    // more choices than registers hold: read the slots here
+                    for (int jb = 0; jb < p.topk; jb += 16) {
+                        int32_t my_slot = -1;
+                        if (row_ok && jb + l16 < p.topk) {
+                            my_slot = p.slot_map[m * p.topk + jb + l16];
+                            if (my_slot >= p.n_slots) {
+                                set_error(p.ctr, MOE_PW_DEVERR_SLOT);
+                                my_slot = -1;
+                            }
+                            if (my_slot >= 0 && n_blk == 0 && h == 0)
+                                p.pool_hdr[my_slot] = p.idx[m * p.topk + jb + l16];
+                        }
+                        const int jn = p.topk - jb < 16 ? p.topk - jb : 16;
+                        for (int j = 0; j < jn; ++j) {
+                            const int32_t slot = __shfl_sync(FULL_MASK, my_slot, (lane & 16) | j);
+                            if (slot >= 0 && col_ok)
+                                __stcs(reinterpret_cast<uint4 *>(p.pool_x + int64_t(slot) * p.N + ncol), val);
+                        }
+                    }
+                }
+                __syncwarp();
+            }
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
