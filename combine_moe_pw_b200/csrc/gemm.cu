@@ -149,6 +149,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
+            // the weights are re-read by every row block: keep them in L2
+            const uint64_t pol_b = policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
             for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -158,7 +160,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                     uint8_t *a_dst = smem + size_t(stage) * STAGE_BYTES;
                     mbar_arrive_expect_tx(&sh->full[stage], STAGE_BYTES);
                     umma::tma_load_2d(a_dst, &tmA, kk * BK, m_blk * BM, &sh->full[stage]);
-                    umma::tma_load_2d(a_dst + A_BYTES, &tmB, kk * BK, n_blk * BN, &sh->full[stage]);
+                    umma::tma_load_2d_hint(a_dst + A_BYTES, &tmB, kk * BK, n_blk * BN,
+                                           &sh->full[stage], pol_b);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -274,7 +277,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint4 val = reinterpret_cast<const uint4 *>(
                         stage_rows + size_t(row) * ROW_PITCH)[l16 ^ (row & 7)];
                     if (p.mode == ROWS) {
-                        if (row_ok && col_ok) reinterpret_cast<uint4 *>(p.C + m * p.ldc + ncol)[0] = val;
+                        if (row_ok && col_ok) __stcs(reinterpret_cast<uint4 *>(p.C + m * p.ldc + ncol), val);
                         continue;
                     }
                     if (p.topk <= SLOTS_IN_REGS) {

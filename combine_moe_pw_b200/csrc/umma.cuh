@@ -134,5 +134,17 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int32_t
         : "memory");
 }
 
+// The same load with an L2 eviction policy (createpolicy) for the tile.
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const void *tmap, int32_t c0,
+                                                 int32_t c1, uint64_t *bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))),
+        "l"(policy)
+        : "memory");
+}
+
 }  // namespace umma
 }  // namespace moe_pw
