@@ -100,8 +100,12 @@ def time_projection(w, dev, stream, steps: int, b=None):
 
     flops = 2.0 * T * D * Dm
     peak, kind = measured_tflops()
+    sustained = peak
+    pth = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pth):
+        sustained = float(json.load(open(pth)).get("bf16_tflops_sustained", peak))
     out = {"model_width": Dm, "latent_width": D, "tokens": T, "flops_per_gemm": flops,
-           "peak_tflops": peak, "peak_kind": kind}
+           "peak_tflops": peak, "peak_sustained_tflops": sustained, "peak_kind": kind}
     ms = timed(lambda: mp.moe_pw_project(h, wd, xl, T, D, Dm, ctr, stream))
     out["down_ms"] = ms
     out["down_tflops"] = flops / ms / 1e9
@@ -110,6 +114,8 @@ def time_projection(w, dev, stream, steps: int, b=None):
     out["up_tflops"] = flops / ms / 1e9
     out["down_frac"] = out["down_tflops"] / peak
     out["up_frac"] = out["up_tflops"] / peak
+    out["down_frac_sustained"] = out["down_tflops"] / sustained
+    out["up_frac_sustained"] = out["up_tflops"] / sustained
     if b is not None:
         cfg = b.cfg
         out["project_pack_ms"] = timed(lambda: mp.moe_pw_project_pack(
@@ -119,6 +125,11 @@ def time_projection(w, dev, stream, steps: int, b=None):
             mp.moe_pw_project(h, wd, b.x, T, D, Dm, b.counters, stream)
             b.pack(stream)
         out["project_then_pack_ms"] = timed(two_step)
+        # the whole routed branch, model width to model width
+        lat = torch.empty(T, D, dtype=torch.int16, device=dev)
+        out["routed_layer_ms"] = timed(lambda: b.run_routed_layer(h, wd, wu, Dm, lat, y, stream))
+        out["routed_layer_tokens_per_s"] = T / (out["routed_layer_ms"] / 1e3)
+        del lat
     del h, wd, wu, xl, y
     torch.cuda.empty_cache()
     return out

@@ -15,6 +15,8 @@
 // the row (8 bf16), issues the loads of all k rows for two chunks before
 // accumulating, and writes 2 x 16 bytes of fp32 per chunk.  Skipped terms are
 // warp-uniform branches.
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 
 namespace moe_pw {
@@ -49,12 +51,20 @@ __device__ __forceinline__ void fma_row(float (&acc)[8], float gj, const uint4 &
     acc[7] = fmaf(gj, __uint_as_float(v.w & 0xFFFF0000u), acc[7]);
 }
 
-template <int KMAX>
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+
+// OUT_BF16: write the sum rounded to bf16 (8 values per 16-byte chunk) instead
+// of fp32, the input format of the up-projection on the tensor cores.
+template <int KMAX, bool OUT_BF16>
 __global__ void MOE_PW_COMBINE_BOUNDS combine_kernel(const uint4 *__restrict__ ret_x,
                                                       const int32_t *__restrict__ ret_hdr,
                                                       const int32_t *__restrict__ slot_map,
                                                       const float *__restrict__ gates,
-                                                      float4 *__restrict__ out, int64_t T,
+                                                      void *__restrict__ out_raw, int64_t T,
                                                       int k, int cpr, int64_t n_slots,
                                                       moe_pw_counters *ctr)
 {
@@ -80,7 +90,8 @@ __global__ void MOE_PW_COMBINE_BOUNDS combine_kernel(const uint4 *__restrict__ r
             slot[j] = __shfl_sync(FULL_MASK, my_slot, j);
             gv[j] = __shfl_sync(FULL_MASK, my_gate, j);
         }
-        float4 *orow = out + t * (cpr * 2);
+        float4 *orow = reinterpret_cast<float4 *>(out_raw) + t * (cpr * 2);
+        uint4 *brow = reinterpret_cast<uint4 *>(out_raw) + t * cpr;
         for (int c0 = lane; c0 < cpr; c0 += 32 * U) {
             float acc[U][8];
 #pragma unroll
@@ -114,17 +125,26 @@ __global__ void MOE_PW_COMBINE_BOUNDS combine_kernel(const uint4 *__restrict__ r
             for (int u = 0; u < U; ++u) {
                 const int c = c0 + 32 * u;
                 if (c < cpr) {
-                    __stcs(orow + 2 * c, make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]));
-                    __stcs(orow + 2 * c + 1, make_float4(acc[u][4], acc[u][5], acc[u][6], acc[u][7]));
+                    if (OUT_BF16) {
+                        uint4 o;
+                        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+                        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+                        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+                        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+                        __stcs(brow + c, o);
+                    } else {
+                        __stcs(orow + 2 * c, make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]));
+                        __stcs(orow + 2 * c + 1, make_float4(acc[u][4], acc[u][5], acc[u][6], acc[u][7]));
+                    }
                 }
             }
         }
     }
 }
 
-template <int KMAX>
+template <int KMAX, bool OUT_BF16>
 cudaError_t launch_k(const Geo &g, const uint16_t *ret_x, const int32_t *ret_hdr,
-                     const int32_t *slot_map, const float *gates, float *out,
+                     const int32_t *slot_map, const float *gates, void *out,
                      moe_pw_counters *ctr, cudaStream_t st)
 {
     DevInfo di;
@@ -132,9 +152,9 @@ cudaError_t launch_k(const Geo &g, const uint16_t *ret_x, const int32_t *ret_hdr
     int64_t blocks = (g.T + 7) / 8;
     if (blocks > int64_t(di.sms) * MOE_PW_COMBINE_BLOCKS_PER_SM)
         blocks = int64_t(di.sms) * MOE_PW_COMBINE_BLOCKS_PER_SM;
-    combine_kernel<KMAX><<<unsigned(blocks), 256, 0, st>>>(
-        reinterpret_cast<const uint4 *>(ret_x), ret_hdr, slot_map, gates,
-        reinterpret_cast<float4 *>(out), g.T, g.k, g.D / 8, g.n_slots, ctr);
+    combine_kernel<KMAX, OUT_BF16><<<unsigned(blocks), 256, 0, st>>>(
+        reinterpret_cast<const uint4 *>(ret_x), ret_hdr, slot_map, gates, out, g.T, g.k, g.D / 8,
+        g.n_slots, ctr);
     return cudaGetLastError();
 }
 
@@ -145,9 +165,19 @@ cudaError_t launch_combine(const Geo &g, const uint16_t *ret_x, const int32_t *r
                            moe_pw_counters *ctr, cudaStream_t st)
 {
     if (g.T == 0) return cudaSuccess;
-    if (g.k <= 8) return launch_k<8>(g, ret_x, ret_hdr, slot_map, gates, out, ctr, st);
-    if (g.k <= 16) return launch_k<16>(g, ret_x, ret_hdr, slot_map, gates, out, ctr, st);
-    return launch_k<32>(g, ret_x, ret_hdr, slot_map, gates, out, ctr, st);
+    if (g.k <= 8) return launch_k<8, false>(g, ret_x, ret_hdr, slot_map, gates, out, ctr, st);
+    if (g.k <= 16) return launch_k<16, false>(g, ret_x, ret_hdr, slot_map, gates, out, ctr, st);
+    return launch_k<32, false>(g, ret_x, ret_hdr, slot_map, gates, out, ctr, st);
+}
+
+cudaError_t launch_combine_bf16(const Geo &g, const uint16_t *ret_x, const int32_t *ret_hdr,
+                                const int32_t *slot_map, const float *gates, uint16_t *out,
+                                moe_pw_counters *ctr, cudaStream_t st)
+{
+    if (g.T == 0) return cudaSuccess;
+    if (g.k <= 8) return launch_k<8, true>(g, ret_x, ret_hdr, slot_map, gates, out, ctr, st);
+    if (g.k <= 16) return launch_k<16, true>(g, ret_x, ret_hdr, slot_map, gates, out, ctr, st);
+    return launch_k<32, true>(g, ret_x, ret_hdr, slot_map, gates, out, ctr, st);
 }
 
 }  // namespace moe_pw

@@ -55,6 +55,9 @@ cudaError_t launch_combine(const Geo &g, const uint16_t *ret_x, const int32_t *r
                            const int32_t *slot_map, const float *gates, float *out,
                            moe_pw_counters *ctr, cudaStream_t st);
 
+cudaError_t launch_combine_bf16(const Geo &g, const uint16_t *ret_x, const int32_t *ret_hdr,
+                                const int32_t *slot_map, const float *gates, uint16_t *out,
+                                moe_pw_counters *ctr, cudaStream_t st);
 cudaError_t launch_combine_backward(const Geo &g, const float *dout, const uint16_t *ret_x,
                                     const int32_t *ret_hdr, const int32_t *slot_map,
                                     const int32_t *idx, const float *gates, uint16_t *d_ret,

@@ -262,6 +262,21 @@ int moe_pw_combine(const moe_pw_config *cfg, const uint16_t *ret_x, const int32_
     return cuda_rc(launch_combine(g, ret_x, ret_hdr, slot_map, gates, out, counters, stream));
 }
 
+int moe_pw_combine_bf16(const moe_pw_config *cfg, const uint16_t *ret_x, const int32_t *ret_hdr,
+                        const int32_t *slot_map, const float *gates, uint16_t *out,
+                        moe_pw_counters *counters, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.T == 0) return MOE_PW_OK;
+    if (!ret_x || !ret_hdr || !slot_map || !gates || !out || !counters) return MOE_PW_EINVAL;
+    if (!aligned(ret_x, 16) || !aligned(out, 16) || !aligned(ret_hdr, 4) ||
+        !aligned(slot_map, 4) || !aligned(gates, 4) || !aligned(counters, 8))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_combine_bf16(g, ret_x, ret_hdr, slot_map, gates, out, counters, stream));
+}
+
 int moe_pw_combine_backward(const moe_pw_config *cfg, const float *dout, const uint16_t *ret_x,
                             const int32_t *ret_hdr, const int32_t *slot_map, const int32_t *idx,
                             const float *gates, uint16_t *d_ret, float *dgates, float *dlogits,

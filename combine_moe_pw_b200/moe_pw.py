@@ -73,6 +73,7 @@ SIGNATURES = {
     "moe_pw_dispatch": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_expert": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_combine": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_combine_bf16": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_combine_backward": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_dispatch_backward": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_project": [_VP, _VP, _VP, _I64, ctypes.c_int32, ctypes.c_int32, _VP, _VP],
@@ -226,6 +227,13 @@ def moe_pw_combine(cfg, ret_x, ret_hdr, slot_map, gates, out, counters, stream=N
         _ptr(counters), _stream(stream)))
 
 
+def moe_pw_combine_bf16(cfg, ret_x, ret_hdr, slot_map, gates, out, counters, stream=None):
+    c = _cfg(cfg)
+    _check("moe_pw_combine_bf16", load_library().moe_pw_combine_bf16(
+        ctypes.byref(c), _ptr(ret_x), _ptr(ret_hdr), _ptr(slot_map), _ptr(gates), _ptr(out),
+        _ptr(counters), _stream(stream)))
+
+
 def moe_pw_combine_backward(cfg, dout, ret_x, ret_hdr, slot_map, idx, gates, d_ret, dgates,
                             dlogits, counters, stream=None):
     c = _cfg(cfg)
@@ -354,6 +362,25 @@ class Buffers:
                       self.d_pool, self.d_pool_hdr, stream)
         moe_pw_dispatch_backward(self.cfg, self.d_pool, self.recv_row, self.slot_map, self.dx,
                                  self.counters, stream)
+
+    def run_routed_layer(self, h, w_down_t, w_up_t, model_width: int, latent_bf16, out_model,
+                         stream=None):
+        """The whole routed branch from model width back to model width:
+        route -> assign -> down-projection fused with the pack -> bucket ->
+        expert op -> combine (bf16 latent) -> up-projection.  h: bf16 [T, Dm],
+        w_down_t: bf16 [D, Dm], w_up_t: bf16 [Dm, D], latent_bf16: bf16 [T, D]
+        (scratch), out_model: bf16 [T, Dm]."""
+        cfg = self.cfg
+        self.route(stream)
+        self.assign(stream)
+        moe_pw_project_pack(cfg, h, w_down_t, model_width, self.idx, self.slot_map, self.occ,
+                            self.pool_x, self.pool_hdr, self.counters, stream)
+        self.bucket(stream)
+        self.expert(stream)
+        moe_pw_combine_bf16(cfg, self.ret_x, self.ret_hdr, self.slot_map, self.gates, latent_bf16,
+                            self.counters, stream)
+        moe_pw_project(latent_bf16, w_up_t, out_model, cfg.T, model_width, cfg.D, self.counters,
+                       stream)
 
     def run_step(self, stream=None):
         """route -> dispatch (assign, pack, bucket) -> expert -> combine."""

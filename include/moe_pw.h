@@ -273,6 +273,15 @@ int moe_pw_combine(const moe_pw_config *cfg, const uint16_t *ret_x, const int32_
                    moe_pw_counters *counters, cudaStream_t stream);
 
 /*
+ * moe_pw_combine with the fp32 sum rounded to bf16 nearest-even (out: bf16
+ * [T, D]), the input of the up-projection (moe_pw_project with the up weights)
+ * that takes the combined latent back to model width (section 二).
+ */
+int moe_pw_combine_bf16(const moe_pw_config *cfg, const uint16_t *ret_x, const int32_t *ret_hdr,
+                        const int32_t *slot_map, const float *gates, uint16_t *out,
+                        moe_pw_counters *counters, cudaStream_t stream);
+
+/*
  * Backward of the combine.  The pages train this model ("Marin 开始公开训练 535B
  * 参数 MoE 模型", section 一) but give no backward; this is the derivative of the
  * forward definitions above.  Given dout = dL/dout (f32 [T, D]):

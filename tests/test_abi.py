@@ -18,7 +18,7 @@ HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 def _declared():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(moe_pw_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(moe_pw_[a-z0-9_]+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")

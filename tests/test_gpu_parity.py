@@ -305,3 +305,14 @@ def test_full_size_sampled_parity(name):
         assert r["kept"] == w.T * w.k
     del b
     torch.cuda.empty_cache()
+
+
+def test_combine_bf16_is_rounded_fp32_combine():
+    """The bf16 combine is the fp32 combine rounded to nearest-even, bit for bit."""
+    lg, x, s = _inputs(TINY)
+    b, st = run_gpu(TINY, lg, x, s)
+    out16 = torch.empty((TINY.T, TINY.D), dtype=torch.int16, device="cuda")
+    mp.moe_pw_combine_bf16(b.cfg, b.ret_x, b.ret_hdr, b.slot_map, b.gates, out16, b.counters)
+    torch.cuda.synchronize()
+    ref = b.out.to(torch.bfloat16).view(torch.int16)
+    assert torch.equal(out16, ref)

@@ -128,3 +128,53 @@ def test_down_projection_full_size_sampled():
     rows = np.unique(np.concatenate([np.random.default_rng(5).integers(0, w.T, 24), [0, w.T - 1]]))
     C = c[torch.from_numpy(rows).cuda()].cpu().numpy().view(np.uint16)
     check_project(h[rows], wd, C)
+
+
+@pytest.mark.parametrize("name,Dm", [("tiny", 256), ("pages_small", 1024)])
+def test_routed_layer_against_oracle_chain(name, Dm):
+    """h -> (down-projection + pack) -> bucket -> expert -> combine (bf16) ->
+    up-projection, against the oracle's chain on its own intermediates.
+    Where the chains may part: a bf16 rounding of the projected or combined
+    latent can land one ulp apart (double vs fp32 sums), so the bound is
+    2^-6 of sum_k |latent_k w_nk| plus 2^-8 of the value, and almost every
+    element must agree far more closely."""
+    w = (synth.WORKLOADS["tiny"] if name == "tiny" else
+         synth.Workload("pages_small", T=64 * 64, R=64, L=6, W=3, P=2, k=8, D=512, seq_len=1024,
+                        logit_kind=synth.LOGIT_SEQBIAS))
+    lg, s = synth.logits(w), synth.scales(w)
+    h, wd, wu = synth.projection_inputs(w, Dm)
+    b = mp.Buffers(mp.Config.from_workload(w))
+    b.logits.copy_(torch.from_numpy(lg))
+    b.scale.copy_(torch.from_numpy(s))
+    lat = torch.empty((w.T, w.D), dtype=torch.int16, device="cuda")
+    out = torch.empty((w.T, Dm), dtype=torch.int16, device="cuda")
+    b.run_routed_layer(torch.from_numpy(h.view(np.int16)).cuda(),
+                       torch.from_numpy(wd.view(np.int16)).cuda(),
+                       torch.from_numpy(wu.view(np.int16)).cuda(), Dm, lat, out)
+    assert b.stats().error == 0
+    # oracle chain
+    x, _, xmag = oracle.project(h, wd, exact=True)
+    r = oracle.run(w, lg, x, s)
+    lat_ref = oracle.bf16_round(r["out"].astype(np.float32))
+    out_ref, out_exact, mag = oracle.project(lat_ref, wu, exact=True)
+    got = _f64(out.cpu().numpy().view(np.uint16))
+    err = np.abs(got - out_exact)
+    assert np.all(err <= 2.0 ** -6 * mag + 2.0 ** -8 * np.abs(out_exact) + 1e-30)
+    assert (err <= 2.0 ** -8 * np.abs(out_exact) + 2.0 ** -18 * mag).mean() > 0.99
+    # the bf16 latent: every term of a token's combine is a multiple of the same
+    # x_i, latent_i = x_i * sum_j g_j s_j, so its error follows x_i's: the
+    # projection's own bound (2^-8 |x| + 2^-20 sum_k |h_k w_ik|, the second term
+    # for near-cancelling sums) and one bf16 ulp each for the expert row and
+    # the latent
+    got_lat = _f64(lat.cpu().numpy().view(np.uint16))
+    ref_lat = r["out"]
+    xf = _f64(x)
+    keep = r["slot_map"] >= 0
+    keep &= r["recv_row"][np.where(keep, r["slot_map"], 0)] >= 0
+    c = (r["gates"] * s[r["idx"]] * keep).sum(axis=1, keepdims=True)
+    bound = (2.0 ** -6 * np.abs(xf) + 2.0 ** -19 * xmag) * c + 1e-30
+    bad = np.abs(got_lat - ref_lat) > bound
+    if bad.any():
+        t, i = np.argwhere(bad)[0]
+        raise AssertionError(f"latent[{t},{i}] got {got_lat[t, i]!r} ref {ref_lat[t, i]!r} "
+                             f"x {xf[t, i]!r} c {c[t, 0]!r} bad {bad.sum()}")
