@@ -437,3 +437,34 @@ extern "C" int moe_pw_assign_noalloc(const moe_pw_config *cfg, const int32_t *id
     if ((rc = noalloc_scratch(&scratch)) != MOE_PW_OK) return rc;
     return cuda_rc(launch_assign(g, idx, slot_map, occ, counters, scratch, stream));
 }
+
+// ---------------------------------------------------------------------------
+// Self-test of the bounded wait every mbarrier wait in this library uses.
+// ---------------------------------------------------------------------------
+
+namespace moe_pw {
+namespace {
+
+// One warp waits on a phase of an mbarrier that nothing ever completes; the
+// wait gives up after `polls` polls and the kernel records the timeout.
+__global__ void selftest_wait_kernel(moe_pw_counters *ctr, uint32_t polls)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) mbar_init(&bar, 1);
+    fence_init_and_proxy();
+    __syncwarp();
+    const bool done = mbar_wait_bounded(&bar, 0u, polls);
+    if (!__all_sync(FULL_MASK, done) && threadIdx.x == 0) set_error(ctr, MOE_PW_DEVERR_TIMEOUT);
+}
+
+}  // namespace
+}  // namespace moe_pw
+
+extern "C" int moe_pw_selftest_wait_timeout(moe_pw_counters *counters, int32_t polls,
+                                            cudaStream_t stream)
+{
+    if (!counters || polls < 1) return MOE_PW_EINVAL;
+    if (!aligned(counters, 8)) return MOE_PW_EUNSUPPORTED;
+    selftest_wait_kernel<<<1, 32, 0, stream>>>(counters, uint32_t(polls));
+    return cuda_rc(cudaGetLastError());
+}

@@ -79,6 +79,7 @@ SIGNATURES = {
     "moe_pw_project": [_VP, _VP, _VP, _I64, ctypes.c_int32, ctypes.c_int32, _VP, _VP],
     "moe_pw_project_pack": [_CFG, _VP, _VP, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_stats": [_CFG, _VP, ctypes.POINTER(moe_pw_drop_stats), _VP],
+    "moe_pw_selftest_wait_timeout": [_VP, ctypes.c_int32, _VP],
 }
 
 _lib = None
@@ -273,6 +274,12 @@ def moe_pw_stats(cfg, counters, stream=None, raise_on_device_error: bool = True)
         return out
     _check("moe_pw_stats", rc)
     return out
+
+
+def moe_pw_selftest_wait_timeout(counters, polls: int = 4096, stream=None):
+    """Run the bounded-wait self-test (see include/moe_pw.h)."""
+    _check("moe_pw_selftest_wait_timeout", load_library().moe_pw_selftest_wait_timeout(
+        _ptr(counters), polls, _stream(stream)))
 
 
 COUNTERS_BYTES = ctypes.sizeof(moe_pw_counters)

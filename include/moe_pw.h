@@ -346,6 +346,16 @@ int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint1
 int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
                  moe_pw_drop_stats *host_out, cudaStream_t stream);
 
+/*
+ * Self-test of failure detection (no counterpart on the pages): launches one
+ * warp that waits, with the library's bounded mbarrier wait, on a barrier
+ * phase that nothing completes.  After `polls` polls the wait gives up, the
+ * kernel sets MOE_PW_DEVERR_TIMEOUT in counters->error and returns, and the
+ * CUDA context stays usable.  Lets a caller check that timeouts surface as a
+ * status instead of a hang.
+ */
+int moe_pw_selftest_wait_timeout(moe_pw_counters *counters, int32_t polls, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

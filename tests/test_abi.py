@@ -110,3 +110,20 @@ def test_empty_batch_plans(lib):
     base = mp.Config.from_workload(synth.WORKLOADS["tiny"])
     s = mp.moe_pw_plan(mp.Config(**{**base.__dict__, "T": 0}))
     assert s.n_slots == 0 and s.C_s == 0 and s.C_r == 0
+
+
+def test_misaligned_pointers_rejected_before_any_launch(lib):
+    cfg = mp.Config.from_workload(synth.WORKLOADS["tiny"])
+    good, odd = 1 << 20, (1 << 20) + 4  # placeholder addresses, never dereferenced
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_route(cfg, odd, good, good, stream=0)      # logits need 16-byte alignment
+    assert ei.value.code == mp.MOE_PW_EUNSUPPORTED
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_combine(cfg, good, good, good, good, odd + 8, good, stream=0)
+    assert ei.value.code == mp.MOE_PW_EUNSUPPORTED
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_project(good, good, good, 128, 264, 100, good, stream=0)  # K % 8 != 0
+    assert ei.value.code == mp.MOE_PW_EUNSUPPORTED
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_selftest_wait_timeout(good + 4, 16, stream=0)
+    assert ei.value.code == mp.MOE_PW_EUNSUPPORTED

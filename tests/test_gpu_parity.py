@@ -316,3 +316,16 @@ def test_combine_bf16_is_rounded_fp32_combine():
     torch.cuda.synchronize()
     ref = b.out.to(torch.bfloat16).view(torch.int16)
     assert torch.equal(out16, ref)
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A wait nothing satisfies gives up after its bound and reports
+    MOE_PW_DEVERR_TIMEOUT; the next real step on the same context is exact."""
+    cfg = mp.Config.from_workload(TINY)
+    ctr = torch.zeros((mp.COUNTERS_BYTES // 8,), dtype=torch.int64, device="cuda")
+    mp.moe_pw_selftest_wait_timeout(ctr, polls=4096)
+    st = mp.moe_pw_stats(cfg, ctr, raise_on_device_error=False)
+    assert st.error & mp.DEVERR_TIMEOUT
+    lg, x, s = _inputs(TINY)
+    b, st = run_gpu(TINY, lg, x, s)
+    check_full(TINY, lg, x, s, b, st)
