@@ -468,16 +468,21 @@ def main():
     if not a.no_projection:
         proj = time_projection(w, dev, stream, min(a.steps, 10), b)
 
-    # end to end through the public API: pinned host inputs in, result out, every step
+    # end to end through the public API: pinned host inputs in, result out, every step.
+    # The headline runs the batches through moe_pw.Pipeline (host copies of
+    # neighbouring batches overlapped with compute); a short one-batch-at-a-time
+    # run is reported beside it.
     e2e = None
     if not a.no_e2e:
         ke = a.e2e_steps or a.steps
         h_lg = torch.from_numpy(lg).pin_memory()
         h_x = torch.from_numpy(x.view(np.int16)).pin_memory()
         h_s = torch.from_numpy(s).pin_memory()
-        h_out = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
         h2d = h_lg.numel() * 4 + h_x.numel() * 2 + h_s.numel() * 4
-        d2h = h_out.numel() * 4 + mp.COUNTERS_BYTES
+        d2h = w.T * w.D * 4 + mp.COUNTERS_BYTES
+
+        # one batch at a time on one buffer set
+        h_out = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
 
         def e2e_step():
             b.logits.copy_(h_lg, non_blocking=True)
@@ -489,19 +494,39 @@ def main():
 
         for _ in range(2):
             e2e_step()
-        if world > 1:
-            dist.barrier()
+        ks = min(ke, 5)
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(ke):
+        for _ in range(ks):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        (e_ms,) = max_over_ranks([e0.elapsed_time(e1)], world, dev)
+        serial_ms = e0.elapsed_time(e1) / ks
+        del b
+        torch.cuda.empty_cache()
+
+        # pipelined
+        pipe = mp.Pipeline(cfg, device=dev, depth=2)
+        h_outs = [torch.empty((w.T, w.D), dtype=torch.float32).pin_memory() for _ in range(2)]
+        for i in range(2):
+            pipe.submit(h_lg, h_x, h_s, h_outs[i % 2])
+        pipe.synchronize()
+        if world > 1:
+            dist.barrier()
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record(pipe.s_in)
+        for i in range(ke):
+            pipe.submit(h_lg, h_x, h_s, h_outs[i % 2])
+        p1.record(pipe.s_out)
+        pipe.synchronize()
+        (e_ms,) = max_over_ranks([p0.elapsed_time(p1)], world, dev)
         e2e = {"value": throughput(w.T * w.k, ke, world, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e_ms / ke}
+               "ms_per_step": e_ms / ke, "pipeline_depth": 2,
+               "serial_ms_per_step": serial_ms,
+               "serial_value": throughput(w.T * w.k, 1, world, serial_ms)}
+        del pipe
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:

@@ -280,10 +280,8 @@ cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, i
     p.g = g;
 
     const size_t smem = rank_smem_bytes(g);
-    static bool attr_done[64] = {};
-    int dev = 0;
-    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
-    if (smem > 48 * 1024 && dev < 64 && !attr_done[dev]) {
+    if (smem > 48 * 1024) {
+        // the opt-in is a per-function attribute; setting it again is harmless
         DevInfo di;
         if (dev_info(&di) != 0) return cudaErrorUnknown;
         if ((err = cudaFuncSetAttribute(assign_count, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -292,7 +290,6 @@ cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, i
         if ((err = cudaFuncSetAttribute(assign_rank, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         di.smem_optin)) != cudaSuccess)
             return err;
-        attr_done[dev] = true;
     }
     assign_count<<<g.n_chunks, AW * 32, smem, st>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;

@@ -10,10 +10,12 @@ namespace moe_pw {
 
 int dev_info(DevInfo *out)
 {
+    static std::mutex mu;
     static DevInfo cache[64];
     static bool have[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    std::lock_guard<std::mutex> lock(mu);
     if (dev >= 0 && dev < 64 && have[dev]) {
         *out = cache[dev];
         return 0;

@@ -395,3 +395,65 @@ class Buffers:
         self.dispatch(stream)
         self.expert(stream)
         self.combine(stream)
+
+
+class Pipeline:
+    """Streams batches from pinned host memory through the path with the host
+    copies of neighbouring batches overlapped with compute.
+
+    ``depth`` device buffer sets are used in turn.  Batch i's inputs go up on
+    the copy-in stream while batch i-1 computes on its own stream and batch
+    i-2's output comes down on the copy-out stream (PCIe is full duplex and
+    the copy engines run beside the SMs).  Events order each buffer set's
+    reuse: inputs are overwritten only after the compute that read them, the
+    output only after its copy to the host.  Nothing blocks the host; call
+    ``synchronize()`` before reading results."""
+
+    def __init__(self, cfg: Config, device="cuda", depth: int = 2):
+        dev = torch.device(device)
+        self.cfg, self.depth, self.n = cfg, depth, 0
+        self.bufs = [Buffers(cfg, dev) for _ in range(depth)]
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+        self.s_comp = [torch.cuda.Stream(dev) for _ in range(depth)]
+        self.inputs_free = [None] * depth   # compute of the last batch in set b has read its inputs
+        self.output_free = [None] * depth   # last output of set b is on the host
+        self.h_counters = [torch.empty_like(b.counters, device="cpu").pin_memory() for b in self.bufs]
+
+    def submit(self, h_logits, h_x, h_scale, h_out):
+        """Queue one batch: pinned host logits f32 [T,E], x bf16 bits [T,D],
+        scale f32 [E]; the result lands in pinned host h_out f32 [T,D]."""
+        k = self.n % self.depth
+        b, sc = self.bufs[k], self.s_comp[k]
+        with torch.cuda.stream(self.s_in):
+            if self.inputs_free[k] is not None:
+                self.s_in.wait_event(self.inputs_free[k])
+            b.logits.copy_(h_logits, non_blocking=True)
+            b.x.copy_(h_x, non_blocking=True)
+            b.scale.copy_(h_scale, non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(self.s_in)
+        sc.wait_event(landed)
+        if self.output_free[k] is not None:
+            sc.wait_event(self.output_free[k])
+        b.run_step(sc)
+        done = torch.cuda.Event()
+        done.record(sc)
+        self.inputs_free[k] = done
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(done)
+            h_out.copy_(b.out, non_blocking=True)
+            self.h_counters[k].copy_(b.counters, non_blocking=True)
+            out_done = torch.cuda.Event()
+            out_done.record(self.s_out)
+        self.output_free[k] = out_done
+        self.n += 1
+        return k
+
+    def synchronize(self):
+        for s in [self.s_in, self.s_out, *self.s_comp]:
+            s.synchronize()
+
+    def stats(self, k: int) -> moe_pw_counters:
+        """Counters of the last batch that used buffer set k (after synchronize)."""
+        return moe_pw_counters.from_buffer_copy(self.h_counters[k].numpy().tobytes())

@@ -329,3 +329,26 @@ def test_bounded_wait_times_out_and_context_survives():
     lg, x, s = _inputs(TINY)
     b, st = run_gpu(TINY, lg, x, s)
     check_full(TINY, lg, x, s, b, st)
+
+
+def test_pipeline_matches_single_steps():
+    """Batches streamed through the overlapped pipeline give the same bytes as
+    one step at a time."""
+    ws = [TINY.with_(seed=i) for i in range(5)]
+    cfg = mp.Config.from_workload(TINY)
+    pipe = mp.Pipeline(cfg, depth=2)
+    outs, ctrs = [], []
+    for w in ws:
+        lg, x, s = _inputs(w)
+        h_out = torch.empty((w.T, w.D), dtype=torch.float32).pin_memory()
+        k = pipe.submit(torch.from_numpy(lg).pin_memory(),
+                        torch.from_numpy(x.view(np.int16)).pin_memory(),
+                        torch.from_numpy(s).pin_memory(), h_out)
+        outs.append(h_out)
+    pipe.synchronize()
+    for w, h_out in zip(ws, outs):
+        lg, x, s = _inputs(w)
+        b, st = run_gpu(w, lg, x, s)
+        assert torch.equal(h_out, b.out.cpu())
+    last = pipe.stats((len(ws) - 1) % 2)
+    assert last.error == 0 and last.kept > 0
