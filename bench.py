@@ -423,7 +423,7 @@ def main():
     bwd = None
     if not a.no_backward:
         b.alloc_backward()
-        b.dout.copy_(torch.from_numpy(synth.dout(w)))
+        b.dout.copy_(torch.from_numpy(synth.dout(w)))  # host copy freed right away
         names = ["combine_bwd", "expert_bwd", "dispatch_bwd"]
 
         def bstep(ev=None):
@@ -461,7 +461,7 @@ def main():
                "hbm_frac_of_peak": sum(bb.values()) / (tot_ms / 1e3) / 1e9 / measured_peaks()[0],
                "alg_bytes_per_step": sum(bb.values()),
                "stage_gbs": {n: bb[n] / (bms[n] / 1e3) / 1e9 for n in names}}
-        del b.d_ret, b.d_pool
+        del b.d_ret, b.d_pool, b.dout, b.dlogits, b.dx
         torch.cuda.empty_cache()
 
     proj = None
@@ -507,8 +507,10 @@ def main():
         torch.cuda.empty_cache()
 
         # pipelined
+        # one pinned result buffer: the downloads are ordered on the copy-out
+        # stream, so consecutive batches never write it at the same time
         pipe = mp.Pipeline(cfg, device=dev, depth=2)
-        h_outs = [torch.empty((w.T, w.D), dtype=torch.float32).pin_memory() for _ in range(2)]
+        h_outs = [h_out, h_out]
         for i in range(2):
             pipe.submit(h_lg, h_x, h_s, h_outs[i % 2])
         pipe.synchronize()
