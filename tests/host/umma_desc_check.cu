@@ -2,6 +2,7 @@
 // CUTLASS's cute::UMMA descriptor unions (compiled as host code, no GPU).
 #include <cstdio>
 #include <cute/arch/mma_sm100_desc.hpp>
+#include <cute/numeric/numeric_types.hpp>
 #include "umma.cuh"
 
 int main()
@@ -26,7 +27,7 @@ int main()
                     ++bad;
                 }
             }
-    for (uint32_t M : {64u, 128u})
+    for (uint32_t M : {64u, 128u, 256u})
         for (uint32_t N : {16u, 64u, 128u, 256u})
             for (int bf : {0, 1}) {
                 cute::UMMA::InstrDescriptor i;
@@ -45,6 +46,20 @@ int main()
                     ++bad;
                 }
             }
+    // the two shapes the kernels issue, against CUTLASS's own constructor
+    // (M = 256 is the two-SM form: 128 rows from each CTA of the pair)
+    {
+        using namespace cute;
+        const uint32_t ref128 = uint32_t(UMMA::make_instr_desc<bfloat16_t, bfloat16_t, float, 128, 256,
+                                                               UMMA::Major::K, UMMA::Major::K>());
+        const uint32_t ref256 = uint32_t(UMMA::make_instr_desc<bfloat16_t, bfloat16_t, float, 256, 256,
+                                                               UMMA::Major::K, UMMA::Major::K>());
+        if (ref128 != moe_pw::umma::idesc_f16(128, 256, true) ||
+            ref256 != moe_pw::umma::idesc_f16(256, 256, true)) {
+            std::printf("make_instr_desc mismatch: %x %x\n", ref128, ref256);
+            ++bad;
+        }
+    }
     std::printf(bad ? "FAIL %d\n" : "OK\n", bad);
     return bad != 0;
 }

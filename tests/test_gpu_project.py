@@ -7,6 +7,10 @@ roundings of partial sums, K <= 6144 < 2^13 gives K * 2^-24 < 2^-11 of the
 magnitude; the bound leaves room), and the bf16 codes must agree on almost
 every element.
 """
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -178,3 +182,44 @@ def test_routed_layer_against_oracle_chain(name, Dm):
         t, i = np.argwhere(bad)[0]
         raise AssertionError(f"latent[{t},{i}] got {got_lat[t, i]!r} ref {ref_lat[t, i]!r} "
                              f"x {xf[t, i]!r} c {c[t, 0]!r} bad {bad.sum()}")
+
+
+_FALLBACK_SHAPES = [(300, 264, 200), (129, 264, 4096), (512, 768, 1024), (1, 8, 8)]
+
+_FALLBACK_CHILD = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, {root!r})
+from combine_moe_pw_b200 import moe_pw as mp, synth
+out = {{}}
+for M, N, K in {shapes!r}:
+    A = synth.matrix_bf16(M, K, 1.0, 40)
+    Bt = synth.matrix_bf16(N, K, K ** -0.5, 41)
+    a = torch.from_numpy(A.view(np.int16)).cuda()
+    b = torch.from_numpy(Bt.view(np.int16)).cuda()
+    c = torch.full((M, N), 0x7FC0, dtype=torch.int16, device="cuda")
+    ctr = torch.zeros((mp.COUNTERS_BYTES // 8,), dtype=torch.int64, device="cuda")
+    mp.moe_pw_project(a, b, c, M, N, K, ctr)
+    torch.cuda.synchronize()
+    assert int(ctr[4].item()) & 0xFFFFFFFF == 0
+    out[f"{{M}}_{{N}}_{{K}}"] = c.cpu().numpy()
+np.savez({path!r}, **out)
+"""
+
+
+def test_one_sm_fallback_matches_pair_kernel(tmp_path):
+    """The one-SM kernel (the fallback where a cluster of two cannot be
+    launched; selected here with MOE_PW_GEMM_PAIR=0 in a child process) and
+    the default two-SM kernel: the same MMA steps in the same K order per
+    output element, so bit-identical products."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    path = str(tmp_path / "one_sm.npz")
+    code = _FALLBACK_CHILD.format(root=root, shapes=_FALLBACK_SHAPES, path=path)
+    env = {**os.environ, "MOE_PW_GEMM_PAIR": "0"}
+    subprocess.run([sys.executable, "-c", code], env=env, check=True, timeout=600)
+    one_sm = np.load(path)
+    for M, N, K in _FALLBACK_SHAPES:
+        A = synth.matrix_bf16(M, K, 1.0, 40)
+        Bt = synth.matrix_bf16(N, K, K ** -0.5, 41)
+        C, _ = gpu_project(A, Bt)
+        check_project(A, Bt, C)
+        np.testing.assert_array_equal(C, one_sm[f"{M}_{N}_{K}"].view(np.uint16))
