@@ -368,9 +368,10 @@ done:
 // Each MMA completion is committed to the same barrier in both CTAs at once
 // (tcgen05.commit to the pair's CTA mask): the odd CTA's producer and
 // epilogue learn of it as early as the even CTA's.  (Forwarding it from the
-// even CTA with a remote mbarrier arrive instead measured 40% slower.)  No
-// TMA load is multicast.  Every wait is bounded as above, and a timeout in
-// one CTA also raises the abort flag of the other.
+// even CTA with a remote mbarrier arrive instead measured 40% slower.)
+// Every TMA load writes only the issuing CTA's own shared memory.  Every
+// wait is bounded as above, and a timeout in one CTA also raises the abort
+// flag of the other.
 // --------------------------------------------------------------------------
 #ifndef MOE_PW_GEMM_PAIR_STAGES
 #define MOE_PW_GEMM_PAIR_STAGES 5

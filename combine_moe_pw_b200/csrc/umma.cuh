@@ -121,7 +121,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
         : "memory");
 }
 
-// 2-D tiled TMA load (no multicast) into shared memory, completion on `bar`.
+// 2-D tiled TMA load into this CTA's shared memory, completion on `bar`.
 // c0 is the inner (contiguous) coordinate in elements.
 __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int32_t c0, int32_t c1,
                                             uint64_t *bar)
