@@ -11,12 +11,17 @@
 //   ragged: one group, bin = expert e, row = offset[e] + rank.
 // Work is split into chunks of consecutive tokens inside a group and done in
 // three deterministic passes (no order-giving atomics):
-//   1. count : per chunk, per-warp histograms in shared memory, summed per bin;
+//   1. count : per chunk, per-warp histograms in shared memory (atomics),
+//              summed per bin;
 //   2. scan  : per (group, bin), exclusive prefix over the group's chunks;
 //   3. rank  : per chunk, recount, per-warp bases = chunk base + earlier warps,
 //              then each warp walks its assignments 32 at a time: lanes with
-//              the same bin find each other with match.any and take ranks in
-//              lane order.
+//              the same bin find each other (one ballot per bit of the bin
+//              id) and take ranks in lane order.
+// Passes 1 and 3 first read the chunk's expert ids with every thread's loads
+// in flight at once and keep their bins in shared memory, so the walks above
+// touch only shared memory (the latency of one global read per chunk instead
+// of one per 32 assignments of a warp).
 // Ragged mode adds a one-block scan of the per-expert totals into offsets.
 #include "common.cuh"
 
@@ -60,6 +65,7 @@ struct Smem {
     int32_t *bin_tab;  // [E]
     int32_t *hist;     // [AW][NB]
     int32_t *off;      // [E + 1] (ragged rank pass)
+    int32_t *bins;     // [chunk_tokens * k]: bin of each assignment of the chunk, -1 if invalid
 };
 
 __device__ __forceinline__ Smem carve(const Geo &g, int32_t *sm)
@@ -68,25 +74,61 @@ __device__ __forceinline__ Smem carve(const Geo &g, int32_t *sm)
     s.bin_tab = sm;
     s.hist = sm + g.E;
     s.off = s.hist + AW * g.NB;
+    s.bins = s.off + g.E + 1;
     return s;
 }
 
-// Per-warp histogram of this warp's slice of the chunk.
-__device__ __forceinline__ void warp_hist(const RankArgs &p, const Smem &s, int64_t wa0,
-                                          int64_t wa1, int warp, int lane)
+// bins[i] for the chunk's assignments a0 + i, i < n; the loads of one thread
+// are issued together.  flag: report ids outside [0, E) (rank pass).
+__device__ __forceinline__ void load_bins(const RankArgs &p, const Smem &s, int64_t a0, int n,
+                                          bool flag)
+{
+    constexpr int U = 8;
+    for (int i0 = threadIdx.x; i0 < n; i0 += U * blockDim.x) {
+        int32_t e[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * int(blockDim.x);
+            e[u] = i < n ? p.idx[a0 + i] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * int(blockDim.x);
+            if (i < n) {
+                int32_t b = -1;
+                if (e[u] >= 0 && e[u] < p.g.E)
+                    b = s.bin_tab[e[u]];
+                else if (flag)
+                    set_error(p.ctr, MOE_PW_DEVERR_EXPERT_ID);
+                s.bins[i] = b;
+            }
+        }
+    }
+}
+
+// Per-warp histogram of this warp's slice [w0, w1) of the chunk
+// (shared-memory atomics: the counts do not depend on their order).
+__device__ __forceinline__ void warp_hist(const RankArgs &p, const Smem &s, int w0, int w1,
+                                          int warp, int lane)
 {
     int32_t *h = s.hist + warp * p.g.NB;
-    for (int64_t a = wa0; a < wa1; a += 32) {
-        const int64_t ai = a + lane;
-        int32_t b = -1;
-        if (ai < wa1) {
-            const int32_t e = p.idx[ai];
-            if (e >= 0 && e < p.g.E) b = s.bin_tab[e];
-        }
-        const unsigned same = __match_any_sync(FULL_MASK, b);
-        if (b >= 0 && lane == __ffs(same) - 1) h[b] += __popc(same);
-        __syncwarp();
+    for (int i = w0 + lane; i < w1; i += 32) {
+        const int32_t b = s.bins[i];
+        if (b >= 0) atomicAdd(&h[b], 1);
     }
+}
+
+// Lanes of the warp holding the same key as this lane (key in [0, 2^nbits)):
+// one ballot per key bit.  All lanes call it with the same nbits.
+__device__ __forceinline__ unsigned equal_lanes(uint32_t key, int nbits)
+{
+    unsigned m = FULL_MASK;
+    for (int i = 0; i < nbits; ++i) {
+        const bool bit = (key >> i) & 1u;
+        const unsigned bal = __ballot_sync(FULL_MASK, bit);
+        m &= bit ? bal : ~bal;
+    }
+    return m;
 }
 
 __device__ __forceinline__ void setup(const RankArgs &p, const Smem &s)
@@ -105,8 +147,10 @@ __global__ void __launch_bounds__(AW * 32) assign_count(RankArgs p)
     int64_t a0, a1;
     int group;
     chunk_range(p.g, blockIdx.x, a0, a1, group);
-    const int64_t n = a1 - a0;
-    warp_hist(p, s, a0 + n * warp / AW, a0 + n * (warp + 1) / AW, warp, lane);
+    const int n = int(a1 - a0);
+    load_bins(p, s, a0, n, false);
+    __syncthreads();
+    warp_hist(p, s, n * warp / AW, n * (warp + 1) / AW, warp, lane);
     __syncthreads();
     int32_t *out = p.counts + int64_t(blockIdx.x) * p.g.NB;
     for (int b = threadIdx.x; b < p.g.NB; b += blockDim.x) {
@@ -210,9 +254,11 @@ __global__ void __launch_bounds__(AW * 32) assign_rank(RankArgs p)
     int64_t a0, a1;
     int group;
     chunk_range(p.g, blockIdx.x, a0, a1, group);
-    const int64_t n = a1 - a0;
-    const int64_t wa0 = a0 + n * warp / AW, wa1 = a0 + n * (warp + 1) / AW;
-    warp_hist(p, s, wa0, wa1, warp, lane);
+    const int n = int(a1 - a0);
+    load_bins(p, s, a0, n, true);
+    __syncthreads();
+    const int w0 = n * warp / AW, w1 = n * (warp + 1) / AW;
+    warp_hist(p, s, w0, w1, warp, lane);
     __syncthreads();
     // turn per-warp counts into per-warp starting ranks
     const int32_t *base = p.counts + int64_t(blockIdx.x) * p.g.NB;
@@ -227,22 +273,16 @@ __global__ void __launch_bounds__(AW * 32) assign_rank(RankArgs p)
     __syncthreads();
     int32_t *h = s.hist + warp * p.g.NB;
     const int64_t pool_base = int64_t(group) * p.g.NB;
-    for (int64_t a = wa0; a < wa1; a += 32) {
-        const int64_t ai = a + lane;
-        int32_t b = -1;
-        if (ai < wa1) {
-            const int32_t e = p.idx[ai];
-            if (e >= 0 && e < p.g.E)
-                b = s.bin_tab[e];
-            else
-                set_error(p.ctr, MOE_PW_DEVERR_EXPERT_ID);
-        }
-        const unsigned same = __match_any_sync(FULL_MASK, b);
+    const int nbits = 32 - __clz(p.g.NB);  // keys b + 1 in [0, NB]
+    for (int a = w0; a < w1; a += 32) {
+        const int i = a + lane;
+        const int32_t b = i < w1 ? s.bins[i] : -1;
+        const unsigned same = equal_lanes(uint32_t(b + 1), nbits);
         const int32_t r = (b >= 0 ? h[b] : 0) + __popc(same & lanemask_lt());
         __syncwarp();
         if (b >= 0 && lane == __ffs(same) - 1) h[b] += __popc(same);
         __syncwarp();
-        if (ai < wa1) {
+        if (i < w1) {
             int32_t slot = -1;
             if (b >= 0) {
                 if (ragged)
@@ -250,14 +290,15 @@ __global__ void __launch_bounds__(AW * 32) assign_rank(RankArgs p)
                 else if (r < p.g.C_s)
                     slot = int32_t((pool_base + b) * p.g.C_s + r);
             }
-            p.slot_map[ai] = slot;
+            p.slot_map[a0 + i] = slot;
         }
     }
 }
 
 size_t rank_smem_bytes(const Geo &g)
 {
-    return sizeof(int32_t) * (size_t(g.E) + size_t(AW) * g.NB + size_t(g.E) + 1);
+    return sizeof(int32_t) * (size_t(g.E) + size_t(AW) * g.NB + size_t(g.E) + 1 +
+                              size_t(g.chunk_tokens) * g.k);
 }
 
 }  // namespace

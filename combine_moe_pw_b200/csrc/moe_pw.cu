@@ -40,6 +40,10 @@ constexpr int64_t MAX_INT32 = 0x7FFFFFFF;
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+#ifndef MOE_PW_ASSIGN_CHUNK
+#define MOE_PW_ASSIGN_CHUNK 2048
+#endif
+
 // Validate a config and derive the kernel geometry.
 int make_geo(const moe_pw_config *c, Geo *g)
 {
@@ -92,8 +96,9 @@ int make_geo(const moe_pw_config *c, Geo *g)
         g->n_groups = 1;
         g->group_tokens = c->T;
     }
-    // ranking chunks: 256 tokens, never straddling a group
-    int64_t ct = 256;
+    // ranking chunks: MOE_PW_ASSIGN_CHUNK assignments (256 tokens at k = 8),
+    // never straddling a group
+    int64_t ct = MOE_PW_ASSIGN_CHUNK / c->k > 0 ? MOE_PW_ASSIGN_CHUNK / c->k : 1;
     if (g->group_tokens < ct) ct = g->group_tokens > 0 ? g->group_tokens : 1;
     g->chunk_tokens = ct;
     g->chunks_per_group = int32_t(ceil_div(g->group_tokens > 0 ? g->group_tokens : 1, ct));
