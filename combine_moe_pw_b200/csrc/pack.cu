@@ -21,8 +21,9 @@
 //   - a stage is refilled once the stores reading it are done
 //     (cp.async.bulk.wait_group.read), LAG tokens later, so about NS - LAG row
 //     loads and LAG tokens of stores stay in flight per warp;
-//   - afterwards every warp zero-fills the empty tails (positions >= occ) of
-//     its share of the pools from a zeroed shared-memory row.
+//   - afterwards the warps zero-fill the empty tails (positions >= occ) of the
+//     pools from a zeroed shared-memory row, taking pools one at a time from
+//     a counter (counters->work) so that uneven tails even out.
 // x is read once (evict_first); pool rows are written once (evict_first).
 // The defaults below came from a sweep on the 262,144-token batch: deeper
 // rings with fewer warps beat more warps with shallow rings; the lag between
@@ -163,8 +164,16 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
     }
     if (!ok && lane == 0) set_error(p.ctr, MOE_PW_DEVERR_TIMEOUT);
 
-    // zero-fill the empty tail of each pool (pooled mode)
-    for (int64_t q = gw; q < p.n_pools; q += GW) {
+    // zero-fill the empty tail of each pool (pooled mode).  Tails differ in
+    // length (0..C_s rows), so a fixed share per warp leaves some warps with
+    // far more rows than others; instead each warp takes the next pool from a
+    // counter once its copies are issued (which warp fills a tail does not
+    // change the result).
+    for (;;) {
+        int64_t q = 0;
+        if (lane == 0) q = atomicAdd(&p.ctr->work, 1);
+        q = __shfl_sync(FULL_MASK, q, 0);
+        if (q >= p.n_pools) break;
         int64_t filled = p.occ[q];
         if (filled < 0) filled = 0;
         if (filled > p.C_s) filled = p.C_s;
@@ -199,10 +208,12 @@ cudaError_t launch_lag(const PackArgs &p, const DevInfo &di, const Geo &g, int n
     if (err != cudaSuccess) return err;
     if (per_sm < 1) per_sm = 1;
     int64_t blocks = int64_t(di.sms) * per_sm;
-    const int64_t work = (g.T > g.n_pools ? g.T : g.n_pools);
-    const int64_t need = (work + nw - 1) / nw;
+    const int64_t units = (g.T > g.n_pools ? g.T : g.n_pools);
+    const int64_t need = (units + nw - 1) / nw;
     if (blocks > need) blocks = need;
     if (blocks < 1) blocks = 1;
+    // the zero-fill phase's pool counter starts at 0 for every launch
+    if ((err = cudaMemsetAsync(&p.ctr->work, 0, sizeof(int32_t), st)) != cudaSuccess) return err;
     pack_kernel<LAGT><<<unsigned(blocks), nw * 32, smem, st>>>(p);
     return cudaGetLastError();
 }

@@ -48,7 +48,7 @@ class moe_pw_counters(ctypes.Structure):
     _fields_ = [("sender_dropped", ctypes.c_uint64), ("receiver_dropped", ctypes.c_uint64),
                 ("kept", ctypes.c_uint64), ("max_occ", ctypes.c_int32),
                 ("max_fill", ctypes.c_int32), ("error", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("work", ctypes.c_int32)]
 
 
 class moe_pw_drop_stats(ctypes.Structure):

@@ -134,7 +134,8 @@ typedef struct moe_pw_sizes {
     int64_t total_bytes;    /* every buffer of the path, logits to out */
 } moe_pw_sizes;
 
-/* Device-side counters, written by the kernels.  moe_pw_assign zeroes them. */
+/* Device-side counters, written by the kernels.  moe_pw_assign zeroes them.
+ * Calls that may run at the same time need counters of their own. */
 typedef struct moe_pw_counters {
     unsigned long long sender_dropped;
     unsigned long long receiver_dropped;
@@ -142,7 +143,8 @@ typedef struct moe_pw_counters {
     int32_t max_occ;     /* largest pool occupancy */
     int32_t max_fill;    /* largest per-expert kept count */
     int32_t error;       /* MOE_PW_DEVERR_* bits */
-    int32_t reserved;
+    int32_t work;        /* scratch: moe_pw_pack's counter of pools handed out for
+                            zero-filling (reset by moe_pw_pack before its kernel) */
 } moe_pw_counters;
 
 /* Host copy of the counters, filled by moe_pw_stats. */
