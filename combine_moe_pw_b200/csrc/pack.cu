@@ -168,12 +168,14 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
     // length (0..C_s rows), so a fixed share per warp leaves some warps with
     // far more rows than others; instead each warp takes the next pool from a
     // counter once its copies are issued (which warp fills a tail does not
-    // change the result).
+    // change the result).  The next pool's number is fetched while the
+    // current tail is being filled, so the counter's round trip is hidden.
+    int32_t q_next = 0;
+    if (lane == 0) q_next = atomicAdd(&p.ctr->work, 1);
     for (;;) {
-        int64_t q = 0;
-        if (lane == 0) q = atomicAdd(&p.ctr->work, 1);
-        q = __shfl_sync(FULL_MASK, q, 0);
+        const int64_t q = __shfl_sync(FULL_MASK, q_next, 0);
         if (q >= p.n_pools) break;
+        if (lane == 0) q_next = atomicAdd(&p.ctr->work, 1);
         int64_t filled = p.occ[q];
         if (filled < 0) filled = 0;
         if (filled > p.C_s) filled = p.C_s;

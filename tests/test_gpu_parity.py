@@ -243,6 +243,24 @@ def test_deterministic_repeat():
         assert torch.equal(getattr(b1, name), getattr(b2, name)), name
 
 
+def test_repeated_pack_refills_every_tail():
+    """The pack's zero-fill phase hands pools out from a counter that the
+    library resets before each launch: a second pack without a new assignment
+    pass (pools poisoned in between) rebuilds the same pools byte for byte."""
+    w = TINY.with_(T=8 * 1024, seq_len=1024, D=256, logit_kind=synth.LOGIT_SEQBIAS)
+    lg, x, s = _inputs(w)
+    b, _ = run_gpu(w, lg, x, s)
+    ref_x, ref_hdr = b.pool_x.clone(), b.pool_hdr.clone()
+    assert (ref_hdr < 0).any()  # there are empty tails to refill
+    for _ in range(2):
+        b.pool_x.fill_(0x1357)
+        b.pool_hdr.fill_(-9)
+        b.pack()
+        torch.cuda.synchronize()
+        assert torch.equal(b.pool_x, ref_x) and torch.equal(b.pool_hdr, ref_hdr)
+    assert b.stats().error == 0
+
+
 def test_empty_batch():
     for mode in (synth.MODE_POOLED, synth.MODE_RAGGED):
         w = TINY.with_(T=0, mode=mode)
