@@ -201,7 +201,10 @@ int moe_pw_assign(const moe_pw_config *cfg, const int32_t *idx, int32_t *slot_ma
  * k writes), writes the expert id into the slot header, and fills the empty
  * tail of every pool (positions >= occ) with zeros and header -1.  Ragged
  * mode: rows only, no empty slots.  A slot_map entry >= n_slots is skipped
- * and flagged in counters->error (which moe_pw_assign zeroed).
+ * and flagged in counters->error (which moe_pw_assign zeroed).  The empty
+ * tails are handed out to the kernel's warps through counters->work, which
+ * this call resets on `stream` before the kernel; two packs that share a
+ * counters struct must not run at the same time.
  */
 int moe_pw_pack(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
                 const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
