@@ -15,7 +15,8 @@
 //
 // combine_bwd_kernel: one warp per token; lanes j < k read (slot, gate,
 // ret_hdr) once and the warp broadcasts them; each lane owns 16-byte chunks
-// of bf16 rows (and the matching 32 bytes of dout), accumulates its share of
+// of bf16 rows (and the matching 32 bytes of dout), two chunks per
+// iteration with all their loads issued first, accumulates its share of
 // every dot product with fmaf in chunk order, writes the gradient rows, and
 // the warp reduces the dots with a fixed xor-butterfly.
 #include <cuda_bf16.h>
@@ -25,6 +26,8 @@
 namespace moe_pw {
 
 namespace {
+
+constexpr int BU = 2;  // chunks per lane per iteration (their loads are in flight together)
 
 // two fp32 -> packed bf16 pair, round to nearest even (lo in the low half)
 __device__ __forceinline__ uint32_t bf16x2_of(float lo, float hi)
@@ -66,38 +69,52 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(
             dot[j] = 0.0f;
         }
         const float4 *drow = dout + t * (2 * int64_t(cpr));
-        for (int c = lane; c < cpr; c += 32) {
-            const float4 d0 = __ldcs(drow + 2 * c), d1 = __ldcs(drow + 2 * c + 1);
+        for (int c0 = lane; c0 < cpr; c0 += 32 * BU) {
+            float4 d0[BU], d1[BU];
+#pragma unroll
+            for (int u = 0; u < BU; ++u)
+                if (c0 + 32 * u < cpr) {
+                    d0[u] = __ldcs(drow + 2 * (c0 + 32 * u));
+                    d1[u] = __ldcs(drow + 2 * (c0 + 32 * u) + 1);
+                }
             // rows in groups of eight: the loads of a group, then its arithmetic
 #pragma unroll
             for (int jg = 0; jg < KMAX; jg += 8) {
-                uint4 y[8];
+                uint4 y[8][BU];
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
                     const int j = jg + jj;
-                    if (j < k && slot[j] >= 0) y[jj] = __ldcs(ret_x + int64_t(slot[j]) * cpr + c);
+                    if (j < k && slot[j] >= 0)
+#pragma unroll
+                        for (int u = 0; u < BU; ++u)
+                            if (c0 + 32 * u < cpr)
+                                y[jj][u] = __ldcs(ret_x + int64_t(slot[j]) * cpr + c0 + 32 * u);
                 }
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
                     const int j = jg + jj;
                     if (!(j < k && slot[j] >= 0)) continue;
-                    float a = dot[j];
-                    a = fmaf(d0.x, __uint_as_float(y[jj].x << 16), a);
-                    a = fmaf(d0.y, __uint_as_float(y[jj].x & 0xFFFF0000u), a);
-                    a = fmaf(d0.z, __uint_as_float(y[jj].y << 16), a);
-                    a = fmaf(d0.w, __uint_as_float(y[jj].y & 0xFFFF0000u), a);
-                    a = fmaf(d1.x, __uint_as_float(y[jj].z << 16), a);
-                    a = fmaf(d1.y, __uint_as_float(y[jj].z & 0xFFFF0000u), a);
-                    a = fmaf(d1.z, __uint_as_float(y[jj].w << 16), a);
-                    a = fmaf(d1.w, __uint_as_float(y[jj].w & 0xFFFF0000u), a);
-                    dot[j] = a;
                     const float g = gv[j];
-                    uint4 gr;
-                    gr.x = bf16x2_of(__fmul_rn(g, d0.x), __fmul_rn(g, d0.y));
-                    gr.y = bf16x2_of(__fmul_rn(g, d0.z), __fmul_rn(g, d0.w));
-                    gr.z = bf16x2_of(__fmul_rn(g, d1.x), __fmul_rn(g, d1.y));
-                    gr.w = bf16x2_of(__fmul_rn(g, d1.z), __fmul_rn(g, d1.w));
-                    __stcs(d_ret + int64_t(slot[j]) * cpr + c, gr);
+#pragma unroll
+                    for (int u = 0; u < BU; ++u) {
+                        if (c0 + 32 * u >= cpr) continue;
+                        float a = dot[j];
+                        a = fmaf(d0[u].x, __uint_as_float(y[jj][u].x << 16), a);
+                        a = fmaf(d0[u].y, __uint_as_float(y[jj][u].x & 0xFFFF0000u), a);
+                        a = fmaf(d0[u].z, __uint_as_float(y[jj][u].y << 16), a);
+                        a = fmaf(d0[u].w, __uint_as_float(y[jj][u].y & 0xFFFF0000u), a);
+                        a = fmaf(d1[u].x, __uint_as_float(y[jj][u].z << 16), a);
+                        a = fmaf(d1[u].y, __uint_as_float(y[jj][u].z & 0xFFFF0000u), a);
+                        a = fmaf(d1[u].z, __uint_as_float(y[jj][u].w << 16), a);
+                        a = fmaf(d1[u].w, __uint_as_float(y[jj][u].w & 0xFFFF0000u), a);
+                        dot[j] = a;
+                        uint4 gr;
+                        gr.x = bf16x2_of(__fmul_rn(g, d0[u].x), __fmul_rn(g, d0[u].y));
+                        gr.y = bf16x2_of(__fmul_rn(g, d0[u].z), __fmul_rn(g, d0[u].w));
+                        gr.z = bf16x2_of(__fmul_rn(g, d1[u].x), __fmul_rn(g, d1[u].y));
+                        gr.w = bf16x2_of(__fmul_rn(g, d1[u].z), __fmul_rn(g, d1[u].w));
+                        __stcs(d_ret + int64_t(slot[j]) * cpr + c0 + 32 * u, gr);
+                    }
                 }
             }
         }
