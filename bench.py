@@ -36,6 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "routed assignments/s and HBM GB/s (% of peak) for dispatch+combine; drop rate"
+HBM_DATASHEET_GBS = 8000.0  # B200 HBM3e, vendor figure (context beside the measured peak)
 UNIT = "assignments/s"
 
 
@@ -550,6 +551,7 @@ def main():
             "config": config_of(w),
             "hbm_gbs": gbs, "hbm_frac_of_peak": gbs / peak, "hbm_peak_gbs": peak,
             "hbm_peak_kind": peak_kind,
+            "hbm_datasheet_gbs": HBM_DATASHEET_GBS, "hbm_frac_of_datasheet": gbs / HBM_DATASHEET_GBS,
             "alg_bytes_per_step": b_alg,
             "drop_rate": {"sender": st.sender_dropped / TK, "receiver": st.receiver_dropped / TK,
                           "total": (st.sender_dropped + st.receiver_dropped) / TK},
