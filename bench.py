@@ -261,6 +261,20 @@ def traffic_from_profiles(kernel: str):
     return float(m_b.group(1))
 
 
+def host_cpu():
+    """The host the oracle is timed on: logical cores and CPU model."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
+
+
 def cpu_oracle_sample(w, n_src: int):
     """Time the CPU oracle (single thread) on the first n_src source shards of
     the batch: route, assignment, pack, bucketing, expert op and combine."""
@@ -303,7 +317,7 @@ def run_reference(a):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, **host_cpu()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -537,7 +551,8 @@ def main():
         cpu = {"value": u / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"first {a.cpu_sample_sources} of {base.R} source shards "
                          f"({a.cpu_sample_sources * (base.T // base.R)} tokens) of the {base.name} "
-                         f"batch, whole oracle path (route..combine), one thread, {dt:.1f} s"}
+                         f"batch, whole oracle path (route..combine), one thread, {dt:.1f} s",
+               **host_cpu()}
 
     if rank == 0:
         TK = w.T * w.k
