@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
     ap.add_argument("--cpu-sample-sources", type=int, default=16)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip the CUDA-graph timing of the whole forward step")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward timing (reported apart from the metric)")
     ap.add_argument("--no-projection", action="store_true",
@@ -395,10 +397,14 @@ def main():
         mark(5)
         b.combine(stream)
         mark(6)
-        return b.stats(stream)
 
+    # the counters are read after the loops, not per step: a per-step read
+    # synchronises the host, and the GPU would then wait for the next step's
+    # first launch inside the timed route stage (every step gives the same
+    # counters: the path is deterministic)
     for _ in range(max(a.warmup, 3)):
-        st = step()
+        step()
+    st = b.stats(stream)
     launches_per_step = 8 if w.mode == 0 else 9
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(a.steps)]
@@ -410,12 +416,40 @@ def main():
     torch.cuda.synchronize(dev)
     start.record(stream)
     for i in range(a.steps):
-        st = step(evs[i])
+        step(evs[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
+    st = b.stats(stream)
+
+    # the whole forward step (expert op included) as one CUDA graph, against
+    # the same step launched call by call
+    graph = None
+    if not a.no_graph:
+        g = b.capture_step()
+        for _ in range(3):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(a.steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        g_ms = e0.elapsed_time(e1) / a.steps
+        e0.record(stream)
+        for _ in range(a.steps):
+            b.run_step(stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        eager_ms = e0.elapsed_time(e1) / a.steps
+        g_ms, eager_ms = max_over_ranks([g_ms, eager_ms], world, dev)
+        graph = {"ms_per_step": g_ms, "eager_ms_per_step": eager_ms,
+                 "scope": "route, dispatch, expert op, combine (whole forward step)",
+                 "host_launches_per_step": 1}
+        del g
 
     total_ms = start.elapsed_time(end)
     per_stage = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(a.steps)]
@@ -575,6 +609,7 @@ def main():
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "alg_bytes_per_launch": ab[dom], "peak_kind": peak_kind},
             "gpu_launches": launches_per_step * a.steps,
+            "graph": graph,
             "backward": bwd,
             "projection": proj,
             "clocks": clocks,

@@ -396,6 +396,24 @@ class Buffers:
         self.expert(stream)
         self.combine(stream)
 
+    def capture_step(self):
+        """One forward step (``run_step``) recorded as a CUDA graph on these
+        buffers.  Every call of the step is asynchronous on its stream with no
+        host synchronisation, so the whole step captures; ``graph.replay()``
+        then runs it with one launch from the host.  The graph reads the
+        buffers' current contents when it runs: copy new logits, x and scales
+        into them and replay.  The step runs once eagerly first (on the
+        capture stream) so that every per-device setup is done before capture."""
+        side = torch.cuda.Stream(device=self.out.device)
+        side.wait_stream(torch.cuda.current_stream(self.out.device))
+        with torch.cuda.stream(side):
+            self.run_step()
+        torch.cuda.current_stream(self.out.device).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            self.run_step()
+        return graph
+
 
 class Pipeline:
     """Streams batches from pinned host memory through the path with the host

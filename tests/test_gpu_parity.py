@@ -370,3 +370,36 @@ def test_pipeline_matches_single_steps():
         assert torch.equal(h_out, b.out.cpu())
     last = pipe.stats((len(ws) - 1) % 2)
     assert last.error == 0 and last.kept > 0
+
+
+def test_captured_step_replays_bit_identical():
+    """The forward step recorded as a CUDA graph: a replay equals an eager
+    step byte for byte, and after new inputs are copied into the same
+    buffers the replay equals an eager step on those inputs."""
+    w = TINY.with_(T=8 * 1024, seq_len=1024, D=256, logit_kind=synth.LOGIT_SEQBIAS)
+    names = ["idx", "gates", "slot_map", "occ", "pool_x", "pool_hdr", "recv_row",
+             "bucket_slot", "expert_counts", "ret_x", "ret_hdr", "out"]
+    lg, x, s = _inputs(w)
+    ref, _ = run_gpu(w, lg, x, s)
+    b, _ = run_gpu(w, lg, x, s)
+    graph = b.capture_step()
+    for n in names:
+        getattr(b, n).fill_(0x55 if getattr(b, n).dtype != torch.float32 else 7.0)
+    graph.replay()
+    torch.cuda.synchronize()
+    for n in names:
+        assert torch.equal(getattr(b, n), getattr(ref, n)), n
+    assert b.stats().error == 0
+    w2 = w.with_(seed=5)
+    lg2, x2, s2 = _inputs(w2)
+    ref2, _ = run_gpu(w2, lg2, x2, s2)
+    b.logits.copy_(torch.from_numpy(lg2))
+    b.x.copy_(torch.from_numpy(x2.view(np.int16)))
+    b.scale.copy_(torch.from_numpy(s2))
+    graph.replay()
+    torch.cuda.synchronize()
+    for n in names:
+        assert torch.equal(getattr(b, n), getattr(ref2, n)), n
+    st, st2 = b.stats(), ref2.stats()
+    assert (st.kept, st.sender_dropped, st.receiver_dropped) == (
+        st2.kept, st2.sender_dropped, st2.receiver_dropped)
