@@ -324,7 +324,11 @@ int moe_pw_dispatch_backward(const moe_pw_config *cfg, const uint16_t *d_pool,
  * fp32 accumulation in TMEM (tcgen05.mma, bf16 operands).  A: bf16 [M, K]
  * row-major, Bt: bf16 [N, K] row-major (one row per output column), C: bf16
  * [M, N].  K % 8 == 0, N % 8 == 0, all three 16-byte aligned.  counters
- * receives MOE_PW_DEVERR_TIMEOUT if a bounded wait gives up.
+ * receives MOE_PW_DEVERR_TIMEOUT if a bounded wait gives up.  The product runs
+ * on pairs of SMs (tcgen05 cta_group::2, 256 x 256 tiles) where a cluster of
+ * two CTAs can be launched, else on single SMs (128 x 256 tiles); setting the
+ * environment variable MOE_PW_GEMM_PAIR=0 before the first call selects the
+ * single-SM kernel.  Both give bit-identical results.
  */
 int moe_pw_project(const uint16_t *A, const uint16_t *Bt, uint16_t *C, int64_t M, int32_t N,
                    int32_t K, moe_pw_counters *counters, cudaStream_t stream);
@@ -335,7 +339,8 @@ int moe_pw_project(const uint16_t *A, const uint16_t *Bt, uint16_t *C, int64_t M
  * the GEMM epilogue directly into the pool slots, headers as in moe_pw_pack,
  * and the empty pool tails zero-filled: the same pools moe_pw_pack builds
  * from x = bf16(h @ w_down_t^T), without materialising x.
- * h: bf16 [T, model_width]; w_down_t: bf16 [D, model_width].
+ * h: bf16 [T, model_width]; w_down_t: bf16 [D, model_width].  The tail fill
+ * uses counters->work as moe_pw_pack does.
  */
 int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint16_t *w_down_t,
                         int32_t model_width, const int32_t *idx, const int32_t *slot_map,
