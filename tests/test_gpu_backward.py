@@ -9,7 +9,9 @@ Tolerances (derived from the arithmetic):
   dgate bound -> 2e-5 * g_j * (M_j + sum_i g_i M_i), M = sum_i |dout_i y_i|.
 - gradient rows (bf16): the fp32 product g_j * dout uses the GPU's gate, which
   can differ from the oracle's by a few fp32 ulp, so a row element may round
-  to the neighbouring bf16 value: |err| <= 1 bf16 ulp, on a tiny fraction.
+  to the neighbouring bf16 value: |err| <= 1 bf16 ulp, on at most 0.1% of the
+  elements or 2 of them, whichever is more (each element flips independently
+  with a tiny probability, so a small case may show one or two).
 - dx: a sum of those bf16 rows (scaled once more): |err| <= 2^-7 * sum of
   |terms|, and all but a tiny fraction within 1e-6 of that sum.
 """
@@ -77,7 +79,7 @@ def check_backward(w, b, st, r, ob, dout):
     assert not d_ret[~live].any()
     got, ref = _f32(d_ret[live]), _f32(ob["d_ret"][live])
     assert np.all(np.abs(got - ref) <= _ulp_bf16(ref))
-    assert (got != ref).mean() < 1e-3
+    assert (got != ref).sum() <= max(1e-3 * got.size, 2)
     # expert backward rows
     d_pool = b.d_pool.cpu().numpy().view(np.uint16)
     assert not d_pool[~live].any()
@@ -89,7 +91,7 @@ def check_backward(w, b, st, r, ob, dout):
     mag = terms.sum(axis=1)
     err = np.abs(dx - ob["dx"])
     assert np.all(err <= 2.0 ** -7 * mag + 1e-30)
-    assert (err > 1e-6 * mag + 1e-30).mean() < 1e-3
+    assert (err > 1e-6 * mag + 1e-30).sum() <= max(1e-3 * err.size, 2)
 
 
 CASES = {
@@ -169,6 +171,6 @@ def test_backward_full_size_sampled(name):
     mag = (np.abs(ref) * s[e][:, :, None] * live[:, :, None]).sum(axis=1) * (1 + 2.0 ** -7)
     err = np.abs(gdx - dx)
     assert np.all(err <= 2.0 ** -7 * mag + 1e-30)
-    assert (err > 1e-6 * mag + 1e-30).mean() < 1e-3
+    assert (err > 1e-6 * mag + 1e-30).sum() <= max(1e-3 * err.size, 2)
     del b
     torch.cuda.empty_cache()

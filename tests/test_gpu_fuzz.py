@@ -12,10 +12,13 @@ the mean load (heavy drops) and far above it.
 import numpy as np
 import pytest
 
+import oracle
 from combine_moe_pw_b200 import synth
 from test_gpu_parity import _inputs, check_full, run_gpu
 
 N_CASES = 24
+N_BACKWARD = 12
+N_PROJECT = 12
 
 
 def random_workload(i: int) -> synth.Workload:
@@ -57,3 +60,40 @@ def test_random_config_full_parity(i):
     lg, x, s = _inputs(w)
     b, st = run_gpu(w, lg, x, s)
     check_full(w, lg, x, s, b, st)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("i", range(N_BACKWARD))
+def test_random_config_backward(i):
+    """The backward (combine, expert op, pack) on further seeded draws, with
+    the bounds of tests/test_gpu_backward.py."""
+    from test_gpu_backward import check_backward, run_both
+    w = random_workload(N_CASES + i)
+    b, st, r, ob, dout = run_both(w)
+    check_backward(w, b, st, r, ob, dout)
+
+
+def random_gemm(i: int):
+    rng = np.random.default_rng(9000 + i)
+    return (int(rng.integers(1, 700)), 8 * int(rng.integers(1, 130)),
+            8 * int(rng.integers(1, 260)))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("i", range(N_PROJECT))
+def test_random_projection(i):
+    """moe_pw_project on seeded shapes (M 1..699, N and K multiples of 8 up to
+    1032 and 2072: ragged row, column and K tails of the 256-row pair tiles),
+    with the bound of tests/test_gpu_project.py; bf16 codes may differ from
+    the oracle's (which sums in double) on at most 2% of the elements or 3 of
+    them, whichever is more."""
+    from test_gpu_project import _f64, gpu_project
+    M, N, K = random_gemm(i)
+    A = synth.matrix_bf16(M, K, 1.0, 50 + i)
+    Bt = synth.matrix_bf16(N, K, K ** -0.5, 80 + i)
+    C, _ = gpu_project(A, Bt)
+    Cr, Ce, mag = oracle.project(A, Bt, exact=True)
+    got = _f64(C)
+    assert np.all(np.isfinite(got))
+    assert np.all(np.abs(got - Ce) <= 2.0 ** -8 * np.abs(Ce) + 2.0 ** -20 * mag + 1e-30)
+    assert (C != Cr).sum() <= max(0.02 * C.size, 3)
