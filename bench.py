@@ -195,6 +195,31 @@ def alg_bytes(w, stats, C_s):
             "expert": 2 * D * K + 8 * S + S * (2 * D + 4)}
 
 
+def metric_bytes(w, stats, C_s):
+    """B_alg of the metric: route + dispatch + combine as the method defines
+    them (what it must move; the exchange moves nothing):
+      route     4TE + 8Tk                      logits in; ids and gates out
+      dispatch  4Tk + 2TD + S(2D+4) + 4Tk + 8S ids in; x rows in; pool rows and
+                                               headers out; slot map out;
+                                               headers in, receiver rows out
+      combine   8Tk + 4K_s + 2DK + 4TD         slot map and gates in; return
+                                               headers of the sender-kept
+                                               assignments in; kept rows in;
+                                               fp32 out
+    with S pool slots, K_s rows the sender kept and K rows the receiver kept.
+    The per-kernel figures of alg_bytes add the metadata each separate kernel
+    reads again (the pack's slot map and ids), which a fused dispatch would
+    not; the metric leaves those out."""
+    T, E, k, D = w.T, w.E, w.k, w.D
+    S = w.R * w.R * w.W * C_s if w.mode == 0 else T * k
+    K_s = T * k - stats.sender_dropped
+    K = stats.kept
+    route = 4 * T * E + 8 * T * k
+    dispatch = 4 * T * k + 2 * T * D + S * (2 * D + 4) + 4 * T * k + 8 * S
+    combine = 8 * T * k + 4 * K_s + 2 * D * K + 4 * T * D
+    return route + dispatch + combine
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons during the timed region (reads only)."""
 
@@ -459,7 +484,7 @@ def main():
     total_ms, dc_ms = max_over_ranks([total_ms, dc_ms], world, dev)
     value = throughput(w.T * w.k, a.steps, world, dc_ms)
     ab = alg_bytes(w, st, sizes.C_s)
-    b_alg = sum(ab[n] for n in dc_stages)
+    b_alg = metric_bytes(w, st, sizes.C_s)
     peak, peak_kind = measured_peaks()
     gbs = b_alg * a.steps / (dc_ms / 1e3) / 1e9
     stage_ms = {n: statistics.mean(v) for n, v in per_stage.items()}

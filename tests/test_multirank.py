@@ -63,3 +63,30 @@ def test_reference_arm_other_ranks_do_no_work(monkeypatch, capsys):
                                       "--steps", "1", "--warmup", "0"])
     bench.main()
     assert capsys.readouterr().out == ""
+
+
+def test_metric_bytes_match_the_definition_and_the_rack_upper_bound():
+    """B_alg of the metric, written out term by term from its definition, and
+    its value at K = T k for the rack batch (262,144 x 3072, C_s = 188):
+    32,399,360,000 bytes, the 32.40 GB upper bound of the scope table."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from combine_moe_pw_b200 import synth
+
+    class St:
+        sender_dropped = 0
+        kept = 0
+
+    w = synth.WORKLOADS["rack"]
+    T, E, k, D = w.T, w.E, w.k, w.D
+    st = St()
+    st.kept = T * k
+    assert bench.metric_bytes(w, st, 188) == 32_399_360_000
+    # with drops: every term that depends on K_s or K moves by its row bytes
+    st.sender_dropped, st.kept = 1000, T * k - 1500
+    assert bench.metric_bytes(w, st, 188) == 32_399_360_000 - 4 * 1000 - 2 * D * 1500
+    # the per-kernel figures add only the pack's second read of ids and slot map
+    ab = bench.alg_bytes(w, st, 188)
+    dc = sum(ab[n] for n in ("route", "assign", "pack", "bucket", "combine"))
+    assert dc - bench.metric_bytes(w, st, 188) == 8 * T * k
