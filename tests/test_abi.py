@@ -127,3 +127,16 @@ def test_misaligned_pointers_rejected_before_any_launch(lib):
     with pytest.raises(mp.MoePwError) as ei:
         mp.moe_pw_selftest_wait_timeout(good + 4, 16, stream=0)
     assert ei.value.code == mp.MOE_PW_EUNSUPPORTED
+
+
+@pytest.mark.parametrize("k,chunks_per_source", [(1, 1), (8, 1), (32, 4)])
+def test_workspace_follows_the_chunk_rule(lib, k, chunks_per_source):
+    """Ranking chunks hold 2048 assignments (2048 // k tokens, never more than
+    a source's tokens): the workspace is the per-chunk counts plus the
+    per-source totals, each padded to 256 bytes."""
+    base = mp.Config.from_workload(synth.WORKLOADS["tiny"])  # 8 sources x 256 tokens
+    cfg = mp.Config(**{**base.__dict__, "k": k})
+    s = mp.moe_pw_plan(cfg)
+    bins = cfg.R * cfg.W
+    pad = lambda b: (b + 255) // 256 * 256
+    assert s.workspace_bytes == pad(4 * cfg.R * chunks_per_source * bins) + pad(4 * cfg.R * bins)
