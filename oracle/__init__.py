@@ -100,6 +100,9 @@ def _configure(lib):
     lib.orc_bucket.argtypes = [gp, vp, vp, vp, vp, vp, vp]
     lib.orc_bucket.restype = i64
     lib.orc_assign_ragged.argtypes = [gp, vp, vp, vp, vp, vp]
+    lib.orc_bucket_ragged.argtypes = [gp, i64, vp, vp, vp, vp]
+    lib.orc_kept.argtypes = [gp, vp]
+    lib.orc_kept.restype = i64
     lib.orc_expert_pooled.argtypes = [gp, i64, vp, vp, vp, vp, vp, vp]
     lib.orc_expert_ragged.argtypes = [gp, i64, vp, vp, vp, vp, vp]
     lib.orc_combine.argtypes = [gp, vp, vp, vp, vp, vp]
@@ -148,6 +151,16 @@ def _c(a, dtype) -> np.ndarray:
     return np.ascontiguousarray(a, dtype=dtype)
 
 
+# Integer outputs are handed to the C code pre-filled with this value, so an
+# entry that a C function forgets to write cannot pass for a plausible one
+# (np.empty could hold zeros or -1 by chance).
+POISON = -0x5A5A5A5B
+
+
+def _out_i32(shape) -> np.ndarray:
+    return np.full(shape, POISON, np.int32)
+
+
 def capacity(T: int, T_s: int, E: int, k: int, P: int, cf_send_pct: int, cf_recv_pct: int):
     """(C_s, C_r) as defined in oracle.c (ceil of factor x uniform-routing mean)."""
     cs, cr = ctypes.c_int64(), ctypes.c_int64()
@@ -168,7 +181,7 @@ def geom_for(w, T: int | None = None, T_s: int | None = None) -> Geom:
 
 def route(g: Geom, logits: np.ndarray):
     lg = _c(logits, np.float32).reshape(g.T, g.E)
-    idx = np.empty((g.T, g.k), np.int32)
+    idx = _out_i32((g.T, g.k))
     gates = np.empty((g.T, g.k), np.float64)
     gc = g.c()
     _load().orc_route(ctypes.byref(gc), _p(lg), _p(idx), _p(gates))
@@ -177,9 +190,9 @@ def route(g: Geom, logits: np.ndarray):
 
 def assign_pooled(g: Geom, idx: np.ndarray):
     idx = _c(idx, np.int32)
-    slot_map = np.empty((g.T, g.k), np.int32)
-    occ = np.empty((g.n_src, g.R, g.W), np.int32)
-    slot_tok = np.empty((g.n_slots,), np.int32)
+    slot_map = _out_i32((g.T, g.k))
+    occ = _out_i32((g.n_src, g.R, g.W))
+    slot_tok = _out_i32((g.n_slots,))
     gc = g.c()
     dropped = _load().orc_assign_pooled(ctypes.byref(gc), _p(idx), _p(slot_map), _p(occ),
                                         _p(slot_tok))
@@ -188,10 +201,10 @@ def assign_pooled(g: Geom, idx: np.ndarray):
 
 def assign_ragged(g: Geom, idx: np.ndarray):
     idx = _c(idx, np.int32)
-    slot_map = np.empty((g.T, g.k), np.int32)
-    row_off = np.empty((g.E + 1,), np.int32)
-    row_cnt = np.empty((g.E,), np.int32)
-    slot_tok = np.empty((g.T * g.k,), np.int32)
+    slot_map = _out_i32((g.T, g.k))
+    row_off = _out_i32((g.E + 1,))
+    row_cnt = _out_i32((g.E,))
+    slot_tok = _out_i32((g.T * g.k,))
     gc = g.c()
     _load().orc_assign_ragged(ctypes.byref(gc), _p(idx), _p(slot_map), _p(row_off),
                               _p(row_cnt), _p(slot_tok))
@@ -201,7 +214,7 @@ def assign_ragged(g: Geom, idx: np.ndarray):
 def pack(g: Geom, n_slots: int, x: np.ndarray, idx: np.ndarray, slot_map: np.ndarray):
     x = _c(x, np.uint16)
     pool_x = np.empty((n_slots, g.D), np.uint16)
-    pool_hdr = np.empty((n_slots,), np.int32)
+    pool_hdr = _out_i32((n_slots,))
     gc = g.c()
     _load().orc_pack(ctypes.byref(gc), n_slots, _p(x), _p(_c(idx, np.int32)),
                      _p(_c(slot_map, np.int32)), _p(pool_x), _p(pool_hdr))
@@ -209,18 +222,36 @@ def pack(g: Geom, n_slots: int, x: np.ndarray, idx: np.ndarray, slot_map: np.nda
 
 
 def pack_headers(g: Geom, n_slots: int, idx: np.ndarray, slot_map: np.ndarray) -> np.ndarray:
-    pool_hdr = np.empty((n_slots,), np.int32)
+    pool_hdr = _out_i32((n_slots,))
     gc = g.c()
     _load().orc_pack_headers(ctypes.byref(gc), n_slots, _p(_c(idx, np.int32)),
                              _p(_c(slot_map, np.int32)), _p(pool_hdr))
     return pool_hdr
 
 
+def kept(g: Geom, bucket_cnt: np.ndarray) -> int:
+    """Rows every expert accepted (the drop statistics' "kept")."""
+    gc = g.c()
+    return int(_load().orc_kept(ctypes.byref(gc), _p(_c(bucket_cnt, np.int32))))
+
+
+def bucket_ragged(g: Geom, row_hdr: np.ndarray):
+    """Dropless receiver: (recv_row, arrivals, bucket_cnt) of every row."""
+    row_hdr = _c(row_hdr, np.int32)
+    recv_row = _out_i32((row_hdr.size,))
+    arrivals = _out_i32((g.E,))
+    bucket_cnt = _out_i32((g.E,))
+    gc = g.c()
+    _load().orc_bucket_ragged(ctypes.byref(gc), row_hdr.size, _p(row_hdr), _p(recv_row),
+                              _p(arrivals), _p(bucket_cnt))
+    return recv_row, arrivals, bucket_cnt
+
+
 def bucket(g: Geom, pool_hdr: np.ndarray, occ: np.ndarray):
-    recv_row = np.empty((g.n_slots,), np.int32)
-    bucket_slot = np.empty((g.E, g.C_r), np.int32)
-    arrivals = np.empty((g.E,), np.int32)
-    bucket_cnt = np.empty((g.E,), np.int32)
+    recv_row = _out_i32((g.n_slots,))
+    bucket_slot = _out_i32((g.E, g.C_r))
+    arrivals = _out_i32((g.E,))
+    bucket_cnt = _out_i32((g.E,))
     gc = g.c()
     dropped = _load().orc_bucket(ctypes.byref(gc), _p(_c(pool_hdr, np.int32)),
                                  _p(_c(occ, np.int32)), _p(recv_row), _p(bucket_slot),
@@ -231,7 +262,7 @@ def bucket(g: Geom, pool_hdr: np.ndarray, occ: np.ndarray):
 def expert_pooled(g: Geom, pool_x, bucket_slot, bucket_cnt, scale):
     n = pool_x.shape[0]
     ret_x = np.empty_like(pool_x)
-    ret_hdr = np.empty((n,), np.int32)
+    ret_hdr = _out_i32((n,))
     gc = g.c()
     _load().orc_expert_pooled(ctypes.byref(gc), n, _p(_c(pool_x, np.uint16)),
                               _p(_c(bucket_slot, np.int32)), _p(_c(bucket_cnt, np.int32)),
@@ -242,7 +273,7 @@ def expert_pooled(g: Geom, pool_x, bucket_slot, bucket_cnt, scale):
 def expert_ragged(g: Geom, rows, row_hdr, scale):
     n = rows.shape[0]
     ret_x = np.empty_like(rows)
-    ret_hdr = np.empty((n,), np.int32)
+    ret_hdr = _out_i32((n,))
     gc = g.c()
     _load().orc_expert_ragged(ctypes.byref(gc), n, _p(_c(rows, np.uint16)),
                               _p(_c(row_hdr, np.int32)), _p(_c(scale, np.float32)),
@@ -291,11 +322,9 @@ def run_headers(w, logits: np.ndarray) -> dict:
         r["slot_map"], r["row_off"], r["row_cnt"], r["slot_tok"] = assign_ragged(g, r["idx"])
         n_rows = g.T * g.k
         r["pool_hdr"] = pack_headers(g, n_rows, r["idx"], r["slot_map"])
-        r["recv_row"] = (np.arange(n_rows, dtype=np.int64)
-                         - np.repeat(r["row_off"][:-1], r["row_cnt"])).astype(np.int32)
+        r["recv_row"], r["arrivals"], r["bucket_cnt"] = bucket_ragged(g, r["pool_hdr"])
         r["sender_dropped"] = r["receiver_dropped"] = 0
-        r["arrivals"] = r["bucket_cnt"] = r["row_cnt"]
-    r["kept"] = int(np.asarray(r["bucket_cnt"], np.int64).sum())
+    r["kept"] = kept(g, r["bucket_cnt"])
     return r
 
 
@@ -406,15 +435,13 @@ def run(w, logits: np.ndarray, x: np.ndarray, scale: np.ndarray, T: int | None =
         r["slot_map"], r["row_off"], r["row_cnt"], r["slot_tok"] = assign_ragged(g, r["idx"])
         n_rows = g.T * g.k
         r["pool_x"], r["pool_hdr"] = pack(g, n_rows, xx, r["idx"], r["slot_map"])
-        r["recv_row"] = (np.arange(n_rows, dtype=np.int64)
-                         - np.repeat(r["row_off"][:-1], r["row_cnt"])).astype(np.int32)
+        r["recv_row"], r["arrivals"], r["bucket_cnt"] = bucket_ragged(g, r["pool_hdr"])
         r["sender_dropped"] = r["receiver_dropped"] = 0
-        r["arrivals"] = r["bucket_cnt"] = r["row_cnt"]
         r["ret_x"], r["ret_hdr"] = expert_ragged(g, r["pool_x"], r["pool_hdr"], scale)
     res = combine(g, r["ret_x"], r["ret_hdr"], r["slot_map"], r["gates"], with_mag=with_mag)
     if with_mag:
         r["out"], r["mag"] = res
     else:
         r["out"] = res
-    r["kept"] = int(np.asarray(r["bucket_cnt"], np.int64).sum())
+    r["kept"] = kept(g, r["bucket_cnt"])
     return r

@@ -288,6 +288,18 @@ int64_t orc_bucket(const orc_geom *g, const int32_t *pool_hdr, const int32_t *oc
     return dropped;
 }
 
+/*
+ * [P1-2] the drops are reported apart; what the receivers accepted is the sum
+ * of the bucket fills.  With the two drop counts it accounts for every one of
+ * the T*k assignments.
+ */
+int64_t orc_kept(const orc_geom *g, const int32_t *bucket_cnt)
+{
+    int64_t kept = 0;
+    for (int32_t e = 0; e < g->E; ++e) kept += bucket_cnt[e];
+    return kept;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Dropless ragged mode.                                                     */
 /* ------------------------------------------------------------------------ */
@@ -320,6 +332,29 @@ void orc_assign_ragged(const orc_geom *g, const int32_t *idx, int32_t *slot_map,
         }
     }
     free(next);
+}
+
+/*
+ * Receiver side of the dropless mode ([P1-4]: every row reaches its expert,
+ * nothing is capped).  Like the pooled receiver, the rows are walked in the
+ * order they arrive (row 0 .. n_rows-1) and each one takes the next free row
+ * of its expert's bucket: recv_row[q] = number of earlier rows whose header
+ * names the same expert.  Rows with header -1 (none in a complete batch) get
+ * -1.  arrivals[e] = bucket_cnt[e] = rows of expert e (no receiver cap).
+ */
+void orc_bucket_ragged(const orc_geom *g, int64_t n_rows, const int32_t *row_hdr,
+                       int32_t *recv_row, int32_t *arrivals, int32_t *bucket_cnt)
+{
+    for (int32_t e = 0; e < g->E; ++e) arrivals[e] = 0;
+    for (int64_t q = 0; q < n_rows; ++q) {
+        const int32_t e = row_hdr[q];
+        if (e < 0) {
+            recv_row[q] = -1;
+            continue;
+        }
+        recv_row[q] = arrivals[e]++;
+    }
+    for (int32_t e = 0; e < g->E; ++e) bucket_cnt[e] = arrivals[e];
 }
 
 /* ------------------------------------------------------------------------ */

@@ -16,6 +16,7 @@ from combine_moe_pw_b200 import synth
 import test_oracle_backward as tb
 import test_oracle_combine as tc
 import test_oracle_dispatch as td
+import test_oracle_headers as th
 import test_oracle_route as tr
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "oracle.c")
@@ -82,6 +83,15 @@ MUTANTS = [
     ("combine_shifted_gate", "const double gj = gates[t * g->k + j];\n            for (int64_t i = 0; i < D; ++i) o[i] +=",
      "const double gj = gates[t * g->k + (j + 1) % g->k];\n            for (int64_t i = 0; i < D; ++i) o[i] +=",
      lambda: tc.test_combine_matches_einsum(_tiny_run())),
+    ("pack_headers_writes_rank", "if (slot >= 0) pool_hdr[slot] = idx[t * g->k + j];",
+     "if (slot >= 0) pool_hdr[slot] = j;",
+     lambda: th.test_run_headers_equals_run("tiny")),
+    ("pack_headers_skips_empty_reset", "for (int64_t q = 0; q < n_slots; ++q) pool_hdr[q] = -1;",
+     "",
+     lambda: th.test_run_headers_equals_run("tiny")),
+    ("ragged_receiver_counts_from_one", "recv_row[q] = arrivals[e]++;",
+     "recv_row[q] = ++arrivals[e];",
+     lambda: th.test_ragged_receiver_rows_brute_force()),
     ("ragged_rows_by_token_desc", "const int32_t row = next[e]++;",
      "const int32_t row = row_off[e] + row_cnt[e] - 1 - (next[e]++ - row_off[e]);",
      lambda: td.test_ragged_assignment()),
