@@ -129,7 +129,7 @@ const char *moe_pw_strerror(int code)
     case MOE_PW_EUNSUPPORTED: return "shape or alignment not supported by this build";
     case MOE_PW_ECUDA: return "CUDA runtime or launch error";
     case MOE_PW_EDEVICE: return "a kernel flagged a violation (see counters.error)";
-    case MOE_PW_ENOMEM: return "buffers exceed the memory budget";
+    case MOE_PW_ENOMEM: return "buffers exceed the memory budget or the built-in scratch limit";
     default: return "unknown error code";
     }
 }
@@ -364,7 +364,8 @@ int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint1
 }
 
 int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
-                 moe_pw_drop_stats *host_out, cudaStream_t stream)
+                 const int32_t *expert_counts, moe_pw_drop_stats *host_out,
+                 int32_t *host_expert_counts, cudaStream_t stream)
 {
     Geo g;
     int rc = make_geo(cfg, &g);
@@ -372,6 +373,10 @@ int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
     if (!counters || !host_out) return MOE_PW_EINVAL;
     moe_pw_counters c;
     if (cudaMemcpyAsync(&c, counters, sizeof(c), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return MOE_PW_ECUDA;
+    if (expert_counts && host_expert_counts &&
+        cudaMemcpyAsync(host_expert_counts, expert_counts, sizeof(int32_t) * 2 * size_t(g.E),
+                        cudaMemcpyDeviceToHost, stream) != cudaSuccess)
         return MOE_PW_ECUDA;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_PW_ECUDA;
     host_out->assignments = g.T * g.k;
@@ -405,22 +410,18 @@ namespace {
 constexpr size_t NOALLOC_SCRATCH_BYTES = MOE_PW_NOALLOC_SCRATCH_BYTES;
 __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch, looked up once per device with that
-// device current (in host code the symbol's name is only a host-side handle).
-std::mutex g_noalloc_mu;
-void *g_noalloc_addr[64];
-
+// Device address of g_noalloc_scratch in the current device's context.  In
+// host code the symbol's name is only a host-side handle, so the address is
+// looked up (cudaGetSymbolAddress, with the target device current) on every
+// call rather than cached: a cached address would outlive a cudaDeviceReset
+// or belong to another context made current on the same device.  The lookup
+// allocates nothing; the first one on a device also loads this library's
+// device code there.
 int noalloc_scratch(void **out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_PW_ECUDA;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_PW_ECUDA;
-        g_noalloc_addr[dev] = p;
-    }
-    *out = g_noalloc_addr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_PW_ECUDA;
+    *out = p;
     return MOE_PW_OK;
 }
 

@@ -145,7 +145,16 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
         const uint32_t parity = uint32_t((i / NS) & 1);
         const bool landed = mbar_wait_bounded(&bar[s], parity, WAIT_LIMIT);
         if (!__all_sync(FULL_MASK, landed)) {
+            // Give up on this warp's rows, but not on its own copies: the
+            // loads already issued (tokens i .. last, one per stage, each on
+            // its own barrier phase) still write this CTA's shared memory, so
+            // wait for each of them before going on, within one more
+            // WAIT_LIMIT polls in all.
             ok = false;
+            const int64_t last = i < LAG ? (n < NS ? n : NS) - 1
+                                         : (i - 1 - LAG + NS < n ? i - 1 - LAG + NS : n - 1);
+            for (int64_t ii = i; ii <= last; ++ii)
+                mbar_wait_bounded(&bar[ii % NS], uint32_t((ii / NS) & 1), WAIT_LIMIT / NS);
             break;
         }
         if (slot >= p.n_slots) {

@@ -15,6 +15,7 @@ import ctypes
 import os
 from dataclasses import dataclass
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,7 +79,7 @@ SIGNATURES = {
     "moe_pw_dispatch_backward": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_project": [_VP, _VP, _VP, _I64, ctypes.c_int32, ctypes.c_int32, _VP, _VP],
     "moe_pw_project_pack": [_CFG, _VP, _VP, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
-    "moe_pw_stats": [_CFG, _VP, ctypes.POINTER(moe_pw_drop_stats), _VP],
+    "moe_pw_stats": [_CFG, _VP, _VP, ctypes.POINTER(moe_pw_drop_stats), _VP, _VP],
     "moe_pw_selftest_wait_timeout": [_VP, ctypes.c_int32, _VP],
 }
 
@@ -265,11 +266,20 @@ def moe_pw_project_pack(cfg, h, w_down_t, model_width: int, idx, slot_map, occ, 
         _ptr(occ), _ptr(pool_x), _ptr(pool_hdr), _ptr(counters), _stream(stream)))
 
 
-def moe_pw_stats(cfg, counters, stream=None, raise_on_device_error: bool = True) -> moe_pw_drop_stats:
+def moe_pw_stats(cfg, counters, stream=None, raise_on_device_error: bool = True,
+                 expert_counts=None, host_expert_counts=None) -> moe_pw_drop_stats:
+    """Drop statistics.  With ``expert_counts`` (device i32 [2, E]) and
+    ``host_expert_counts`` (a C-contiguous numpy int32 [2, E] array) the
+    per-expert arrivals and kept rows are copied into the latter as well."""
     c = _cfg(cfg)
     out = moe_pw_drop_stats()
-    rc = load_library().moe_pw_stats(ctypes.byref(c), _ptr(counters), ctypes.byref(out),
-                                     _stream(stream))
+    hp = None
+    if host_expert_counts is not None:
+        assert host_expert_counts.dtype == np.int32 and host_expert_counts.flags.c_contiguous
+        assert host_expert_counts.size >= 2 * c.E
+        hp = host_expert_counts.ctypes.data
+    rc = load_library().moe_pw_stats(ctypes.byref(c), _ptr(counters), _ptr(expert_counts),
+                                     ctypes.byref(out), hp, _stream(stream))
     if rc == MOE_PW_EDEVICE and not raise_on_device_error:
         return out
     _check("moe_pw_stats", rc)
@@ -309,6 +319,7 @@ class Buffers:
         self.recv_row = torch.empty((s.n_slots,), dtype=i32, device=dev)
         self.bucket_slot = torch.empty((max(s.bucket_len, 1),), dtype=i32, device=dev)
         self.expert_counts = torch.empty((2, E), dtype=i32, device=dev)
+        self.host_expert_counts = np.zeros((2, E), np.int32)
         self.ret_x = torch.empty((s.n_slots, D), dtype=i16, device=dev)
         self.ret_hdr = torch.empty((s.n_slots,), dtype=i32, device=dev)
         self.out = torch.empty((T, D), dtype=f32, device=dev)
@@ -344,7 +355,10 @@ class Buffers:
                        self.counters, stream)
 
     def stats(self, stream=None, raise_on_device_error: bool = True) -> moe_pw_drop_stats:
-        return moe_pw_stats(self.cfg, self.counters, stream, raise_on_device_error)
+        """Drop statistics; the per-expert arrivals and kept rows land in
+        ``self.host_expert_counts`` (numpy int32 [2, E])."""
+        return moe_pw_stats(self.cfg, self.counters, stream, raise_on_device_error,
+                            self.expert_counts, self.host_expert_counts)
 
     def alloc_backward(self):
         """Gradient buffers: dout (input), d_ret / d_pool (gradient pools),

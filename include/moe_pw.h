@@ -94,7 +94,8 @@ extern "C" {
 #define MOE_PW_EUNSUPPORTED (-2)  /* shape or alignment this build does not handle */
 #define MOE_PW_ECUDA (-3)         /* a CUDA runtime call or a launch failed */
 #define MOE_PW_EDEVICE (-4)       /* a kernel flagged a violation (moe_pw_stats) */
-#define MOE_PW_ENOMEM (-5)        /* buffers exceed the caller's budget (moe_pw_plan) */
+#define MOE_PW_ENOMEM (-5)        /* buffers exceed the caller's budget (moe_pw_plan) or the
+                                     built-in scratch (moe_pw_assign_noalloc) */
 
 #define MOE_PW_POOLED 0
 #define MOE_PW_RAGGED 1
@@ -102,7 +103,12 @@ extern "C" {
 /* counters->error bits */
 #define MOE_PW_DEVERR_EXPERT_ID 1   /* idx entry outside [0, E) */
 #define MOE_PW_DEVERR_HEADER 2      /* pool header outside its (d, w) experts */
-#define MOE_PW_DEVERR_TIMEOUT 4     /* a bounded wait gave up */
+#define MOE_PW_DEVERR_TIMEOUT 4     /* a bounded wait gave up: that launch's outputs are
+                                       incomplete.  The kernel first waits, again with a
+                                       bound, for the copies it has in flight; if those
+                                       waits run out too, copies may still land after the
+                                       kernel ends, so treat the outputs (and, to be safe,
+                                       the context) as suspect and re-run the step */
 #define MOE_PW_DEVERR_SLOT 8        /* slot_map entry outside [-1, n_slots) */
 
 /* Problem description.  Limits of this build: 1 <= k <= 32, k <= E,
@@ -237,9 +243,10 @@ int moe_pw_bucket(const moe_pw_config *cfg, const int32_t *pool_hdr, const int32
  *     moe_pw_plan above the limit) is refused with MOE_PW_ENOMEM before any
  *     launch; the rack-scale batch (262,144 tokens, 64 ranks, 3 waves) needs
  *     under 1 MiB.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *   - Every call looks up the array's device address in the current
+ *     device's context (cudaGetSymbolAddress, with that device current); the
+ *     first call on a device also loads the library's device code there, so
+ *     make that first call before any stream capture.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents; nothing in it needs to start at zero (each call writes every
  *     entry it reads).  Calls whose kernels overlap on the GPU, such as calls
@@ -349,12 +356,16 @@ int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint1
 
 /*
  * Drop statistics (section 二: the two kinds of drop are reported apart).
- * Copies *counters (device) to *host_out (host memory) and synchronises the
+ * Copies *counters (device) to *host_out (host memory) and, when both
+ * expert_counts (device, i32 [2, E] as written by moe_pw_bucket) and
+ * host_expert_counts (host, i32 [2, E]) are given, the per-expert arrivals
+ * and kept rows too; either may be NULL to skip that copy.  Synchronises the
  * stream.  Returns MOE_PW_EDEVICE when a kernel flagged a violation (the
  * stats are still filled).
  */
 int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
-                 moe_pw_drop_stats *host_out, cudaStream_t stream);
+                 const int32_t *expert_counts, moe_pw_drop_stats *host_out,
+                 int32_t *host_expert_counts, cudaStream_t stream);
 
 /*
  * Self-test of failure detection (no counterpart on the pages): launches one

@@ -90,6 +90,9 @@ def check_full(w, lg, x, s, b, st):
     ec = _np(b.expert_counts)
     np.testing.assert_array_equal(ec[0], r["arrivals"])
     np.testing.assert_array_equal(ec[1], r["bucket_cnt"])
+    # the host copy moe_pw_stats made of the per-expert counts
+    np.testing.assert_array_equal(b.host_expert_counts[0], r["arrivals"])
+    np.testing.assert_array_equal(b.host_expert_counts[1], r["bucket_cnt"])
     np.testing.assert_array_equal(_u16(b.ret_x), r["ret_x"])
     np.testing.assert_array_equal(_np(b.ret_hdr), r["ret_hdr"])
     err = check_combine(_np(b.out), r["out"], r["mag"])
@@ -119,6 +122,9 @@ def check_sampled(w, lg, x, s, b, st, n_tok=1024, n_slot=8192, seed=0):
     ec = _np(b.expert_counts)
     np.testing.assert_array_equal(ec[0], r["arrivals"])
     np.testing.assert_array_equal(ec[1], r["bucket_cnt"])
+    # the host copy moe_pw_stats made of the per-expert counts
+    np.testing.assert_array_equal(b.host_expert_counts[0], r["arrivals"])
+    np.testing.assert_array_equal(b.host_expert_counts[1], r["bucket_cnt"])
     assert (st.sender_dropped, st.receiver_dropped, st.kept, st.error) == (
         r["sender_dropped"], r["receiver_dropped"], r["kept"], 0)
 
