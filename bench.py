@@ -268,24 +268,28 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def traffic_from_profiles(kernel: str):
-    """DRAM bytes per launch for ``kernel`` from a committed ncu summary, if the
-    kernel source is unchanged since the capture (sha256 recorded there)."""
+def traffic_from_profiles(kernel: str, alg_bytes: float):
+    """DRAM bytes per launch for ``kernel``, scaled from a committed small-case
+    ncu summary: the capture's dram__bytes_read.sum + dram__bytes_write.sum
+    over that launch's algorithmic bytes, times this launch's algorithmic
+    bytes (the kernel streams its rows once, so its traffic grows in
+    proportion).  None unless the kernel source is unchanged since the capture
+    (its sha256 is recorded there)."""
     import hashlib
     import re
-    prof = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
+    prof = os.path.join(ROOT, "profiles", f"{kernel}_small_case_traffic.txt")
     if not os.path.exists(prof):
         return None
     text = open(prof).read()
-    m_b = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
+    m_r = re.search(r"^traffic_per_algorithmic_byte:\s*([0-9.eE+]+)", text, re.M)
     m_h = re.search(r"^source_sha256:\s*([0-9a-f]+)", text, re.M)
     m_f = re.search(r"^source_file:\s*(\S+)", text, re.M)
-    if not (m_b and m_h and m_f):
+    if not (m_r and m_h and m_f):
         return None
     src = os.path.join(ROOT, m_f.group(1))
     if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != m_h.group(1):
         return None
-    return float(m_b.group(1))
+    return float(m_r.group(1)) * alg_bytes
 
 
 def host_cpu():
@@ -491,7 +495,7 @@ def main():
     dom = max(["pack", "combine"], key=lambda n: stage_ms[n])
     kname = {"pack": "pack_kernel", "combine": "combine_kernel"}[dom]
     achieved = ab[dom] / (stage_ms[dom] / 1e3) / 1e9
-    traffic = traffic_from_profiles(kname + "_" + a.workload)
+    traffic = traffic_from_profiles(kname, ab[dom])
 
     # backward (gradient of dispatch/combine), timed in its own loop
     bwd = None
@@ -632,7 +636,9 @@ def main():
             "stage_ms": stage_ms,
             "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                         "alg_bytes_per_launch": ab[dom], "peak_kind": peak_kind},
+                         "alg_bytes_per_launch": ab[dom], "peak_kind": peak_kind,
+                         "traffic_source": "32,768-token capture of the same kernel, scaled by "
+                                           "algorithmic bytes" if traffic else None},
             "gpu_launches": launches_per_step * a.steps,
             "graph": graph,
             "backward": bwd,
