@@ -61,6 +61,13 @@ def parse():
                     help="time only the tensor-core projections (profiling)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the batch's token count (profiling a smaller case)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism over the GPUs even at one GPU (the default for "
+                         "more than one): the R ranks split over the GPUs, the pools "
+                         "exchanged by the kernels' peer stores")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with several GPUs: an independent batch per GPU instead of one "
+                         "expert-parallel batch")
     return ap.parse_args()
 
 
@@ -132,7 +139,18 @@ def time_projection(w, dev, stream, steps: int, b=None):
         lat = torch.empty(T, D, dtype=torch.int16, device=dev)
         out["routed_layer_ms"] = timed(lambda: b.run_routed_layer(h, wd, wu, Dm, lat, y, stream))
         out["routed_layer_tokens_per_s"] = T / (out["routed_layer_ms"] / 1e3)
-        del lat
+        # merged with a shared-path output, sequential and with the combine
+        # and up-projection overlapped in 8192-token blocks
+        sh = torch.randn(T, Dm, device=dev, generator=g).to(torch.bfloat16).view(torch.int16)
+        out["routed_layer_merged_ms"] = timed(
+            lambda: b.run_routed_layer(h, wd, wu, Dm, lat, y, stream, shared_out=sh))
+        for chunk in (4096, 8192, 16384):
+            out[f"routed_layer_merged_pipelined_{chunk}_ms"] = timed(
+                lambda: b.run_routed_layer_pipelined(h, wd, wu, Dm, y, shared_out=sh,
+                                                     chunk_tokens=chunk, stream=stream))
+        out["routed_layer_merged_pipelined_ms"] = min(
+            out[f"routed_layer_merged_pipelined_{c}_ms"] for c in (4096, 8192, 16384))
+        del lat, sh
     del h, wd, wu, xl, y
     torch.cuda.empty_cache()
     return out
@@ -364,6 +382,145 @@ def config_of(w):
             "metric_scope": "route + assign + pack + bucket + combine; expert op timed apart"}
 
 
+NVLINK_PEER_GBS = 770.0  # measured peer copy per direction on this machine (900 nominal)
+
+
+def ep_link_bytes(share, D: int, n: int) -> int:
+    """Bytes one GPU sends to the other GPUs per step, per direction: its
+    pools' rows and headers (fixed shape, zero tails included) to the
+    destinations' GPUs, and the same volume of returned rows back; the pools
+    for its own experts stay in its memory (1/n of them)."""
+    return share.n_slots * (2 * D + 4) * (n - 1) // n
+
+
+def run_ep_bench(a, world: int, rank: int, local: int):
+    """Expert-parallel run: the rack-shaped batch is split over the GPUs by
+    rank, weak scaling (every GPU holds the single-GPU batch's token count,
+    so the whole batch has world x that many tokens over the same 64 ranks).
+    One step = route, assign, pack and send (per wave, overlapped with the
+    previous wave's bucketing and expert op, whose kernel returns the rows),
+    combine; barriers are one-element NCCL all-reduces on the step's stream."""
+    import torch
+    import torch.distributed as dist
+    from combine_moe_pw_b200 import ep
+    from combine_moe_pw_b200 import moe_pw as mp
+    from combine_moe_pw_b200 import synth
+
+    dev = torch.device("cuda", local)
+    base = synth.WORKLOADS[a.workload]
+    w = base.with_(T=(a.tokens or base.T) * world)
+    cfg = mp.Config.from_workload(w)
+    b = ep.EpBuffers(cfg, world, rank, dev)
+    t = b.share.token_range
+    b.logits.copy_(torch.from_numpy(synth.logits_rows(w, t.start, len(t))))
+    b.x.copy_(torch.from_numpy(synth.x_bf16_rows(w, t.start, len(t)).view(np.int16)))
+    b.scale.copy_(torch.from_numpy(synth.scales(w)))
+    torch.cuda.synchronize(dev)
+    links = ep.PeerLinks(b, dist.all_gather_object) if world > 1 else None
+    one = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def barrier(stream):
+        if world > 1:
+            with torch.cuda.stream(stream):
+                dist.all_reduce(one)
+
+    sa = torch.cuda.current_stream(dev)
+    sb = torch.cuda.Stream(dev)
+
+    def timed(overlap: bool, steps: int):
+        for _ in range(max(a.warmup, 3)):
+            ep.run_step(b, barrier, sa, sb, overlap)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(sa)
+        for _ in range(steps):
+            ep.run_step(b, barrier, sa, sb, overlap)
+        e1.record(sa)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / steps
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ms = timed(True, a.steps)
+    clocks = sampler.stop()
+    ms_one = timed(False, a.steps)
+    st = b.stats(sa)
+    counts = torch.tensor([st.assignments, st.kept, st.sender_dropped, st.receiver_dropped,
+                           st.error], dtype=torch.int64, device=dev)
+    if world > 1:
+        dist.all_reduce(counts)
+    ms, ms_one = max_over_ranks([ms, ms_one], world, dev)
+    TK, kept, sd, rd, err = [int(v) for v in counts.tolist()]
+    value = TK / (ms / 1e3)
+    link = ep_link_bytes(b.share, w.D, world)
+
+    # end to end: this GPU's inputs from pinned host memory, its output back
+    h_lg = b.logits.cpu().pin_memory()
+    h_x = b.x.cpu().pin_memory()
+    h_out = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
+
+    def e2e_step():
+        b.logits.copy_(h_lg, non_blocking=True)
+        b.x.copy_(h_x, non_blocking=True)
+        ep.run_step(b, barrier, sa, sb, True)
+        h_out.copy_(b.out, non_blocking=True)
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ke = min(a.e2e_steps or a.steps, 10)
+    e0.record(sa)
+    for _ in range(ke):
+        e2e_step()
+    e1.record(sa)
+    torch.cuda.synchronize(dev)
+    (e_ms,) = max_over_ranks([e0.elapsed_time(e1) / ke], world, dev)
+    if links is not None:
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        links.close()
+        dist.barrier()
+    if rank == 0:
+        cfg_out = config_of(w)
+        cfg_out.update({"parallelism": f"ep{world}", "tokens_per_gpu": len(t),
+                        "metric_scope": "route + assign + pack/send + bucket + expert op/return "
+                                        "+ combine: across GPUs the expert kernel carries the "
+                                        "return exchange, so it is inside the step"})
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": a.steps, "warmup": max(a.warmup, 3), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "payload_dtype": "bf16", "data": "synthetic", "config": cfg_out,
+            "drop_rate": {"sender": sd / TK, "receiver": rd / TK, "total": (sd + rd) / TK},
+            "roofline": {"bound": "nvlink", "achieved": 2 * link / (ms / 1e3) / 1e9,
+                         "peak": 2 * NVLINK_PEER_GBS, "unit": "GB/s",
+                         "frac": (2 * link / (ms / 1e3) / 1e9) / (2 * NVLINK_PEER_GBS),
+                         "traffic": None,
+                         "link_bytes_per_step_per_direction": link,
+                         "peak_kind": "measured peer copy, both directions"},
+            "ep": {"ms_per_step_waves_overlapped": ms, "ms_per_step_one_pack": ms_one,
+                   "barriers_per_step": len(ep.schedule(w.W, True)) - 1},
+            # per step: route, 3 assignment kernels, and per wave a pack, a
+            # bucketing and an expert kernel, then the combine (NCCL's own
+            # all-reduce kernels not counted)
+            "gpu_launches": (5 + 3 * w.W) * a.steps,
+            "clocks": clocks,
+            "e2e": {"value": TK / (e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": h_lg.numel() * 4 + h_x.numel() * 2,
+                    "d2h_bytes_per_step": h_out.numel() * 4, "ms_per_step": e_ms},
+            "cpu_baseline": None,
+            "kept": kept, "device_error": err,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     a = parse()
     if a.impl == "reference":
@@ -383,6 +540,20 @@ def main():
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+    if a.ep or (world > 1 and not a.replicas):
+        # the exchange stores into the other GPUs' memory: every pair of this
+        # node's GPUs must reach each other (NVLink / NVSwitch peer access)
+        peers_ok = all(torch.cuda.can_device_access_peer(local, j)
+                       for j in range(world) if j != local)
+        ok = torch.tensor([1 if peers_ok else 0], dtype=torch.int32, device=dev)
+        if world > 1:
+            dist.all_reduce(ok, op=dist.ReduceOp.MIN)
+        if int(ok.item()) == 1:
+            run_ep_bench(a, world, rank, local)
+            return
+        if rank == 0:
+            print("expert-parallel mode needs peer access between every pair of GPUs; "
+                  "running independent batches instead", file=sys.stderr, flush=True)
 
     base = synth.WORKLOADS[a.workload]
     if a.tokens:

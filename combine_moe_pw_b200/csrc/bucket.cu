@@ -23,6 +23,7 @@ struct BucketArgs {
     int32_t *expert_counts;
     moe_pw_counters *ctr;
     Geo g;
+    uint32_t wave_mask;  // waves whose blocks run
 };
 
 // One block per (destination d, wave w).  Its positions q = s * C_s + c run
@@ -83,13 +84,18 @@ __global__ void __launch_bounds__(BK_THREADS, 2) bucket_pooled(BucketArgs p)
     int32_t *row_sm = sm + BK_TILE / 4;              // [BK_TILE + BK_TILE / 32], padded
     int32_t *carry = row_sm + BK_TILE + BK_TILE / 32;  // [P]
     int32_t *wsum = carry + P;                       // [BK_THREADS / 32 + 1]
+    // block (d, w): d is this GPU's d-th destination rank (all of them on one
+    // GPU); its pools (s, d, w) for the R sources s sit at pool_s0 + s * pool_step
     const int dw = blockIdx.x;
     const int d = dw / p.g.W, w = dw - d * p.g.W;
-    const int32_t e0 = d * p.g.L + w * p.g.P;
+    if (!((p.wave_mask >> w) & 1u)) return;
+    const int32_t e_base = p.g.ep_g * p.g.Rn * p.g.L;  // first expert on this GPU
+    const int32_t E_out = p.g.Rn * p.g.L;              // experts of this GPU
+    const int32_t e0 = (p.g.ep_g * p.g.Rn + d) * p.g.L + w * p.g.P;
     const int64_t C_s = p.g.C_s, C_r = p.g.C_r;
     const int64_t npos = int64_t(R) * C_s;
-    const int64_t pool_s0 = int64_t(d) * p.g.W + w;  // pool (s, d, w) = pool_s0 + s * pool_step
-    const int64_t pool_step = int64_t(R) * p.g.W;
+    const int64_t pool_s0 = int64_t(d) * p.g.W + w;
+    const int64_t pool_step = int64_t(p.g.Rn) * p.g.W;
     for (int i = threadIdx.x; i < P; i += blockDim.x) carry[i] = 0;
 
     for (int64_t t0 = 0; t0 < npos; t0 += BK_TILE) {
@@ -111,7 +117,7 @@ __global__ void __launch_bounds__(BK_THREADS, 2) bucket_pooled(BucketArgs p)
                     cc[u] = uint32_t(q) - sq * Cs32;
                     const int64_t pool = pool_s0 + int64_t(sq) * pool_step;
                     slot[u] = uint32_t(pool * C_s + cc[u]);
-                    occ[u] = p.occ[pool];
+                    occ[u] = p.occ ? p.occ[pool] : 0;
                     hdr[u] = p.pool_hdr[slot[u]];
                 }
             }
@@ -120,7 +126,9 @@ __global__ void __launch_bounds__(BK_THREADS, 2) bucket_pooled(BucketArgs p)
                 const int j = j0 + u * BK_THREADS + threadIdx.x;
                 int pe = -1;
                 if (t0 + j < npos) {
-                    if (int32_t(cc[u]) < occ[u]) {
+                    // filled: below the pool's occupancy, or (no counts
+                    // exchanged) a header other than -1
+                    if (p.occ ? int32_t(cc[u]) < occ[u] : hdr[u] != -1) {
                         pe = hdr[u] - e0;
                         if (pe < 0 || pe >= P) {
                             set_error(p.ctr, MOE_PW_DEVERR_HEADER);
@@ -175,7 +183,7 @@ __global__ void __launch_bounds__(BK_THREADS, 2) bucket_pooled(BucketArgs p)
                 const int64_t slot = (pool_s0 + int64_t(sq) * pool_step) * C_s + c;
                 const int32_t row = row_sm[j + (j >> 5)];
                 p.recv_row[slot] = row;
-                if (row >= 0) p.bucket_slot[int64_t(e0 + pe) * C_r + row] = int32_t(slot);
+                if (row >= 0) p.bucket_slot[int64_t(e0 - e_base + pe) * C_r + row] = int32_t(slot);
             }
         }
         __syncthreads();  // pe_sm and row_sm are refilled by the next tile
@@ -184,12 +192,12 @@ __global__ void __launch_bounds__(BK_THREADS, 2) bucket_pooled(BucketArgs p)
     for (int pp = 0; pp < P; ++pp) {
         const int32_t arrivals = carry[pp];
         const int64_t kept = arrivals < C_r ? arrivals : C_r;
-        const int32_t e = e0 + pp;
+        const int32_t e = e0 - e_base + pp;  // index among this GPU's experts
         for (int64_t r = kept + threadIdx.x; r < C_r; r += blockDim.x)
             p.bucket_slot[int64_t(e) * C_r + r] = -1;
         if (threadIdx.x == 0) {
             p.expert_counts[e] = arrivals;
-            p.expert_counts[p.g.E + e] = int32_t(kept);
+            p.expert_counts[E_out + e] = int32_t(kept);
             if (arrivals > kept)
                 atomicAdd(&p.ctr->receiver_dropped, (unsigned long long)(arrivals - kept));
             atomicAdd(&p.ctr->kept, (unsigned long long)kept);
@@ -224,7 +232,7 @@ __global__ void bucket_ragged(BucketArgs p)
 
 cudaError_t launch_bucket(const Geo &g, const int32_t *pool_hdr, const int32_t *occ,
                           int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,
-                          moe_pw_counters *ctr, cudaStream_t st)
+                          moe_pw_counters *ctr, cudaStream_t st, uint32_t wave_mask)
 {
     BucketArgs p;
     p.pool_hdr = pool_hdr;
@@ -234,14 +242,16 @@ cudaError_t launch_bucket(const Geo &g, const int32_t *pool_hdr, const int32_t *
     p.expert_counts = expert_counts;
     p.ctr = ctr;
     p.g = g;
-    if (g.T == 0) return cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * 2 * g.E, st);
+    p.wave_mask = wave_mask;
+    if (g.T == 0 && g.ep_n == 1)
+        return cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * 2 * g.E, st);
     if (g.mode == MOE_PW_POOLED) {
         const size_t smem = BK_TILE + sizeof(int32_t) * (BK_TILE + BK_TILE / 32 + size_t(g.P) +
                                                          BK_THREADS / 32 + 1);
         const cudaError_t aerr = cudaFuncSetAttribute(
             bucket_pooled, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (aerr != cudaSuccess) return aerr;
-        bucket_pooled<<<g.R * g.W, BK_THREADS, smem, st>>>(p);
+        bucket_pooled<<<g.Rn * g.W, BK_THREADS, smem, st>>>(p);
     } else {
         DevInfo di;
         if (dev_info(&di) != 0) return cudaErrorUnknown;

@@ -28,6 +28,16 @@ struct Geo {
     int64_t chunk_tokens;   // tokens per chunk
     int32_t chunks_per_group;
     int32_t n_chunks;
+    // expert parallelism over GPUs: this GPU is ep_g of ep_n and hosts the
+    // Rn = R / ep_n logical ranks [ep_g * Rn, (ep_g + 1) * Rn) (one GPU:
+    // ep_n = 1, ep_g = 0, Rn = R)
+    int32_t ep_n, ep_g, Rn;
+};
+
+// Peer tables of an expert-parallel run, passed to the kernels by value.
+struct EpRows {
+    uint16_t *x[MOE_PW_EP_MAX_GPUS];
+    int32_t *hdr[MOE_PW_EP_MAX_GPUS];
 };
 
 // Per-device attributes, cached on first use.
@@ -42,15 +52,23 @@ cudaError_t launch_route(const Geo &g, const float *logits, int32_t *idx, float 
                          cudaStream_t st);
 cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, int32_t *occ,
                           moe_pw_counters *ctr, void *ws, cudaStream_t st);
+// ep (optional): the receive pools of every GPU of an expert-parallel run;
+// rows then go to the destination's GPU, only for waves in wave_mask.
 cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
                         const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
-                        int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st);
+                        int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st,
+                        const EpRows *ep = nullptr, uint32_t wave_mask = ~0u);
+// occ == nullptr: an empty slot is one whose header is -1 (expert-parallel
+// receive pools, where no counts are exchanged).
 cudaError_t launch_bucket(const Geo &g, const int32_t *pool_hdr, const int32_t *occ,
                           int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,
-                          moe_pw_counters *ctr, cudaStream_t st);
+                          moe_pw_counters *ctr, cudaStream_t st, uint32_t wave_mask = ~0u);
+// ep (optional): the return pools of every GPU; results then go to the
+// source's GPU, only for waves in wave_mask.
 cudaError_t launch_expert(const Geo &g, const uint16_t *pool_x, const int32_t *pool_hdr,
                           const int32_t *recv_row, const float *scale, uint16_t *ret_x,
-                          int32_t *ret_hdr, cudaStream_t st);
+                          int32_t *ret_hdr, cudaStream_t st, const EpRows *ep = nullptr,
+                          uint32_t wave_mask = ~0u);
 cudaError_t launch_combine(const Geo &g, const uint16_t *ret_x, const int32_t *ret_hdr,
                            const int32_t *slot_map, const float *gates, float *out,
                            moe_pw_counters *ctr, cudaStream_t st);
@@ -67,7 +85,8 @@ cudaError_t launch_combine_backward(const Geo &g, const float *dout, const uint1
 cudaError_t launch_gemm(const uint16_t *A, const uint16_t *Bt, int64_t M, int32_t N, int32_t K,
                         int32_t mode, uint16_t *C, int64_t ldc, const int32_t *slot_map,
                         const int32_t *idx, int32_t topk, uint16_t *pool_x, int32_t *pool_hdr,
-                        int64_t n_slots, moe_pw_counters *ctr, cudaStream_t st);
+                        int64_t n_slots, moe_pw_counters *ctr, cudaStream_t st,
+                        const uint16_t *add = nullptr);
 
 // Workspace layout of the ranking pass.
 inline int64_t align256(int64_t b) { return (b + 255) & ~int64_t(255); }
@@ -189,6 +208,39 @@ __device__ __forceinline__ uint64_t policy_evict_last()
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
     return p;
+}
+
+// Expert-parallel relabelling of a pool slot (32-bit: slot ids fit in int32).
+// Send slot q = ((s_loc*R + d)*W + w)*C_s + c of GPU g -> the destination's
+// GPU h = d / Rn and its receive slot ((s*Rn + d_loc)*W + w)*C_s + c.
+__device__ __forceinline__ uint32_t ep_send_to_recv(const Geo &g, uint32_t q, int &h, int &w)
+{
+    const uint32_t Cs = uint32_t(g.C_s), W = uint32_t(g.W), R = uint32_t(g.R),
+                   Rn = uint32_t(g.Rn);
+    const uint32_t c = q % Cs, r1 = q / Cs;
+    w = int(r1 % W);
+    const uint32_t r2 = r1 / W;
+    const uint32_t d = r2 % R, s_loc = r2 / R;
+    h = int(d / Rn);
+    const uint32_t d_loc = d - uint32_t(h) * Rn;
+    const uint32_t s = uint32_t(g.ep_g) * Rn + s_loc;
+    return ((s * Rn + d_loc) * W + uint32_t(w)) * Cs + c;
+}
+
+// Receive slot rq = ((s*Rn + d_loc)*W + w)*C_s + c of GPU g -> the source's
+// GPU h = s / Rn and its send slot ((s_loc*R + d)*W + w)*C_s + c.
+__device__ __forceinline__ uint32_t ep_recv_to_send(const Geo &g, uint32_t rq, int &h, int &w)
+{
+    const uint32_t Cs = uint32_t(g.C_s), W = uint32_t(g.W), R = uint32_t(g.R),
+                   Rn = uint32_t(g.Rn);
+    const uint32_t c = rq % Cs, r1 = rq / Cs;
+    w = int(r1 % W);
+    const uint32_t r2 = r1 / W;
+    const uint32_t d_loc = r2 % Rn, s = r2 / Rn;
+    h = int(s / Rn);
+    const uint32_t s_loc = s - uint32_t(h) * Rn;
+    const uint32_t d = uint32_t(g.ep_g) * Rn + d_loc;
+    return ((s_loc * R + d) * W + uint32_t(w)) * Cs + c;
 }
 
 __device__ __forceinline__ void set_error(moe_pw_counters *ctr, int bits)

@@ -10,6 +10,8 @@
 // stores, four chunks in flight per lane.
 #include <cuda_bf16.h>
 
+#include <cstring>
+
 #include "common.cuh"
 
 namespace moe_pw {
@@ -24,23 +26,48 @@ __device__ __forceinline__ uint32_t scale_pair(uint32_t packed, float s)
     return *reinterpret_cast<const uint32_t *>(&r);
 }
 
-__global__ void __launch_bounds__(256) expert_kernel(const uint4 *__restrict__ pool_x,
-                                                     const int32_t *__restrict__ pool_hdr,
-                                                     const int32_t *__restrict__ recv_row,
-                                                     const float *__restrict__ scale,
-                                                     uint4 *__restrict__ ret_x,
-                                                     int32_t *__restrict__ ret_hdr,
-                                                     int64_t n_slots, int cpr, int E)
+// Where the result of slot `slot` goes: the same slot of the local return
+// pool, or (expert-parallel runs) the source's send slot in the return pool of
+// the source's GPU.
+struct ExpertArgs {
+    const uint4 *pool_x;
+    const int32_t *pool_hdr;
+    const int32_t *recv_row;
+    const float *scale;
+    uint4 *ret_x;
+    int32_t *ret_hdr;
+    int64_t n_slots;
+    int cpr;
+    int E;
+    uint32_t wave_mask;
+    Geo geo;
+    EpRows ep;
+};
+
+template <bool EP>
+__global__ void __launch_bounds__(256) expert_kernel(ExpertArgs a)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarp = (int64_t(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t slot = warp; slot < n_slots; slot += nwarp) {
-        const int32_t e = pool_hdr[slot];
-        const bool keep = recv_row[slot] >= 0 && e >= 0 && e < E;
-        const float s = keep ? scale[e] : 0.0f;
-        const uint4 *src = pool_x + slot * cpr;
-        uint4 *dst = ret_x + slot * cpr;
+    const int cpr = a.cpr;
+    for (int64_t slot = warp; slot < a.n_slots; slot += nwarp) {
+        uint4 *dst;
+        int32_t *dst_hdr;
+        if (EP) {
+            int h, w;
+            const uint32_t q = ep_recv_to_send(a.geo, uint32_t(slot), h, w);
+            if (!((a.wave_mask >> w) & 1u)) continue;
+            dst = reinterpret_cast<uint4 *>(a.ep.x[h]) + int64_t(q) * cpr;
+            dst_hdr = a.ep.hdr[h] + q;
+        } else {
+            dst = a.ret_x + slot * cpr;
+            dst_hdr = a.ret_hdr + slot;
+        }
+        const int32_t e = a.pool_hdr[slot];
+        const bool keep = a.recv_row[slot] >= 0 && e >= 0 && e < a.E;
+        const float s = keep ? a.scale[e] : 0.0f;
+        const uint4 *src = a.pool_x + slot * cpr;
         if (keep) {
             int c = lane;
             for (; c + 96 < cpr; c += 128) {
@@ -69,24 +96,42 @@ __global__ void __launch_bounds__(256) expert_kernel(const uint4 *__restrict__ p
         } else {
             for (int c = lane; c < cpr; c += 32) __stcs(dst + c, make_uint4(0, 0, 0, 0));
         }
-        if (lane == 0) ret_hdr[slot] = keep ? e : -1;
+        if (lane == 0) *dst_hdr = keep ? e : -1;
     }
+    if (EP) __threadfence_system();  // peer stores ordered before any later signal
 }
 
 }  // namespace
 
 cudaError_t launch_expert(const Geo &g, const uint16_t *pool_x, const int32_t *pool_hdr,
                           const int32_t *recv_row, const float *scale, uint16_t *ret_x,
-                          int32_t *ret_hdr, cudaStream_t st)
+                          int32_t *ret_hdr, cudaStream_t st, const EpRows *ep,
+                          uint32_t wave_mask)
 {
     if (g.n_slots == 0) return cudaSuccess;
     DevInfo di;
     if (dev_info(&di) != 0) return cudaErrorUnknown;
     int64_t blocks = (g.n_slots + 7) / 8;
     if (blocks > int64_t(di.sms) * 8) blocks = int64_t(di.sms) * 8;
-    expert_kernel<<<unsigned(blocks), 256, 0, st>>>(
-        reinterpret_cast<const uint4 *>(pool_x), pool_hdr, recv_row, scale,
-        reinterpret_cast<uint4 *>(ret_x), ret_hdr, g.n_slots, g.D / 8, g.E);
+    ExpertArgs a;
+    a.pool_x = reinterpret_cast<const uint4 *>(pool_x);
+    a.pool_hdr = pool_hdr;
+    a.recv_row = recv_row;
+    a.scale = scale;
+    a.ret_x = reinterpret_cast<uint4 *>(ret_x);
+    a.ret_hdr = ret_hdr;
+    a.n_slots = g.n_slots;
+    a.cpr = g.D / 8;
+    a.E = g.E;
+    a.wave_mask = wave_mask;
+    a.geo = g;
+    if (ep) {
+        a.ep = *ep;
+        expert_kernel<true><<<unsigned(blocks), 256, 0, st>>>(a);
+    } else {
+        std::memset(&a.ep, 0, sizeof(a.ep));
+        expert_kernel<false><<<unsigned(blocks), 256, 0, st>>>(a);
+    }
     return cudaGetLastError();
 }
 

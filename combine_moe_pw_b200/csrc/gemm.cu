@@ -82,6 +82,8 @@ struct GemmArgs {
     // ROWS
     uint16_t *C;
     int64_t ldc;
+    const uint16_t *add;  // ROWS, optional: bf16 [M, ldc] added in fp32 before rounding
+                          // (may be C itself: each element is read before it is written)
     // SCATTER
     const int32_t *slot_map;
     const int32_t *idx;
@@ -159,19 +161,47 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &p, uint8_t *stage_
     for (int h = 0; h < 2; ++h) {
         // 1. TMEM -> bf16 -> this thread's row (half h) in shared memory
         uint8_t *my_row = stage_rows + size_t(lane) * ROW_PITCH;
+        const int64_t my_m = m0 + q * 32 + lane;
 #pragma unroll 1
         for (int c = 0; c < HALF / 32; ++c) {
+            // merge operand of this thread's row, 32 columns (loaded before
+            // the accumulator so the two latencies overlap)
+            uint32_t ad[16];
+            if (p.add) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int col = n0 + h * HALF + c * 32 + 8 * i;
+                    uint4 a4 = make_uint4(0, 0, 0, 0);
+                    if (my_m < p.M && col + 8 <= p.N)
+                        a4 = __ldcs(reinterpret_cast<const uint4 *>(p.add + my_m * p.ldc + col));
+                    ad[4 * i + 0] = a4.x;
+                    ad[4 * i + 1] = a4.y;
+                    ad[4 * i + 2] = a4.z;
+                    ad[4 * i + 3] = a4.w;
+                }
+            }
             uint32_t v[32];
             umma::tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) +
                                 uint32_t(acc * BN + h * HALF + c * 32),
                             v);
+            float f[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+            if (p.add) {
+                // the merge: fp32 sum, one rounding to bf16 below
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    f[2 * i] = __fadd_rn(f[2 * i], __uint_as_float(ad[i] << 16));
+                    f[2 * i + 1] = __fadd_rn(f[2 * i + 1], __uint_as_float(ad[i] & 0xFFFF0000u));
+                }
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 uint4 o;
-                o.x = pack_bf16(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
-                o.y = pack_bf16(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-                o.z = pack_bf16(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-                o.w = pack_bf16(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+                o.x = pack_bf16(f[8 * i + 0], f[8 * i + 1]);
+                o.y = pack_bf16(f[8 * i + 2], f[8 * i + 3]);
+                o.z = pack_bf16(f[8 * i + 4], f[8 * i + 5]);
+                o.w = pack_bf16(f[8 * i + 6], f[8 * i + 7]);
                 const int chunk = (c * 4 + i) ^ (lane & 7);
                 reinterpret_cast<uint4 *>(my_row)[chunk] = o;
             }
@@ -622,7 +652,8 @@ int pair_clusters_resident()
 cudaError_t launch_gemm(const uint16_t *A, const uint16_t *Bt, int64_t M, int32_t N, int32_t K,
                         int32_t mode, uint16_t *C, int64_t ldc, const int32_t *slot_map,
                         const int32_t *idx, int32_t topk, uint16_t *pool_x, int32_t *pool_hdr,
-                        int64_t n_slots, moe_pw_counters *ctr, cudaStream_t st)
+                        int64_t n_slots, moe_pw_counters *ctr, cudaStream_t st,
+                        const uint16_t *add)
 {
     if (M == 0 || N == 0) return cudaSuccess;
     DevInfo di;
@@ -639,6 +670,7 @@ cudaError_t launch_gemm(const uint16_t *A, const uint16_t *Bt, int64_t M, int32_
     p.mode = mode;
     p.C = C;
     p.ldc = ldc;
+    p.add = add;
     p.slot_map = slot_map;
     p.idx = idx;
     p.topk = topk;

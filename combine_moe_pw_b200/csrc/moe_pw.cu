@@ -62,6 +62,9 @@ int make_geo(const moe_pw_config *c, Geo *g)
 
     std::memset(g, 0, sizeof(*g));
     g->T = c->T;
+    g->ep_n = 1;
+    g->ep_g = 0;
+    g->Rn = c->R;
     g->E = c->E;
     g->k = c->k;
     g->D = c->D;
@@ -105,6 +108,30 @@ int make_geo(const moe_pw_config *c, Geo *g)
     const int64_t nch = int64_t(g->n_groups) * g->chunks_per_group;
     if (nch > MAX_INT32) return MOE_PW_EUNSUPPORTED;
     g->n_chunks = int32_t(nch);
+    return MOE_PW_OK;
+}
+
+// The share of GPU ep->gpu in an expert-parallel run: the single-GPU
+// geometry of the whole batch (capacities included), narrowed to this GPU's
+// Rn sources (its tokens, send pools and send slots) and Rn destinations.
+int make_geo_ep(const moe_pw_config *c, const moe_pw_ep *ep, Geo *g)
+{
+    int rc = make_geo(c, g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!ep || ep->n_gpus < 1 || ep->n_gpus > MOE_PW_EP_MAX_GPUS || ep->gpu < 0 ||
+        ep->gpu >= ep->n_gpus)
+        return MOE_PW_EINVAL;
+    if (c->mode != MOE_PW_POOLED) return MOE_PW_EUNSUPPORTED;
+    if (c->R % ep->n_gpus != 0) return MOE_PW_EINVAL;
+    const int32_t Rn = c->R / ep->n_gpus;
+    g->ep_n = ep->n_gpus;
+    g->ep_g = ep->gpu;
+    g->Rn = Rn;
+    g->T = int64_t(Rn) * g->T_s;
+    g->n_groups = Rn;
+    g->n_pools = int64_t(Rn) * c->R * c->W;
+    g->n_slots = g->n_pools * g->C_s;
+    g->n_chunks = Rn * g->chunks_per_group;
     return MOE_PW_OK;
 }
 
@@ -284,6 +311,28 @@ int moe_pw_combine_bf16(const moe_pw_config *cfg, const uint16_t *ret_x, const i
     return cuda_rc(launch_combine_bf16(g, ret_x, ret_hdr, slot_map, gates, out, counters, stream));
 }
 
+int moe_pw_combine_bf16_rows(const moe_pw_config *cfg, const uint16_t *ret_x,
+                             const int32_t *ret_hdr, const int32_t *slot_map, const float *gates,
+                             int64_t first_token, int64_t n_tokens, uint16_t *out,
+                             moe_pw_counters *counters, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (first_token < 0 || n_tokens < 0 || first_token + n_tokens > g.T) return MOE_PW_EINVAL;
+    if (n_tokens == 0) return MOE_PW_OK;
+    if (!ret_x || !ret_hdr || !slot_map || !gates || !out || !counters) return MOE_PW_EINVAL;
+    if (!aligned(ret_x, 16) || !aligned(out, 16) || !aligned(ret_hdr, 4) ||
+        !aligned(slot_map, 4) || !aligned(gates, 4) || !aligned(counters, 8))
+        return MOE_PW_EUNSUPPORTED;
+    // the same kernel on the token range: the pool (and its slot ids) is the
+    // whole batch's, only the tokens are narrowed
+    Geo rows = g;
+    rows.T = n_tokens;
+    return cuda_rc(launch_combine_bf16(rows, ret_x, ret_hdr, slot_map + first_token * g.k,
+                                       gates + first_token * g.k, out, counters, stream));
+}
+
 int moe_pw_combine_backward(const moe_pw_config *cfg, const float *dout, const uint16_t *ret_x,
                             const int32_t *ret_hdr, const int32_t *slot_map, const int32_t *idx,
                             const float *gates, uint16_t *d_ret, float *dgates, float *dlogits,
@@ -332,6 +381,21 @@ int moe_pw_project(const uint16_t *A, const uint16_t *Bt, uint16_t *C, int64_t M
         return MOE_PW_EUNSUPPORTED;
     return cuda_rc(launch_gemm(A, Bt, M, N, K, 0, C, N, nullptr, nullptr, 0, nullptr, nullptr, 0,
                                counters, stream));
+}
+
+int moe_pw_project_add(const uint16_t *A, const uint16_t *Bt, const uint16_t *add, uint16_t *C,
+                       int64_t M, int32_t N, int32_t K, moe_pw_counters *counters,
+                       cudaStream_t stream)
+{
+    if (M < 0 || N < 0 || K < 1 || M > MAX_INT32) return MOE_PW_EINVAL;
+    if (M == 0 || N == 0) return MOE_PW_OK;
+    if (!A || !Bt || !add || !C || !counters) return MOE_PW_EINVAL;
+    if (K % 8 != 0 || N % 8 != 0) return MOE_PW_EUNSUPPORTED;
+    if (!aligned(A, 16) || !aligned(Bt, 16) || !aligned(add, 16) || !aligned(C, 16) ||
+        !aligned(counters, 8))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_gemm(A, Bt, M, N, K, 0, C, N, nullptr, nullptr, 0, nullptr, nullptr, 0,
+                               counters, stream, add));
 }
 
 int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint16_t *w_down_t,
@@ -476,3 +540,261 @@ extern "C" int moe_pw_selftest_wait_timeout(moe_pw_counters *counters, int32_t p
     selftest_wait_kernel<<<1, 32, 0, stream>>>(counters, uint32_t(polls));
     return cuda_rc(cudaGetLastError());
 }
+
+// ---------------------------------------------------------------------------
+// Expert parallelism over several GPUs: the same kernels on each GPU's share,
+// with the pack and the expert op storing into peer GPUs' pools.
+// ---------------------------------------------------------------------------
+
+namespace moe_pw {
+namespace {
+
+// Copy the receive (or return) column of the caller's peer table; every entry
+// of the run's GPUs must be set and aligned.
+int ep_rows(const Geo &g, uint16_t *const *x, int32_t *const *hdr, EpRows *out)
+{
+    std::memset(out, 0, sizeof(*out));
+    for (int h = 0; h < g.ep_n; ++h) {
+        if (!x[h] || !hdr[h]) return MOE_PW_EINVAL;
+        if (!aligned(x[h], 16) || !aligned(hdr[h], 4)) return MOE_PW_EUNSUPPORTED;
+        out->x[h] = x[h];
+        out->hdr[h] = hdr[h];
+    }
+    return MOE_PW_OK;
+}
+
+uint32_t wave_bits(const Geo &g, uint32_t mask) { return mask & ((1u << g.W) - 1u); }
+
+}  // namespace
+}  // namespace moe_pw
+
+extern "C" {
+
+int moe_pw_ep_plan(const moe_pw_config *cfg, const moe_pw_ep *ep, int64_t budget_bytes,
+                   moe_pw_ep_sizes *out)
+{
+    if (!out) return MOE_PW_EINVAL;
+    Geo g;
+    const int rc = make_geo_ep(cfg, ep, &g);
+    if (rc != MOE_PW_OK) return rc;
+    std::memset(out, 0, sizeof(*out));
+    const int64_t T = g.T, E = g.E, k = g.k, D = g.D, S = g.n_slots;
+    const int64_t El = int64_t(g.Rn) * g.L;
+    out->tokens = T;
+    out->first_token = int64_t(g.ep_g) * T;
+    out->C_s = g.C_s;
+    out->C_r = g.C_r;
+    out->n_pools = g.n_pools;
+    out->n_slots = S;
+    out->local_experts = El;
+    out->bucket_len = El * g.C_r;
+    out->workspace_bytes = ws_bytes(g);
+    out->total_bytes = 4 * T * E + 8 * T * k + 2 * T * D + 4 * T * k  // logits .. slot_map
+                       + 4 * g.n_pools                                 // occ
+                       + 2 * (2 * S * D) + 3 * (4 * S) + 4 * S         // recv / ret pools + headers
+                       + 4 * out->bucket_len + 8 * El + 4 * E           // buckets, counts, scale
+                       + 4 * T * D                                      // out
+                       + int64_t(sizeof(moe_pw_counters)) + out->workspace_bytes;
+    if (budget_bytes > 0 && out->total_bytes > budget_bytes) return MOE_PW_ENOMEM;
+    return MOE_PW_OK;
+}
+
+int moe_pw_ep_route(const moe_pw_config *cfg, const moe_pw_ep *ep, const float *logits,
+                    int32_t *idx, float *gates, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo_ep(cfg, ep, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.E % 4 != 0) return MOE_PW_EUNSUPPORTED;
+    if (g.T == 0) return MOE_PW_OK;
+    if (!logits || !idx || !gates) return MOE_PW_EINVAL;
+    if (!aligned(logits, 16) || !aligned(idx, 4) || !aligned(gates, 4)) return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_route(g, logits, idx, gates, stream));
+}
+
+int moe_pw_ep_assign(const moe_pw_config *cfg, const moe_pw_ep *ep, const int32_t *idx,
+                     int32_t *slot_map, int32_t *occ, moe_pw_counters *counters,
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo_ep(cfg, ep, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!counters || !occ) return MOE_PW_EINVAL;
+    if (g.T > 0 && (!idx || !slot_map || !workspace)) return MOE_PW_EINVAL;
+    if (g.T > 0 && int64_t(workspace_bytes) < ws_bytes(g)) return MOE_PW_EINVAL;
+    if (!aligned(counters, 8) || !aligned(occ, 4) || (g.T > 0 && (!aligned(idx, 4) ||
+        !aligned(slot_map, 4) || !aligned(workspace, 256))))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_assign(g, idx, slot_map, occ, counters, workspace, stream));
+}
+
+int moe_pw_ep_pack(const moe_pw_config *cfg, const moe_pw_ep *ep, const moe_pw_ep_peers *peers,
+                   const uint16_t *x, const int32_t *idx, const int32_t *slot_map,
+                   const int32_t *occ, uint32_t wave_mask, moe_pw_counters *counters,
+                   cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo_ep(cfg, ep, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!peers) return MOE_PW_EINVAL;
+    if (g.n_slots == 0 || wave_bits(g, wave_mask) == 0) return MOE_PW_OK;
+    if (!x || !idx || !slot_map || !occ || !counters) return MOE_PW_EINVAL;
+    if (!aligned(x, 16) || !aligned(idx, 4) || !aligned(slot_map, 4) || !aligned(occ, 4) ||
+        !aligned(counters, 8))
+        return MOE_PW_EUNSUPPORTED;
+    EpRows rows;
+    if ((rc = ep_rows(g, peers->recv_x, peers->recv_hdr, &rows)) != MOE_PW_OK) return rc;
+    return cuda_rc(launch_pack(g, x, idx, slot_map, occ, nullptr, nullptr, counters, stream,
+                               &rows, wave_bits(g, wave_mask)));
+}
+
+int moe_pw_ep_bucket(const moe_pw_config *cfg, const moe_pw_ep *ep, const int32_t *recv_hdr,
+                     int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,
+                     uint32_t wave_mask, moe_pw_counters *counters, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo_ep(cfg, ep, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!counters || !expert_counts || !recv_hdr || !recv_row || !bucket_slot)
+        return MOE_PW_EINVAL;
+    if (!aligned(counters, 8) || !aligned(expert_counts, 4) || !aligned(recv_hdr, 4) ||
+        !aligned(recv_row, 4) || !aligned(bucket_slot, 4))
+        return MOE_PW_EUNSUPPORTED;
+    if (wave_bits(g, wave_mask) == 0) return MOE_PW_OK;
+    return cuda_rc(launch_bucket(g, recv_hdr, nullptr, recv_row, bucket_slot, expert_counts,
+                                 counters, stream, wave_bits(g, wave_mask)));
+}
+
+int moe_pw_ep_expert(const moe_pw_config *cfg, const moe_pw_ep *ep, const moe_pw_ep_peers *peers,
+                     const uint16_t *recv_x, const int32_t *recv_hdr, const int32_t *recv_row,
+                     const float *scale, uint32_t wave_mask, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo_ep(cfg, ep, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!peers) return MOE_PW_EINVAL;
+    if (g.n_slots == 0 || wave_bits(g, wave_mask) == 0) return MOE_PW_OK;
+    if (!recv_x || !recv_hdr || !recv_row || !scale) return MOE_PW_EINVAL;
+    if (!aligned(recv_x, 16) || !aligned(recv_hdr, 4) || !aligned(recv_row, 4) ||
+        !aligned(scale, 4))
+        return MOE_PW_EUNSUPPORTED;
+    EpRows rows;
+    if ((rc = ep_rows(g, peers->ret_x, peers->ret_hdr, &rows)) != MOE_PW_OK) return rc;
+    return cuda_rc(launch_expert(g, recv_x, recv_hdr, recv_row, scale, nullptr, nullptr, stream,
+                                 &rows, wave_bits(g, wave_mask)));
+}
+
+int moe_pw_ep_combine(const moe_pw_config *cfg, const moe_pw_ep *ep, const uint16_t *ret_x,
+                      const int32_t *ret_hdr, const int32_t *slot_map, const float *gates,
+                      float *out, moe_pw_counters *counters, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo_ep(cfg, ep, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.T == 0) return MOE_PW_OK;
+    if (!ret_x || !ret_hdr || !slot_map || !gates || !out || !counters) return MOE_PW_EINVAL;
+    if (!aligned(ret_x, 16) || !aligned(out, 16) || !aligned(ret_hdr, 4) ||
+        !aligned(slot_map, 4) || !aligned(gates, 4) || !aligned(counters, 8))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_combine(g, ret_x, ret_hdr, slot_map, gates, out, counters, stream));
+}
+
+int moe_pw_ep_stats(const moe_pw_config *cfg, const moe_pw_ep *ep,
+                    const moe_pw_counters *counters, const int32_t *expert_counts,
+                    moe_pw_drop_stats *host_out, int32_t *host_expert_counts,
+                    cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo_ep(cfg, ep, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!counters || !host_out) return MOE_PW_EINVAL;
+    moe_pw_counters c;
+    if (cudaMemcpyAsync(&c, counters, sizeof(c), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return MOE_PW_ECUDA;
+    const size_t el = size_t(g.Rn) * g.L;
+    if (expert_counts && host_expert_counts &&
+        cudaMemcpyAsync(host_expert_counts, expert_counts, sizeof(int32_t) * 2 * el,
+                        cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return MOE_PW_ECUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_PW_ECUDA;
+    host_out->assignments = g.T * g.k;
+    host_out->kept = int64_t(c.kept);
+    host_out->sender_dropped = int64_t(c.sender_dropped);
+    host_out->receiver_dropped = int64_t(c.receiver_dropped);
+    host_out->max_occ = c.max_occ;
+    host_out->max_fill = c.max_fill;
+    host_out->error = c.error;
+    host_out->reserved = 0;
+    return c.error != 0 ? MOE_PW_EDEVICE : MOE_PW_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Buffer sharing between the processes of an expert-parallel run.
+// ---------------------------------------------------------------------------
+
+namespace moe_pw {
+namespace {
+
+// cuMemGetAddressRange from the driver, fetched through the runtime (the
+// library links only the runtime): the base of the allocation holding a
+// device pointer, which cudaIpcGetMemHandle describes.
+typedef int (*mem_range_fn)(unsigned long long *, size_t *, unsigned long long);
+
+mem_range_fn mem_range()
+{
+    static mem_range_fn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return mem_range_fn(nullptr);
+        return reinterpret_cast<mem_range_fn>(p);
+    }();
+    return fn;
+}
+
+}  // namespace
+}  // namespace moe_pw
+
+extern "C" {
+
+int moe_pw_ipc_export(const void *dev_ptr, moe_pw_ipc_handle *out)
+{
+    if (!dev_ptr || !out) return MOE_PW_EINVAL;
+    static_assert(sizeof(cudaIpcMemHandle_t) == sizeof(out->handle), "IPC handle size");
+    const mem_range_fn range = mem_range();
+    if (!range) return MOE_PW_ECUDA;
+    unsigned long long base = 0;
+    size_t size = 0;
+    if (range(&base, &size, reinterpret_cast<unsigned long long>(dev_ptr)) != 0)
+        return MOE_PW_ECUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base)) != cudaSuccess)
+        return MOE_PW_ECUDA;
+    std::memcpy(out->handle, &h, sizeof(h));
+    out->offset = reinterpret_cast<unsigned long long>(dev_ptr) - base;
+    return MOE_PW_OK;
+}
+
+int moe_pw_ipc_open(const moe_pw_ipc_handle *h, void **dev_ptr)
+{
+    if (!h || !dev_ptr) return MOE_PW_EINVAL;
+    cudaIpcMemHandle_t ch;
+    std::memcpy(&ch, h->handle, sizeof(ch));
+    void *base = nullptr;
+    if (cudaIpcOpenMemHandle(&base, ch, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess)
+        return MOE_PW_ECUDA;
+    *dev_ptr = static_cast<char *>(base) + h->offset;
+    return MOE_PW_OK;
+}
+
+int moe_pw_ipc_close(void *dev_ptr, const moe_pw_ipc_handle *h)
+{
+    if (!dev_ptr || !h) return MOE_PW_EINVAL;
+    return cuda_rc(cudaIpcCloseMemHandle(static_cast<char *>(dev_ptr) - h->offset));
+}
+
+}  // extern "C"

@@ -28,6 +28,8 @@
 // The defaults below came from a sweep on the 262,144-token batch: deeper
 // rings with fewer warps beat more warps with shallow rings; the lag between
 // 8 and 20 made no measurable difference.
+#include <cstring>
+
 #include "common.cuh"
 
 namespace moe_pw {
@@ -74,9 +76,14 @@ struct PackArgs {
     int32_t D;
     int32_t stages;
     uint32_t rowbytes;
+    // expert-parallel runs: the receive pools of every GPU and the waves sent
+    Geo geo;
+    uint32_t wave_mask;
+    EpRows ep;
 };
 
-template <int LAG>
+// EP: rows and tails go to the destination GPUs' receive pools (peer stores).
+template <int LAG, bool EP>
 __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
 {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -160,8 +167,17 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
         if (slot >= p.n_slots) {
             set_error(p.ctr, MOE_PW_DEVERR_SLOT);
         } else if (slot >= 0) {
-            bulk_s2g(p.pool_x + int64_t(slot) * D, buf + size_t(s) * rb, rb, pol_pool);
-            p.pool_hdr[slot] = e;
+            if (EP) {
+                int h, w;
+                const uint32_t rq = ep_send_to_recv(p.geo, uint32_t(slot), h, w);
+                if ((p.wave_mask >> w) & 1u) {
+                    bulk_s2g(p.ep.x[h] + int64_t(rq) * D, buf + size_t(s) * rb, rb, pol_pool);
+                    p.ep.hdr[h][rq] = e;
+                }
+            } else {
+                bulk_s2g(p.pool_x + int64_t(slot) * D, buf + size_t(s) * rb, rb, pol_pool);
+                p.pool_hdr[slot] = e;
+            }
         }
         bulk_commit();
         if (i >= LAG) {
@@ -188,6 +204,19 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
         int64_t filled = p.occ[q];
         if (filled < 0) filled = 0;
         if (filled > p.C_s) filled = p.C_s;
+        if (EP) {
+            // the tail is contiguous in the destination's receive pool too
+            int h, w;
+            const uint32_t rq0 = ep_send_to_recv(p.geo, uint32_t(q * p.C_s), h, w);
+            if (!((p.wave_mask >> w) & 1u)) continue;
+            for (int64_t c = filled + lane; c < p.C_s; c += 32) {
+                bulk_s2g(p.ep.x[h] + (int64_t(rq0) + c) * D, zero, rb, pol_pool);
+                p.ep.hdr[h][rq0 + c] = -1;
+            }
+            bulk_commit();
+            bulk_wait_read<8>();
+            continue;
+        }
 #if MOE_PW_PACK_ZERO_TMA
         for (int64_t c = filled + lane; c < p.C_s; c += 32) {
             const int64_t slot = q * p.C_s + c;
@@ -205,17 +234,24 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
 #endif
     }
     bulk_wait_all();
+    if (EP) {
+        // the peer stores (bulk and plain) are performed; order them before
+        // anything this GPU signals to the others after the kernel
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence_system();
+    }
 }
 
-template <int LAGT>
+template <int LAGT, bool EP>
 cudaError_t launch_lag(const PackArgs &p, const DevInfo &di, const Geo &g, int nw, size_t smem,
                        cudaStream_t st)
 {
-    cudaError_t err = cudaFuncSetAttribute(pack_kernel<LAGT>,
+    cudaError_t err = cudaFuncSetAttribute(pack_kernel<LAGT, EP>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (err != cudaSuccess) return err;
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pack_kernel<LAGT>, nw * 32, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pack_kernel<LAGT, EP>, nw * 32,
+                                                        smem);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) per_sm = 1;
     int64_t blocks = int64_t(di.sms) * per_sm;
@@ -225,15 +261,26 @@ cudaError_t launch_lag(const PackArgs &p, const DevInfo &di, const Geo &g, int n
     if (blocks < 1) blocks = 1;
     // the zero-fill phase's pool counter starts at 0 for every launch
     if ((err = cudaMemsetAsync(&p.ctr->work, 0, sizeof(int32_t), st)) != cudaSuccess) return err;
-    pack_kernel<LAGT><<<unsigned(blocks), nw * 32, smem, st>>>(p);
+    pack_kernel<LAGT, EP><<<unsigned(blocks), nw * 32, smem, st>>>(p);
     return cudaGetLastError();
+}
+
+template <bool EP>
+cudaError_t launch_ep(const PackArgs &p, const DevInfo &di, const Geo &g, int nw, size_t smem,
+                      int lag_cap, cudaStream_t st)
+{
+    if (lag_cap >= 12 && LAG >= 12) return launch_lag<12, EP>(p, di, g, nw, smem, st);
+    if (lag_cap >= 8) return launch_lag<8, EP>(p, di, g, nw, smem, st);
+    if (lag_cap >= 4) return launch_lag<4, EP>(p, di, g, nw, smem, st);
+    return launch_lag<2, EP>(p, di, g, nw, smem, st);
 }
 
 }  // namespace
 
 cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
                         const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
-                        int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st)
+                        int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st,
+                        const EpRows *ep, uint32_t wave_mask)
 {
     if (g.T == 0 && g.n_pools == 0) return cudaSuccess;
     DevInfo di;
@@ -253,6 +300,10 @@ cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
     p.k = g.k;
     p.D = g.D;
     p.rowbytes = uint32_t(g.D) * 2u;
+    p.geo = g;
+    p.wave_mask = wave_mask;
+    if (ep) p.ep = *ep;
+    else std::memset(&p.ep, 0, sizeof(p.ep));
 
     // warps and stages per warp: as many rows as fit next to the zero row,
     // MIN_STAGES .. MOE_PW_PACK_MAX_STAGES, dropping warps for very wide rows
@@ -269,10 +320,8 @@ cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
     const size_t smem = bar_bytes + p.rowbytes + size_t(PACK_WARPS) * stages * p.rowbytes;
     // the deepest store lag (<= LAG) that leaves two stages for loads
     const int lag_cap = stages - 2 < LAG ? stages - 2 : LAG;
-    if (lag_cap >= 12 && LAG >= 12) return launch_lag<12>(p, di, g, nw, smem, st);
-    if (lag_cap >= 8) return launch_lag<8>(p, di, g, nw, smem, st);
-    if (lag_cap >= 4) return launch_lag<4>(p, di, g, nw, smem, st);
-    return launch_lag<2>(p, di, g, nw, smem, st);
+    return ep ? launch_ep<true>(p, di, g, nw, smem, lag_cap, st)
+              : launch_ep<false>(p, di, g, nw, smem, lag_cap, st);
 }
 
 }  // namespace moe_pw

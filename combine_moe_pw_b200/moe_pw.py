@@ -59,6 +59,30 @@ class moe_pw_drop_stats(ctypes.Structure):
                 ("error", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
+EP_MAX_GPUS = 64  # MOE_PW_EP_MAX_GPUS
+
+
+class moe_pw_ep(ctypes.Structure):
+    _fields_ = [("n_gpus", ctypes.c_int32), ("gpu", ctypes.c_int32)]
+
+
+class moe_pw_ep_peers(ctypes.Structure):
+    _fields_ = [("recv_x", ctypes.c_void_p * EP_MAX_GPUS),
+                ("recv_hdr", ctypes.c_void_p * EP_MAX_GPUS),
+                ("ret_x", ctypes.c_void_p * EP_MAX_GPUS),
+                ("ret_hdr", ctypes.c_void_p * EP_MAX_GPUS)]
+
+
+class moe_pw_ep_sizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("tokens", "first_token", "C_s", "C_r", "n_pools",
+                                              "n_slots", "local_experts", "bucket_len",
+                                              "workspace_bytes", "total_bytes")]
+
+
+class moe_pw_ipc_handle(ctypes.Structure):
+    _fields_ = [("handle", ctypes.c_ubyte * 64), ("offset", ctypes.c_uint64)]
+
+
 # name -> argument types (after the config pointer); every function returns int
 _VP, _SZ, _I64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64
 _CFG = ctypes.POINTER(moe_pw_config)
@@ -75,12 +99,29 @@ SIGNATURES = {
     "moe_pw_expert": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_combine": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_combine_bf16": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_combine_bf16_rows": [_CFG, _VP, _VP, _VP, _VP, _I64, _I64, _VP, _VP, _VP],
     "moe_pw_combine_backward": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_dispatch_backward": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_project": [_VP, _VP, _VP, _I64, ctypes.c_int32, ctypes.c_int32, _VP, _VP],
+    "moe_pw_project_add": [_VP, _VP, _VP, _VP, _I64, ctypes.c_int32, ctypes.c_int32, _VP, _VP],
     "moe_pw_project_pack": [_CFG, _VP, _VP, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_stats": [_CFG, _VP, _VP, ctypes.POINTER(moe_pw_drop_stats), _VP, _VP],
     "moe_pw_selftest_wait_timeout": [_VP, ctypes.c_int32, _VP],
+    "moe_pw_ep_plan": [_CFG, ctypes.POINTER(moe_pw_ep), _I64, ctypes.POINTER(moe_pw_ep_sizes)],
+    "moe_pw_ep_route": [_CFG, ctypes.POINTER(moe_pw_ep), _VP, _VP, _VP, _VP],
+    "moe_pw_ep_assign": [_CFG, ctypes.POINTER(moe_pw_ep), _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "moe_pw_ep_pack": [_CFG, ctypes.POINTER(moe_pw_ep), ctypes.POINTER(moe_pw_ep_peers), _VP, _VP,
+                       _VP, _VP, ctypes.c_uint32, _VP, _VP],
+    "moe_pw_ep_bucket": [_CFG, ctypes.POINTER(moe_pw_ep), _VP, _VP, _VP, _VP, ctypes.c_uint32,
+                         _VP, _VP],
+    "moe_pw_ep_expert": [_CFG, ctypes.POINTER(moe_pw_ep), ctypes.POINTER(moe_pw_ep_peers), _VP,
+                         _VP, _VP, _VP, ctypes.c_uint32, _VP],
+    "moe_pw_ep_combine": [_CFG, ctypes.POINTER(moe_pw_ep), _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_ep_stats": [_CFG, ctypes.POINTER(moe_pw_ep), _VP, _VP,
+                        ctypes.POINTER(moe_pw_drop_stats), _VP, _VP],
+    "moe_pw_ipc_export": [_VP, ctypes.POINTER(moe_pw_ipc_handle)],
+    "moe_pw_ipc_open": [ctypes.POINTER(moe_pw_ipc_handle), ctypes.POINTER(ctypes.c_void_p)],
+    "moe_pw_ipc_close": [_VP, ctypes.POINTER(moe_pw_ipc_handle)],
 }
 
 _lib = None
@@ -236,6 +277,14 @@ def moe_pw_combine_bf16(cfg, ret_x, ret_hdr, slot_map, gates, out, counters, str
         _ptr(counters), _stream(stream)))
 
 
+def moe_pw_combine_bf16_rows(cfg, ret_x, ret_hdr, slot_map, gates, first_token: int,
+                             n_tokens: int, out, counters, stream=None):
+    c = _cfg(cfg)
+    _check("moe_pw_combine_bf16_rows", load_library().moe_pw_combine_bf16_rows(
+        ctypes.byref(c), _ptr(ret_x), _ptr(ret_hdr), _ptr(slot_map), _ptr(gates), first_token,
+        n_tokens, _ptr(out), _ptr(counters), _stream(stream)))
+
+
 def moe_pw_combine_backward(cfg, dout, ret_x, ret_hdr, slot_map, idx, gates, d_ret, dgates,
                             dlogits, counters, stream=None):
     c = _cfg(cfg)
@@ -255,6 +304,12 @@ def moe_pw_project(A, Bt, C, M: int, N: int, K: int, counters, stream=None):
     """C = bf16(A @ Bt^T) on the tensor cores (bf16 operands, fp32 accumulation)."""
     _check("moe_pw_project", load_library().moe_pw_project(
         _ptr(A), _ptr(Bt), _ptr(C), M, N, K, _ptr(counters), _stream(stream)))
+
+
+def moe_pw_project_add(A, Bt, add, C, M: int, N: int, K: int, counters, stream=None):
+    """C = bf16(A @ Bt^T + add): the up-projection merged with the shared path."""
+    _check("moe_pw_project_add", load_library().moe_pw_project_add(
+        _ptr(A), _ptr(Bt), _ptr(add), _ptr(C), M, N, K, _ptr(counters), _stream(stream)))
 
 
 def moe_pw_project_pack(cfg, h, w_down_t, model_width: int, idx, slot_map, occ, pool_x, pool_hdr,
@@ -290,6 +345,97 @@ def moe_pw_selftest_wait_timeout(counters, polls: int = 4096, stream=None):
     """Run the bounded-wait self-test (see include/moe_pw.h)."""
     _check("moe_pw_selftest_wait_timeout", load_library().moe_pw_selftest_wait_timeout(
         _ptr(counters), polls, _stream(stream)))
+
+
+def _ep(n_gpus: int, gpu: int) -> moe_pw_ep:
+    return moe_pw_ep(n_gpus, gpu)
+
+
+def moe_pw_ep_plan(cfg, n_gpus: int, gpu: int, budget_bytes: int = 0) -> moe_pw_ep_sizes:
+    out = moe_pw_ep_sizes()
+    c, e = _cfg(cfg), _ep(n_gpus, gpu)
+    _check("moe_pw_ep_plan", load_library().moe_pw_ep_plan(ctypes.byref(c), ctypes.byref(e),
+                                                           budget_bytes, ctypes.byref(out)))
+    return out
+
+
+def moe_pw_ep_route(cfg, n_gpus, gpu, logits, idx, gates, stream=None):
+    c, e = _cfg(cfg), _ep(n_gpus, gpu)
+    _check("moe_pw_ep_route", load_library().moe_pw_ep_route(
+        ctypes.byref(c), ctypes.byref(e), _ptr(logits), _ptr(idx), _ptr(gates), _stream(stream)))
+
+
+def moe_pw_ep_assign(cfg, n_gpus, gpu, idx, slot_map, occ, counters, workspace, stream=None):
+    c, e = _cfg(cfg), _ep(n_gpus, gpu)
+    wsb = workspace.numel() * workspace.element_size()
+    _check("moe_pw_ep_assign", load_library().moe_pw_ep_assign(
+        ctypes.byref(c), ctypes.byref(e), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(counters),
+        _ptr(workspace), wsb, _stream(stream)))
+
+
+def moe_pw_ep_pack(cfg, n_gpus, gpu, peers: moe_pw_ep_peers, x, idx, slot_map, occ, wave_mask,
+                   counters, stream=None):
+    c, e = _cfg(cfg), _ep(n_gpus, gpu)
+    _check("moe_pw_ep_pack", load_library().moe_pw_ep_pack(
+        ctypes.byref(c), ctypes.byref(e), ctypes.byref(peers), _ptr(x), _ptr(idx), _ptr(slot_map),
+        _ptr(occ), wave_mask, _ptr(counters), _stream(stream)))
+
+
+def moe_pw_ep_bucket(cfg, n_gpus, gpu, recv_hdr, recv_row, bucket_slot, expert_counts, wave_mask,
+                     counters, stream=None):
+    c, e = _cfg(cfg), _ep(n_gpus, gpu)
+    _check("moe_pw_ep_bucket", load_library().moe_pw_ep_bucket(
+        ctypes.byref(c), ctypes.byref(e), _ptr(recv_hdr), _ptr(recv_row), _ptr(bucket_slot),
+        _ptr(expert_counts), wave_mask, _ptr(counters), _stream(stream)))
+
+
+def moe_pw_ep_expert(cfg, n_gpus, gpu, peers: moe_pw_ep_peers, recv_x, recv_hdr, recv_row, scale,
+                     wave_mask, stream=None):
+    c, e = _cfg(cfg), _ep(n_gpus, gpu)
+    _check("moe_pw_ep_expert", load_library().moe_pw_ep_expert(
+        ctypes.byref(c), ctypes.byref(e), ctypes.byref(peers), _ptr(recv_x), _ptr(recv_hdr),
+        _ptr(recv_row), _ptr(scale), wave_mask, _stream(stream)))
+
+
+def moe_pw_ep_combine(cfg, n_gpus, gpu, ret_x, ret_hdr, slot_map, gates, out, counters,
+                      stream=None):
+    c, e = _cfg(cfg), _ep(n_gpus, gpu)
+    _check("moe_pw_ep_combine", load_library().moe_pw_ep_combine(
+        ctypes.byref(c), ctypes.byref(e), _ptr(ret_x), _ptr(ret_hdr), _ptr(slot_map), _ptr(gates),
+        _ptr(out), _ptr(counters), _stream(stream)))
+
+
+def moe_pw_ep_stats(cfg, n_gpus, gpu, counters, expert_counts=None, host_expert_counts=None,
+                    stream=None, raise_on_device_error: bool = True) -> moe_pw_drop_stats:
+    c, e = _cfg(cfg), _ep(n_gpus, gpu)
+    out = moe_pw_drop_stats()
+    hp = None
+    if host_expert_counts is not None:
+        assert host_expert_counts.dtype == np.int32 and host_expert_counts.flags.c_contiguous
+        hp = host_expert_counts.ctypes.data
+    rc = load_library().moe_pw_ep_stats(ctypes.byref(c), ctypes.byref(e), _ptr(counters),
+                                        _ptr(expert_counts), ctypes.byref(out), hp,
+                                        _stream(stream))
+    if rc == MOE_PW_EDEVICE and not raise_on_device_error:
+        return out
+    _check("moe_pw_ep_stats", rc)
+    return out
+
+
+def moe_pw_ipc_export(t) -> moe_pw_ipc_handle:
+    h = moe_pw_ipc_handle()
+    _check("moe_pw_ipc_export", load_library().moe_pw_ipc_export(_ptr(t), ctypes.byref(h)))
+    return h
+
+
+def moe_pw_ipc_open(h: moe_pw_ipc_handle) -> int:
+    p = ctypes.c_void_p()
+    _check("moe_pw_ipc_open", load_library().moe_pw_ipc_open(ctypes.byref(h), ctypes.byref(p)))
+    return int(p.value)
+
+
+def moe_pw_ipc_close(ptr: int, h: moe_pw_ipc_handle):
+    _check("moe_pw_ipc_close", load_library().moe_pw_ipc_close(ptr, ctypes.byref(h)))
 
 
 COUNTERS_BYTES = ctypes.sizeof(moe_pw_counters)
@@ -385,12 +531,14 @@ class Buffers:
                                  self.counters, stream)
 
     def run_routed_layer(self, h, w_down_t, w_up_t, model_width: int, latent_bf16, out_model,
-                         stream=None):
+                         stream=None, shared_out=None):
         """The whole routed branch from model width back to model width:
         route -> assign -> down-projection fused with the pack -> bucket ->
         expert op -> combine (bf16 latent) -> up-projection.  h: bf16 [T, Dm],
         w_down_t: bf16 [D, Dm], w_up_t: bf16 [Dm, D], latent_bf16: bf16 [T, D]
-        (scratch), out_model: bf16 [T, Dm]."""
+        (scratch), out_model: bf16 [T, Dm].  With shared_out (bf16 [T, Dm],
+        the shared experts' output) the up-projection's epilogue adds it: the
+        merge of the two paths."""
         cfg = self.cfg
         self.route(stream)
         self.assign(stream)
@@ -400,8 +548,70 @@ class Buffers:
         self.expert(stream)
         moe_pw_combine_bf16(cfg, self.ret_x, self.ret_hdr, self.slot_map, self.gates, latent_bf16,
                             self.counters, stream)
-        moe_pw_project(latent_bf16, w_up_t, out_model, cfg.T, model_width, cfg.D, self.counters,
-                       stream)
+        if shared_out is None:
+            moe_pw_project(latent_bf16, w_up_t, out_model, cfg.T, model_width, cfg.D,
+                           self.counters, stream)
+        else:
+            moe_pw_project_add(latent_bf16, w_up_t, shared_out, out_model, cfg.T, model_width,
+                               cfg.D, self.counters, stream)
+
+    def run_routed_layer_pipelined(self, h, w_down_t, w_up_t, model_width: int, out_model,
+                                   shared_out=None, chunk_tokens: int = 8192, stream=None,
+                                   side_stream=None, latent_chunks=None):
+        """run_routed_layer with the combine and the up-projection overlapped
+        block by block: the combine of token block c + 1 (HBM-bound) runs on
+        one stream while the up-projection of block c (tensor-bound) runs on
+        another, and the bf16 latent passes through two buffers of
+        chunk_tokens rows (latent_chunks, allocated here if not given) that
+        are rewritten before they can leave L2.  Same kernels, same per-row
+        arithmetic: the output equals run_routed_layer's bit for bit."""
+        cfg = self.cfg
+        dev = self.out.device
+        s0 = stream if stream is not None else torch.cuda.current_stream(dev)
+        if side_stream is None:
+            if getattr(self, "_side", None) is None:
+                self._side = torch.cuda.Stream(dev)
+            side_stream = self._side
+        s1 = side_stream
+        if latent_chunks is None:
+            # kept with the buffers: the side stream may still read them after return
+            key = ("latent_chunks", chunk_tokens)
+            if getattr(self, "_chunks_key", None) != key:
+                self._chunks = [torch.empty((chunk_tokens, cfg.D), dtype=torch.int16, device=dev)
+                                for _ in range(2)]
+                self._chunks_key = key
+            latent_chunks = self._chunks
+        self.route(s0)
+        self.assign(s0)
+        moe_pw_project_pack(cfg, h, w_down_t, model_width, self.idx, self.slot_map, self.occ,
+                            self.pool_x, self.pool_hdr, self.counters, s0)
+        self.bucket(s0)
+        self.expert(s0)
+        n_chunks = (cfg.T + chunk_tokens - 1) // chunk_tokens
+        freed = [None, None]
+        for c in range(n_chunks):
+            t0 = c * chunk_tokens
+            n = min(chunk_tokens, cfg.T - t0)
+            lat = latent_chunks[c % 2]
+            if freed[c % 2] is not None:
+                s0.wait_event(freed[c % 2])
+            moe_pw_combine_bf16_rows(cfg, self.ret_x, self.ret_hdr, self.slot_map, self.gates,
+                                     t0, n, lat, self.counters, s0)
+            ready = torch.cuda.Event()
+            ready.record(s0)
+            s1.wait_event(ready)
+            rows = out_model[t0:t0 + n]
+            if shared_out is None:
+                moe_pw_project(lat, w_up_t, rows, n, model_width, cfg.D, self.counters, s1)
+            else:
+                moe_pw_project_add(lat, w_up_t, shared_out[t0:t0 + n], rows, n, model_width,
+                                   cfg.D, self.counters, s1)
+            done = torch.cuda.Event()
+            done.record(s1)
+            freed[c % 2] = done
+        for ev in freed:
+            if ev is not None:
+                s0.wait_event(ev)
 
     def run_step(self, stream=None):
         """route -> dispatch (assign, pack, bucket) -> expert -> combine."""

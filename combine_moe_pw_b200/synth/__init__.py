@@ -100,6 +100,8 @@ def _load():
                                   ctypes.c_double, ctypes.c_void_p)
         lib.synth_logits.argtypes = [ctypes.c_int, i64, i32, i64, f64, u64, vp]
         lib.synth_x_bf16.argtypes = [i64, i32, u64, vp]
+        lib.synth_logits_rows.argtypes = [ctypes.c_int, i64, i64, i32, i64, f64, u64, vp]
+        lib.synth_x_bf16_rows.argtypes = [i64, i64, i32, u64, vp]
         lib.synth_scales.argtypes = [i32, f64, f64, u64, vp]
         lib.synth_dout_f32.argtypes = [i64, i32, u64, vp]
         lib.synth_matrix_bf16.argtypes = [i64, i64, f64, u64, u64, vp]
@@ -123,6 +125,23 @@ def logits(w: Workload, out: np.ndarray | None = None) -> np.ndarray:
     rc = _load().synth_logits(w.logit_kind, w.T, w.E, w.seq_len, w.sigma_b, w.seed, _ptr(out))
     if rc != 0:
         raise ValueError(f"synth_logits failed for {w}")
+    return out
+
+
+def logits_rows(w: Workload, t0: int, n: int) -> np.ndarray:
+    """Rows [t0, t0 + n) of ``logits(w)`` (one GPU's share of a batch)."""
+    out = np.empty((n, w.E), np.float32)
+    if _load().synth_logits_rows(w.logit_kind, t0, n, w.E, w.seq_len, w.sigma_b, w.seed,
+                                 _ptr(out)) != 0:
+        raise ValueError(f"synth_logits_rows failed for {w}")
+    return out
+
+
+def x_bf16_rows(w: Workload, t0: int, n: int) -> np.ndarray:
+    """Rows [t0, t0 + n) of ``x_bf16(w)``."""
+    out = np.empty((n, w.D), np.uint16)
+    if _load().synth_x_bf16_rows(t0, n, w.D, w.seed, _ptr(out)) != 0:
+        raise ValueError("synth_x_bf16_rows failed")
     return out
 
 

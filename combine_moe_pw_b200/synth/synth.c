@@ -72,10 +72,20 @@ enum { ST_LOGIT = 1, ST_SEQBIAS = 2, ST_X = 3, ST_SCALE = 4, ST_PERM = 5, ST_DOU
  *           (Zipf popularity with exponent 1 over a shuffled expert order)
  * The sum is formed in double and rounded once to fp32.
  */
+int synth_logits_rows(int kind, int64_t t0, int64_t T, int32_t E, int64_t seq_len,
+                      double sigma_b, uint64_t seed, float *out);
+
 int synth_logits(int kind, int64_t T, int32_t E, int64_t seq_len, double sigma_b,
                  uint64_t seed, float *out)
 {
-    if (T < 0 || E <= 0 || !out) return -1;
+    return synth_logits_rows(kind, 0, T, E, seq_len, sigma_b, seed, out);
+}
+
+/* Rows t0 .. t0+T-1 of the same logits (a slice of a larger batch). */
+int synth_logits_rows(int kind, int64_t t0, int64_t T, int32_t E, int64_t seq_len,
+                      double sigma_b, uint64_t seed, float *out)
+{
+    if (t0 < 0 || T < 0 || E <= 0 || !out) return -1;
     if (kind == 1 && seq_len <= 0) return -1;
     const uint64_t kz = stream_key(seed, ST_LOGIT);
     const uint64_t kb = stream_key(seed, ST_SEQBIAS);
@@ -94,7 +104,8 @@ int synth_logits(int kind, int64_t T, int32_t E, int64_t seq_len, double sigma_b
         }
     }
 #pragma omp parallel for schedule(static)
-    for (int64_t t = 0; t < T; ++t) {
+    for (int64_t i = 0; i < T; ++i) {
+        const int64_t t = t0 + i;
         for (int32_t e = 0; e < E; ++e) {
             double v = draw_normal(kz, (uint64_t)t * (uint64_t)E + (uint64_t)e);
             if (kind == 1) {
@@ -103,22 +114,28 @@ int synth_logits(int kind, int64_t T, int32_t E, int64_t seq_len, double sigma_b
             } else if (kind == 2) {
                 v -= lnrank[e];
             }
-            out[t * E + e] = (float)v;
+            out[i * E + e] = (float)v;
         }
     }
     return 0;
 }
 
-/* Latent rows, row-major [T, D] bf16 bits: N(0,1) rounded to fp32, then to bf16 (RNE). */
-int synth_x_bf16(int64_t T, int32_t D, uint64_t seed, uint16_t *out)
+/* Latent rows t0 .. t0+T-1, row-major [T, D] bf16 bits: N(0,1) rounded to
+ * fp32, then to bf16 (RNE). */
+int synth_x_bf16_rows(int64_t t0, int64_t T, int32_t D, uint64_t seed, uint16_t *out)
 {
-    if (T < 0 || D <= 0 || !out) return -1;
+    if (t0 < 0 || T < 0 || D <= 0 || !out) return -1;
     const uint64_t kx = stream_key(seed, ST_X);
-    const int64_t n = T * (int64_t)D;
+    const int64_t n = T * (int64_t)D, i0 = t0 * (int64_t)D;
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i)
-        out[i] = f32_bits_to_bf16((float)draw_normal(kx, (uint64_t)i));
+        out[i] = f32_bits_to_bf16((float)draw_normal(kx, (uint64_t)(i0 + i)));
     return 0;
+}
+
+int synth_x_bf16(int64_t T, int32_t D, uint64_t seed, uint16_t *out)
+{
+    return synth_x_bf16_rows(0, T, D, seed, out);
 }
 
 /* Upstream gradient dL/dout, row-major [T, D] fp32: N(0,1) rounded to fp32. */

@@ -294,6 +294,19 @@ int moe_pw_combine_bf16(const moe_pw_config *cfg, const uint16_t *ret_x, const i
                         moe_pw_counters *counters, cudaStream_t stream);
 
 /*
+ * moe_pw_combine_bf16 for the tokens [first_token, first_token + n_tokens) of
+ * the batch only: out (bf16 [n_tokens, D]) row i is token first_token + i.
+ * Lets the combine of one block of tokens run while the up-projection of the
+ * previous block is on the tensor cores (Buffers.run_routed_layer with
+ * chunk_tokens), so the latent passes through a small buffer that stays in
+ * L2.  MOE_PW_EINVAL if the range leaves the batch.
+ */
+int moe_pw_combine_bf16_rows(const moe_pw_config *cfg, const uint16_t *ret_x,
+                             const int32_t *ret_hdr, const int32_t *slot_map, const float *gates,
+                             int64_t first_token, int64_t n_tokens, uint16_t *out,
+                             moe_pw_counters *counters, cudaStream_t stream);
+
+/*
  * Backward of the combine.  The pages train this model ("Marin 开始公开训练 535B
  * 参数 MoE 模型", section 一) but give no backward; this is the derivative of the
  * forward definitions above.  Given dout = dL/dout (f32 [T, D]):
@@ -341,6 +354,19 @@ int moe_pw_project(const uint16_t *A, const uint16_t *Bt, uint16_t *C, int64_t M
                    int32_t K, moe_pw_counters *counters, cudaStream_t stream);
 
 /*
+ * Up-projection merged with the shared-expert path (section 二: the routed
+ * outputs are projected back to model width before they merge with the two
+ * shared experts, which run locally on every token):
+ *   C[m][n] = bf16_rn(sum_k A[m][k] * Bt[n][k] + add[m][n]),
+ * the sum accumulated in fp32 (TMEM), add (bf16 [M, N], the shared path's
+ * output) added in fp32 in the epilogue, one rounding to bf16.  add may be C
+ * itself (in place).  Shapes, alignment and kernels as moe_pw_project.
+ */
+int moe_pw_project_add(const uint16_t *A, const uint16_t *Bt, const uint16_t *add, uint16_t *C,
+                       int64_t M, int32_t N, int32_t K, moe_pw_counters *counters,
+                       cudaStream_t stream);
+
+/*
  * Down-projection fused with the pack: pool_x[slot] = bf16(h[t] @ w_down_t^T)
  * for every (t, j) the sender kept (slot_map from moe_pw_assign), written by
  * the GEMM epilogue directly into the pool slots, headers as in moe_pw_pack,
@@ -366,6 +392,166 @@ int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint1
 int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
                  const int32_t *expert_counts, moe_pw_drop_stats *host_out,
                  int32_t *host_expert_counts, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Expert parallelism over several GPUs.                                     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * "Marin 开始公开训练 535B 参数 MoE 模型", section 二: the experts sit on a
+ * 64-GPU expert-parallel domain, and the fixed pools cross GPUs in three waves
+ * of identical shape with the expert id in the payload; the huxiu article's
+ * JAX section adds that the exchange should overlap the expert compute.
+ *
+ * Here the R logical ranks are spread over n_gpus GPUs, Rn = R / n_gpus on
+ * each: GPU g holds the token shards of sources s in [g*Rn, (g+1)*Rn) (global
+ * tokens [g*Rn*T_s, (g+1)*Rn*T_s), T_s = T / R) and the experts of
+ * destinations d in [g*Rn, (g+1)*Rn).  Capacities are those of the whole
+ * batch.  On each GPU (n_slots = Rn * R * W * C_s, the same for all three
+ * pool arrays):
+ *   send side   slot_map / occ / ret_x / ret_hdr use the local send slot
+ *               q = ((s_loc*R + d)*W + w)*C_s + c, s_loc = s - g*Rn, i.e. the
+ *               single-GPU slot ids of this GPU's sources;
+ *   receive     recv_x / recv_hdr / recv_row use the receive slot
+ *   side        rq = ((s*Rn + d_loc)*W + w)*C_s + c, d_loc = d - g*Rn, for all
+ *               R sources s;
+ *   buckets     bucket_slot [Rn*L, C_r] (receive slots) and expert_counts
+ *               [2, Rn*L] cover the local experts e - g*Rn*L.
+ * Every array of GPU g holds exactly the single-GPU arrays' entries for its
+ * sources or its destinations, relabelled as above.
+ *
+ * The exchange is done by the kernels themselves, over peer memory: the pack
+ * stores each kept row (TMA bulk store, no multicast) and its header straight
+ * into the receive pool of the destination's GPU, and zero-fills the empty
+ * pool tails there; the expert op stores each result row into the return
+ * pool of the source's GPU.  The peer addresses come from a table
+ * (moe_pw_ep_peers): device pointers as this GPU addresses them, from
+ * cudaIpcOpenMemHandle (moe_pw_ipc_open) or, for this GPU's own entry or GPUs
+ * of one process, plain device pointers.
+ *
+ * Order across GPUs is the caller's: every GPU's pack must be complete before
+ * any GPU buckets those waves, and every expert op before any combine (a
+ * stream-ordered barrier, such as a one-element NCCL all-reduce after the
+ * kernels, does it).  The kernels end with a system-scope fence so that their
+ * peer stores are visible once the kernel has completed.
+ *
+ * Waves: wave_mask (bit w = wave w; (1 << W) - 1 = all) selects the waves a
+ * pack, bucket or expert call handles, so wave w can be exchanged while the
+ * expert op of wave w - 1 runs.  Pooled mode only.
+ */
+#define MOE_PW_EP_MAX_GPUS 64
+
+typedef struct moe_pw_ep {
+    int32_t n_gpus;  /* GPUs sharing the R logical ranks; R % n_gpus == 0 */
+    int32_t gpu;     /* this GPU's index, 0 <= gpu < n_gpus */
+} moe_pw_ep;
+
+/* Where the kernels of this GPU write: entry h is GPU h's array, as a device
+ * pointer valid on this GPU (entries >= n_gpus are ignored). */
+typedef struct moe_pw_ep_peers {
+    uint16_t *recv_x[MOE_PW_EP_MAX_GPUS];   /* bf16 [n_slots, D] receive pools */
+    int32_t *recv_hdr[MOE_PW_EP_MAX_GPUS];  /* i32 [n_slots] their headers */
+    uint16_t *ret_x[MOE_PW_EP_MAX_GPUS];    /* bf16 [n_slots, D] return pools */
+    int32_t *ret_hdr[MOE_PW_EP_MAX_GPUS];   /* i32 [n_slots] their headers */
+} moe_pw_ep_peers;
+
+/* Per-GPU sizes (element counts unless "bytes"). */
+typedef struct moe_pw_ep_sizes {
+    int64_t tokens;          /* Rn * T_s tokens on this GPU */
+    int64_t first_token;     /* global index of its first token */
+    int64_t C_s, C_r;        /* capacities of the whole batch */
+    int64_t n_pools;         /* Rn * R * W send pools */
+    int64_t n_slots;         /* rows of every pool array on this GPU */
+    int64_t local_experts;   /* Rn * L */
+    int64_t bucket_len;      /* local_experts * C_r */
+    int64_t workspace_bytes; /* scratch for moe_pw_ep_assign */
+    int64_t total_bytes;     /* every buffer of this GPU's share */
+} moe_pw_ep_sizes;
+
+/* Host-only: validates cfg (pooled mode) and ep and fills *out; with
+ * budget_bytes > 0, MOE_PW_ENOMEM when out->total_bytes exceeds it. */
+int moe_pw_ep_plan(const moe_pw_config *cfg, const moe_pw_ep *ep, int64_t budget_bytes,
+                   moe_pw_ep_sizes *out);
+
+/* moe_pw_route on this GPU's tokens (logits f32 [tokens, E]). */
+int moe_pw_ep_route(const moe_pw_config *cfg, const moe_pw_ep *ep, const float *logits,
+                    int32_t *idx, float *gates, cudaStream_t stream);
+
+/* moe_pw_assign for this GPU's sources: slot_map [tokens, k] receives local
+ * send slots, occ [Rn, R, W] the rows kept per pool.  Zeroes *counters. */
+int moe_pw_ep_assign(const moe_pw_config *cfg, const moe_pw_ep *ep, const int32_t *idx,
+                     int32_t *slot_map, int32_t *occ, moe_pw_counters *counters,
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Pack and send (section 二: fixed per-destination pools, expert id in the
+ * payload).  For every kept (t, j) whose wave is in wave_mask, the row x[t]
+ * (loaded once into shared memory) is bulk-stored into the receive pool of
+ * the destination's GPU (peers->recv_x[d / Rn]) at its receive slot, with the
+ * expert id as its header; the empty tails (c >= occ) of this GPU's pools of
+ * those waves get zero rows and header -1 there.  Uses counters->work like
+ * moe_pw_pack.  x bf16 [tokens, D].
+ */
+int moe_pw_ep_pack(const moe_pw_config *cfg, const moe_pw_ep *ep, const moe_pw_ep_peers *peers,
+                   const uint16_t *x, const int32_t *idx, const int32_t *slot_map,
+                   const int32_t *occ, uint32_t wave_mask, moe_pw_counters *counters,
+                   cudaStream_t stream);
+
+/*
+ * Receiver bucketing (section 二: receiver factor) over this GPU's receive
+ * pool, for the waves in wave_mask: per (local destination, wave), sources
+ * ascending, then slots ascending; an empty slot is recognised by its header
+ * -1 alone (no counts are exchanged).  Writes recv_row, bucket_slot (receive
+ * slots) and expert_counts of the local experts of those waves and adds
+ * receiver drops and kept rows to *counters.
+ */
+int moe_pw_ep_bucket(const moe_pw_config *cfg, const moe_pw_ep *ep, const int32_t *recv_hdr,
+                     int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,
+                     uint32_t wave_mask, moe_pw_counters *counters, cudaStream_t stream);
+
+/*
+ * Per-expert op and return trip (huxiu: results come back by a second
+ * all-to-all).  For every receive slot of the waves in wave_mask: if the
+ * receiver kept it, bf16_rn(scale[e] * row) and header e, else zeros and -1,
+ * stored into the return pool of the source's GPU (peers->ret_x[s / Rn]) at
+ * the source's send slot.
+ */
+int moe_pw_ep_expert(const moe_pw_config *cfg, const moe_pw_ep *ep, const moe_pw_ep_peers *peers,
+                     const uint16_t *recv_x, const int32_t *recv_hdr, const int32_t *recv_row,
+                     const float *scale, uint32_t wave_mask, cudaStream_t stream);
+
+/* moe_pw_combine on this GPU's tokens and return pool (out f32 [tokens, D]). */
+int moe_pw_ep_combine(const moe_pw_config *cfg, const moe_pw_ep *ep, const uint16_t *ret_x,
+                      const int32_t *ret_hdr, const int32_t *slot_map, const float *gates,
+                      float *out, moe_pw_counters *counters, cudaStream_t stream);
+
+/* moe_pw_stats for this GPU: assignments = tokens * k; sender drops of its
+ * sources; receiver drops, kept rows and expert_counts ([2, Rn*L]) of its
+ * experts.  Summed over the GPUs they give the whole batch's statistics. */
+int moe_pw_ep_stats(const moe_pw_config *cfg, const moe_pw_ep *ep,
+                    const moe_pw_counters *counters, const int32_t *expert_counts,
+                    moe_pw_drop_stats *host_out, int32_t *host_expert_counts,
+                    cudaStream_t stream);
+
+/*
+ * Sharing device buffers between the processes of an expert-parallel run
+ * (one process per GPU).  moe_pw_ipc_export describes the allocation that
+ * holds dev_ptr (cudaIpcGetMemHandle of its base) and dev_ptr's offset in it;
+ * moe_pw_ipc_open maps such a description exported by another process into
+ * this one (cudaIpcOpenMemHandle with peer access enabled) and returns the
+ * same byte as a pointer valid on the current device; moe_pw_ipc_close
+ * unmaps it (pass the pointer open returned and the same description).  A
+ * process cannot open its own handles; use the pointer itself.  Host-only,
+ * synchronous.
+ */
+typedef struct moe_pw_ipc_handle {
+    unsigned char handle[64];  /* cudaIpcMemHandle_t of the allocation */
+    uint64_t offset;           /* dev_ptr - allocation base */
+} moe_pw_ipc_handle;
+
+int moe_pw_ipc_export(const void *dev_ptr, moe_pw_ipc_handle *out);
+int moe_pw_ipc_open(const moe_pw_ipc_handle *h, void **dev_ptr);
+int moe_pw_ipc_close(void *dev_ptr, const moe_pw_ipc_handle *h);
 
 /*
  * Self-test of failure detection (no counterpart on the pages): launches one

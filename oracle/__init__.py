@@ -111,7 +111,7 @@ def _configure(lib):
     lib.orc_combine_backward.argtypes = [gp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.orc_dispatch_backward.argtypes = [gp, vp, vp, vp, vp]
     lib.orc_backward_tokens.argtypes = [gp, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp]
-    lib.orc_project.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp]
+    lib.orc_project.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp]
     lib.orc_bf16_round.argtypes = [vp, vp, i64]
     lib.orc_expert_product.argtypes = [vp, vp, vp, i64]
     return lib
@@ -385,18 +385,21 @@ def run_backward(w, r: dict, dout: np.ndarray, scale: np.ndarray) -> dict:
     return b
 
 
-def project(A: np.ndarray, Bt: np.ndarray, exact: bool = False):
-    """C = bf16(A @ Bt^T) (bf16 bits); with exact=True also the double sums
-    and sum |terms|."""
+def project(A: np.ndarray, Bt: np.ndarray, exact: bool = False, add: np.ndarray | None = None):
+    """C = bf16(A @ Bt^T [+ add]) (bf16 bits); with exact=True also the
+    double sums and sum |terms|."""
     A, Bt = _c(A, np.uint16), _c(Bt, np.uint16)
     M, K = A.shape
     N = Bt.shape[0]
     assert Bt.shape[1] == K
+    if add is not None:
+        add = _c(add, np.uint16)
+        assert add.shape == (M, N)
     C = np.empty((M, N), np.uint16)
     Ce = np.empty((M, N), np.float64) if exact else None
     mag = np.empty((M, N), np.float64) if exact else None
-    _load().orc_project(_p(A), _p(Bt), M, N, K, _p(C), _p(Ce) if exact else None,
-                        _p(mag) if exact else None)
+    _load().orc_project(_p(A), _p(Bt), M, N, K, _p(add) if add is not None else None, _p(C),
+                        _p(Ce) if exact else None, _p(mag) if exact else None)
     return (C, Ce, mag) if exact else C
 
 

@@ -647,11 +647,16 @@ void orc_backward_tokens(const orc_geom *g, const uint16_t *x, const int32_t *id
  *   C[m][n] = bf16( sum_k A[m][k] * Bt[n][k] ),
  * the sum in double, rounded to fp32 and then to bf16 nearest-even (the
  * device accumulates in fp32).  Bt is stored row n = output column n.
- * Also returns, per element, sum_k |A[m][k] * Bt[n][k]| (the accumulation
- * error is measured against it).
+ * The merge with the shared path (same passage: routed outputs, back at model
+ * width, meet the shared experts' output) is READ as a plain sum: with add
+ * (bf16 [M, N], the shared path's output) given,
+ *   C[m][n] = bf16( sum_k A[m][k] * Bt[n][k] + add[m][n] ),
+ * again formed in double and rounded once through fp32.
+ * Also returns, per element, the exact value and sum_k |A[m][k] * Bt[n][k]|
+ * plus |add[m][n]| (the accumulation error is measured against it).
  */
 void orc_project(const uint16_t *A, const uint16_t *Bt, int64_t M, int64_t N, int64_t K,
-                 uint16_t *C, double *Cexact, double *mag)
+                 const uint16_t *add, uint16_t *C, double *Cexact, double *mag)
 {
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t n = 0; n < N; ++n) {
@@ -660,6 +665,11 @@ void orc_project(const uint16_t *A, const uint16_t *Bt, int64_t M, int64_t N, in
                 const double p = (double)bf16_to_f32(A[m * K + kk]) * (double)bf16_to_f32(Bt[n * K + kk]);
                 acc += p;
                 am += fabs(p);
+            }
+            if (add) {
+                const double s = (double)bf16_to_f32(add[m * N + n]);
+                acc += s;
+                am += fabs(s);
             }
             C[m * N + n] = f32_to_bf16_rne((float)acc);
             if (Cexact) Cexact[m * N + n] = acc;

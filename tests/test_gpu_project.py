@@ -184,6 +184,109 @@ def test_routed_layer_against_oracle_chain(name, Dm):
                              f"x {xf[t, i]!r} c {c[t, 0]!r} bad {bad.sum()}")
 
 
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 264, 200), (1, 8, 8),
+                                   (129, 1032, 2072), (515, 512, 3072)])
+def test_project_add_merges_shared_path(M, N, K):
+    """C = bf16(A @ Bt^T + add) against the oracle's merge, with the
+    projection's bound (its magnitude now includes |add|); then in place
+    (add is C) with the same bytes."""
+    A = synth.matrix_bf16(M, K, 1.0, 60)
+    Bt = synth.matrix_bf16(N, K, K ** -0.5, 61)
+    S = synth.matrix_bf16(M, N, 1.0, 62)
+    a = torch.from_numpy(A.view(np.int16)).cuda()
+    b = torch.from_numpy(Bt.view(np.int16)).cuda()
+    sh = torch.from_numpy(S.view(np.int16)).cuda()
+    c = torch.full((M, N), 0x7FC0, dtype=torch.int16, device="cuda")
+    ctr = _ctr()
+    mp.moe_pw_project_add(a, b, sh, c, M, N, K, ctr)
+    inplace = sh.clone()
+    mp.moe_pw_project_add(a, b, inplace, inplace, M, N, K, ctr)
+    torch.cuda.synchronize()
+    assert mp.moe_pw_stats(mp.Config(T=0, E=8, k=1, D=8, R=1, L=8, W=1, P=8), ctr).error == 0
+    C = c.cpu().numpy().view(np.uint16)
+    Cr, Ce, mag = oracle.project(A, Bt, exact=True, add=S)
+    got = _f64(C)
+    assert np.all(np.isfinite(got))
+    assert np.all(np.abs(got - Ce) <= 2.0 ** -8 * np.abs(Ce) + 2.0 ** -20 * mag + 1e-30)
+    assert (C != Cr).mean() < 0.02
+    assert torch.equal(inplace, c)
+
+
+def test_routed_layer_with_shared_merge():
+    """The routed branch ending in the merge: the up-projection's epilogue
+    adds the shared path's output.  Against the oracle's chain extended by
+    the same merge, with the routed-layer bound."""
+    w = synth.WORKLOADS["tiny"]
+    Dm = 256
+    lg, s = synth.logits(w), synth.scales(w)
+    h, wd, wu = synth.projection_inputs(w, Dm)
+    S = synth.matrix_bf16(w.T, Dm, 1.0, 63)
+    b = mp.Buffers(mp.Config.from_workload(w))
+    b.logits.copy_(torch.from_numpy(lg))
+    b.scale.copy_(torch.from_numpy(s))
+    lat = torch.empty((w.T, w.D), dtype=torch.int16, device="cuda")
+    out = torch.empty((w.T, Dm), dtype=torch.int16, device="cuda")
+    b.run_routed_layer(torch.from_numpy(h.view(np.int16)).cuda(),
+                       torch.from_numpy(wd.view(np.int16)).cuda(),
+                       torch.from_numpy(wu.view(np.int16)).cuda(), Dm, lat, out,
+                       shared_out=torch.from_numpy(S.view(np.int16)).cuda())
+    assert b.stats().error == 0
+    x = oracle.project(h, wd)
+    r = oracle.run(w, lg, x, s)
+    lat_ref = oracle.bf16_round(r["out"].astype(np.float32))
+    _, out_exact, mag = oracle.project(lat_ref, wu, exact=True, add=S)
+    got = _f64(out.cpu().numpy().view(np.uint16))
+    err = np.abs(got - out_exact)
+    assert np.all(err <= 2.0 ** -6 * mag + 2.0 ** -8 * np.abs(out_exact) + 1e-30)
+    assert (err <= 2.0 ** -8 * np.abs(out_exact) + 2.0 ** -18 * mag).mean() > 0.99
+
+
+@pytest.mark.parametrize("chunk", [1000, 2048, 4096])
+def test_pipelined_routed_layer_equals_sequential(chunk):
+    """The routed layer with the combine and the up-projection overlapped in
+    token blocks (two latent buffers, two streams): the same bytes as the
+    sequential chain, with and without the shared-path merge; block sizes
+    that divide the batch and one that leaves a ragged last block."""
+    w = synth.Workload("pages_small", T=64 * 64, R=64, L=6, W=3, P=2, k=8, D=512, seq_len=1024,
+                       logit_kind=synth.LOGIT_SEQBIAS)
+    Dm = 1024
+    lg, s = synth.logits(w), synth.scales(w)
+    h, wd, wu = (torch.from_numpy(a.view(np.int16)).cuda() for a in synth.projection_inputs(w, Dm))
+    S = torch.from_numpy(synth.matrix_bf16(w.T, Dm, 1.0, 64).view(np.int16)).cuda()
+    b = mp.Buffers(mp.Config.from_workload(w))
+    b.logits.copy_(torch.from_numpy(lg))
+    b.scale.copy_(torch.from_numpy(s))
+    lat = torch.empty((w.T, w.D), dtype=torch.int16, device="cuda")
+    for shared in (None, S):
+        ref = torch.empty((w.T, Dm), dtype=torch.int16, device="cuda")
+        b.run_routed_layer(h, wd, wu, Dm, lat, ref, shared_out=shared)
+        got = torch.full((w.T, Dm), 0x7FC0, dtype=torch.int16, device="cuda")
+        b.run_routed_layer_pipelined(h, wd, wu, Dm, got, shared_out=shared, chunk_tokens=chunk)
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref)
+    assert b.stats().error == 0
+
+
+def test_combine_rows_is_the_combine_of_those_tokens():
+    w = synth.WORKLOADS["tiny"]
+    lg = synth.logits(w)
+    b = mp.Buffers(mp.Config.from_workload(w))
+    b.logits.copy_(torch.from_numpy(lg))
+    b.x.copy_(torch.from_numpy(synth.x_bf16(w).view(np.int16)))
+    b.scale.copy_(torch.from_numpy(synth.scales(w)))
+    b.run_step()
+    full = torch.empty((w.T, w.D), dtype=torch.int16, device="cuda")
+    mp.moe_pw_combine_bf16(b.cfg, b.ret_x, b.ret_hdr, b.slot_map, b.gates, full, b.counters)
+    part = torch.full((300, w.D), 0x7FC0, dtype=torch.int16, device="cuda")
+    mp.moe_pw_combine_bf16_rows(b.cfg, b.ret_x, b.ret_hdr, b.slot_map, b.gates, 1001, 300, part,
+                                b.counters)
+    torch.cuda.synchronize()
+    assert torch.equal(part, full[1001:1301])
+    with pytest.raises(mp.MoePwError):
+        mp.moe_pw_combine_bf16_rows(b.cfg, b.ret_x, b.ret_hdr, b.slot_map, b.gates, w.T - 5, 6,
+                                    part, b.counters)
+
+
 _FALLBACK_SHAPES = [(300, 264, 200), (129, 264, 4096), (512, 768, 1024), (1, 8, 8)]
 
 _FALLBACK_CHILD = r"""

@@ -36,3 +36,23 @@ def test_projection_inputs_shapes():
     h, wd, wu = synth.projection_inputs(w, model_width=256)
     assert h.shape == (16, 256) and wd.shape == (w.D, 256) and wu.shape == (256, w.D)
     assert abs(_f64(wd).std() - 256 ** -0.5) < 0.01
+
+
+def test_project_with_shared_path_merge():
+    """The merge with the shared path: bf16(A @ Bt^T + add), formed exactly
+    and rounded once, against numpy's float64 product plus the addend and
+    torch's fp32 -> bf16 rounding; add = 0 gives the plain projection."""
+    A = synth.matrix_bf16(29, 136, 1.0, 23)
+    Bt = synth.matrix_bf16(40, 136, 136 ** -0.5, 24)
+    add = synth.matrix_bf16(29, 40, 1.0, 25)
+    C, Ce, mag = oracle.project(A, Bt, exact=True, add=add)
+    ref = _f64(A) @ _f64(Bt).T + _f64(add)
+    np.testing.assert_allclose(Ce, ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(mag, np.abs(_f64(A)) @ np.abs(_f64(Bt)).T + np.abs(_f64(add)),
+                               rtol=1e-12)
+    expect = torch.from_numpy(ref.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy()
+    np.testing.assert_array_equal(C, expect.view(np.uint16))
+    np.testing.assert_array_equal(oracle.project(A, Bt, add=np.zeros((29, 40), np.uint16)),
+                                  oracle.project(A, Bt))
+    # a zero product leaves the addend itself
+    np.testing.assert_array_equal(oracle.project(np.zeros_like(A), Bt, add=add), add)

@@ -75,3 +75,14 @@ def test_workloads_match_recipes():
     for name in ["layer", "rack", "long", "ragged"]:
         w = W[name]
         assert (w.E, w.k, w.D, w.R, w.L, w.W, w.P) == (384, 8, 3072, 64, 6, 3, 2)
+
+
+def test_row_slices_equal_the_whole():
+    """One GPU's share of a batch is generated on its own: rows [t0, t0+n)
+    equal the same rows of the whole batch, for every logit kind."""
+    for kind in (synth.LOGIT_IID, synth.LOGIT_SEQBIAS, synth.LOGIT_ZIPF):
+        w = synth.WORKLOADS["tiny"].with_(logit_kind=kind, seq_len=100)
+        lg, x = synth.logits(w), synth.x_bf16(w)
+        for t0, n in [(0, 5), (37, 300), (w.T - 9, 9)]:
+            np.testing.assert_array_equal(synth.logits_rows(w, t0, n), lg[t0:t0 + n])
+            np.testing.assert_array_equal(synth.x_bf16_rows(w, t0, n), x[t0:t0 + n])
