@@ -733,13 +733,13 @@ def main():
         # one batch at a time on one buffer set
         h_out = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
 
+        h_ctr = torch.empty_like(b.counters, device="cpu").pin_memory()
+        dev_bufs = b.device_buffers()
+
         def e2e_step():
-            b.logits.copy_(h_lg, non_blocking=True)
-            b.x.copy_(h_x, non_blocking=True)
-            b.scale.copy_(h_s, non_blocking=True)
-            b.run_step(stream)
-            h_out.copy_(b.out, non_blocking=True)
-            return b.stats(stream)  # synchronises: the step's result is on the host
+            # the C-ABI step with host buffers: upload, path, download, on one stream
+            mp.moe_pw_step_host(cfg, h_lg, h_x, h_s, h_out, h_ctr, dev_bufs, stream)
+            stream.synchronize()  # the step's result is on the host
 
         for _ in range(2):
             e2e_step()
@@ -775,6 +775,7 @@ def main():
         e2e = {"value": throughput(w.T * w.k, ke, world, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / ke, "pipeline_depth": 2,
+               "api": "moe_pw_step_host (C ABI, host buffers in and out)",
                "serial_ms_per_step": serial_ms,
                "serial_value": throughput(w.T * w.k, 1, world, serial_ms)}
         del pipe

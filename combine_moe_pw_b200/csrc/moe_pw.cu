@@ -222,7 +222,8 @@ int moe_pw_assign(const moe_pw_config *cfg, const int32_t *idx, int32_t *slot_ma
 
 int moe_pw_pack(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
                 const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr,
-                moe_pw_counters *counters, cudaStream_t stream)
+                moe_pw_counters *counters, void *workspace, size_t workspace_bytes,
+                cudaStream_t stream)
 {
     Geo g;
     int rc = make_geo(cfg, &g);
@@ -232,7 +233,15 @@ int moe_pw_pack(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
     if (!aligned(x, 16) || !aligned(pool_x, 16) || !aligned(idx, 4) || !aligned(slot_map, 4) ||
         !aligned(occ, 4) || !aligned(pool_hdr, 4) || !aligned(counters, 8))
         return MOE_PW_EUNSUPPORTED;
-    return cuda_rc(launch_pack(g, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream));
+    // the workspace only serves the dropless mode; too small or absent, the
+    // pack sweeps the tokens instead
+    void *ws = nullptr;
+    if (g.mode == MOE_PW_RAGGED && workspace && int64_t(workspace_bytes) >= ws_bytes(g)) {
+        if (!aligned(workspace, 256)) return MOE_PW_EUNSUPPORTED;
+        ws = workspace;
+    }
+    return cuda_rc(launch_pack(g, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream,
+                               nullptr, ~0u, ws));
 }
 
 int moe_pw_bucket(const moe_pw_config *cfg, const int32_t *pool_hdr, const int32_t *occ,
@@ -260,7 +269,8 @@ int moe_pw_dispatch(const moe_pw_config *cfg, const uint16_t *x, const int32_t *
 {
     int rc = moe_pw_assign(cfg, idx, slot_map, occ, counters, workspace, workspace_bytes, stream);
     if (rc != MOE_PW_OK) return rc;
-    rc = moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream);
+    rc = moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, workspace,
+                     workspace_bytes, stream);
     if (rc != MOE_PW_OK) return rc;
     return moe_pw_bucket(cfg, pool_hdr, occ, recv_row, bucket_slot, expert_counts, counters,
                          stream);
@@ -539,6 +549,81 @@ extern "C" int moe_pw_selftest_wait_timeout(moe_pw_counters *counters, int32_t p
     if (!aligned(counters, 8)) return MOE_PW_EUNSUPPORTED;
     selftest_wait_kernel<<<1, 32, 0, stream>>>(counters, uint32_t(polls));
     return cuda_rc(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------------------
+// One step from host memory to host memory.
+// ---------------------------------------------------------------------------
+
+namespace moe_pw {
+namespace {
+
+// Make `waiter` wait for the work enqueued so far on `signaller` (a one-shot
+// event, released as soon as it is recorded: CUDA keeps it alive until the
+// wait is resolved).  Nothing to do when the two are the same stream.
+cudaError_t order(cudaStream_t signaller, cudaStream_t waiter)
+{
+    if (signaller == waiter) return cudaSuccess;
+    cudaEvent_t ev;
+    cudaError_t e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+    e = cudaEventRecord(ev, signaller);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(waiter, ev, 0);
+    const cudaError_t d = cudaEventDestroy(ev);
+    return e != cudaSuccess ? e : d;
+}
+
+}  // namespace
+}  // namespace moe_pw
+
+extern "C" int moe_pw_step_host(const moe_pw_config *cfg, const float *h_logits,
+                                const uint16_t *h_x, const float *h_scale, float *h_out,
+                                moe_pw_counters *h_counters, const moe_pw_device_buffers *dev,
+                                cudaStream_t compute, cudaStream_t copy_in,
+                                cudaStream_t copy_out)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!dev || !h_scale || !h_counters || !dev->scale || !dev->counters) return MOE_PW_EINVAL;
+    if (g.T > 0 && (!h_logits || !h_x || !h_out || !dev->logits || !dev->x || !dev->out))
+        return MOE_PW_EINVAL;
+    const size_t T = size_t(g.T), E = size_t(g.E), D = size_t(g.D);
+    // inputs up
+    if (T > 0) {
+        if (cudaMemcpyAsync(dev->logits, h_logits, 4 * T * E, cudaMemcpyHostToDevice, copy_in) !=
+                cudaSuccess ||
+            cudaMemcpyAsync(dev->x, h_x, 2 * T * D, cudaMemcpyHostToDevice, copy_in) !=
+                cudaSuccess)
+            return MOE_PW_ECUDA;
+    }
+    if (cudaMemcpyAsync(dev->scale, h_scale, 4 * E, cudaMemcpyHostToDevice, copy_in) !=
+        cudaSuccess)
+        return MOE_PW_ECUDA;
+    if (order(copy_in, compute) != cudaSuccess) return MOE_PW_ECUDA;
+    // the path, every step in this library's kernels
+    if ((rc = moe_pw_route(cfg, dev->logits, dev->idx, dev->gates, compute)) != MOE_PW_OK)
+        return rc;
+    if ((rc = moe_pw_dispatch(cfg, dev->x, dev->idx, dev->slot_map, dev->occ, dev->pool_x,
+                              dev->pool_hdr, dev->recv_row, dev->bucket_slot, dev->expert_counts,
+                              dev->counters, dev->workspace, dev->workspace_bytes, compute)) !=
+        MOE_PW_OK)
+        return rc;
+    if ((rc = moe_pw_expert(cfg, dev->pool_x, dev->pool_hdr, dev->recv_row, dev->scale,
+                            dev->ret_x, dev->ret_hdr, compute)) != MOE_PW_OK)
+        return rc;
+    if ((rc = moe_pw_combine(cfg, dev->ret_x, dev->ret_hdr, dev->slot_map, dev->gates, dev->out,
+                             dev->counters, compute)) != MOE_PW_OK)
+        return rc;
+    // result down
+    if (order(compute, copy_out) != cudaSuccess) return MOE_PW_ECUDA;
+    if (T > 0 &&
+        cudaMemcpyAsync(h_out, dev->out, 4 * T * D, cudaMemcpyDeviceToHost, copy_out) != cudaSuccess)
+        return MOE_PW_ECUDA;
+    if (cudaMemcpyAsync(h_counters, dev->counters, sizeof(moe_pw_counters), cudaMemcpyDeviceToHost,
+                        copy_out) != cudaSuccess)
+        return MOE_PW_ECUDA;
+    return MOE_PW_OK;
 }
 
 // ---------------------------------------------------------------------------

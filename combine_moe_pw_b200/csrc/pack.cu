@@ -28,6 +28,7 @@
 // The defaults below came from a sweep on the 262,144-token batch: deeper
 // rings with fewer warps beat more warps with shallow rings; the lag between
 // 8 and 20 made no measurable difference.
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -275,14 +276,30 @@ cudaError_t launch_ep(const PackArgs &p, const DevInfo &di, const Geo &g, int nw
     return launch_lag<2, EP>(p, di, g, nw, smem, st);
 }
 
+// MOE_PW_RAGGED_PACK=sweep in the environment (read once) keeps the dropless
+// mode on the token sweep of this file; by default it writes rows in their
+// own order (pack_ragged.cu).  Both give the same bytes.
+bool ragged_pack_enabled()
+{
+    static const bool on = [] {
+        const char *v = getenv("MOE_PW_RAGGED_PACK");
+        return !(v && strcmp(v, "sweep") == 0);
+    }();
+    return on;
+}
+
 }  // namespace
 
 cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
                         const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
                         int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st,
-                        const EpRows *ep, uint32_t wave_mask)
+                        const EpRows *ep, uint32_t wave_mask, void *ws)
 {
     if (g.T == 0 && g.n_pools == 0) return cudaSuccess;
+    if (g.mode == MOE_PW_RAGGED && ws && !ep && ragged_pack_enabled()) {
+        const cudaError_t e = launch_pack_ragged(g, x, slot_map, occ, pool_x, pool_hdr, ctr, ws, st);
+        if (e != cudaErrorNotSupported) return e;
+    }
     DevInfo di;
     if (dev_info(&di) != 0) return cudaErrorUnknown;
     PackArgs p;

@@ -59,6 +59,13 @@ class moe_pw_drop_stats(ctypes.Structure):
                 ("error", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
+class moe_pw_device_buffers(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "logits", "x", "scale", "idx", "gates", "slot_map", "occ", "pool_x", "pool_hdr",
+        "recv_row", "bucket_slot", "expert_counts", "ret_x", "ret_hdr", "out", "counters",
+        "workspace")] + [("workspace_bytes", ctypes.c_size_t)]
+
+
 EP_MAX_GPUS = 64  # MOE_PW_EP_MAX_GPUS
 
 
@@ -93,7 +100,7 @@ SIGNATURES = {
     "moe_pw_route": [_CFG, _VP, _VP, _VP, _VP],
     "moe_pw_assign": [_CFG, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_assign_noalloc": [_CFG, _VP, _VP, _VP, _VP, _VP],
-    "moe_pw_pack": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_pack": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_bucket": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_dispatch": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_expert": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
@@ -107,6 +114,8 @@ SIGNATURES = {
     "moe_pw_project_pack": [_CFG, _VP, _VP, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_stats": [_CFG, _VP, _VP, ctypes.POINTER(moe_pw_drop_stats), _VP, _VP],
     "moe_pw_selftest_wait_timeout": [_VP, ctypes.c_int32, _VP],
+    "moe_pw_step_host": [_CFG, _VP, _VP, _VP, _VP, _VP, ctypes.POINTER(moe_pw_device_buffers),
+                         _VP, _VP, _VP],
     "moe_pw_ep_plan": [_CFG, ctypes.POINTER(moe_pw_ep), _I64, ctypes.POINTER(moe_pw_ep_sizes)],
     "moe_pw_ep_route": [_CFG, ctypes.POINTER(moe_pw_ep), _VP, _VP, _VP, _VP],
     "moe_pw_ep_assign": [_CFG, ctypes.POINTER(moe_pw_ep), _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
@@ -232,11 +241,13 @@ def moe_pw_assign_noalloc(cfg, idx, slot_map, occ, counters, stream=None):
         ctypes.byref(c), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(counters), _stream(stream)))
 
 
-def moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream=None):
+def moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream=None,
+                workspace=None):
     c = _cfg(cfg)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("moe_pw_pack", load_library().moe_pw_pack(
         ctypes.byref(c), _ptr(x), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(pool_x),
-        _ptr(pool_hdr), _ptr(counters), _stream(stream)))
+        _ptr(pool_hdr), _ptr(counters), _ptr(workspace), wsb, _stream(stream)))
 
 
 def moe_pw_bucket(cfg, pool_hdr, occ, recv_row, bucket_slot, expert_counts, counters, stream=None):
@@ -345,6 +356,19 @@ def moe_pw_selftest_wait_timeout(counters, polls: int = 4096, stream=None):
     """Run the bounded-wait self-test (see include/moe_pw.h)."""
     _check("moe_pw_selftest_wait_timeout", load_library().moe_pw_selftest_wait_timeout(
         _ptr(counters), polls, _stream(stream)))
+
+
+def moe_pw_step_host(cfg, h_logits, h_x, h_scale, h_out, h_counters,
+                     dev: moe_pw_device_buffers, compute=None, copy_in=None, copy_out=None):
+    """One step from host buffers to host buffers, enqueued on three streams
+    (see include/moe_pw.h).  Host arrays: pinned torch CPU tensors."""
+    c = _cfg(cfg)
+    s_c = _stream(compute)
+    s_i = s_c if copy_in is None else _stream(copy_in)
+    s_o = s_c if copy_out is None else _stream(copy_out)
+    _check("moe_pw_step_host", load_library().moe_pw_step_host(
+        ctypes.byref(c), _ptr(h_logits), _ptr(h_x), _ptr(h_scale), _ptr(h_out),
+        _ptr(h_counters), ctypes.byref(dev), s_c, s_i, s_o))
 
 
 def _ep(n_gpus: int, gpu: int) -> moe_pw_ep:
@@ -472,6 +496,16 @@ class Buffers:
         self.counters = torch.zeros((COUNTERS_BYTES // 8,), dtype=torch.int64, device=dev)
         self.workspace = torch.empty((max(s.workspace_bytes, 256),), dtype=torch.uint8, device=dev)
 
+    def device_buffers(self) -> moe_pw_device_buffers:
+        """The device arrays as the C struct moe_pw_step_host takes."""
+        d = moe_pw_device_buffers()
+        for name in ("logits", "x", "scale", "idx", "gates", "slot_map", "occ", "pool_x",
+                     "pool_hdr", "recv_row", "bucket_slot", "expert_counts", "ret_x", "ret_hdr",
+                     "out", "counters", "workspace"):
+            setattr(d, name, getattr(self, name).data_ptr())
+        d.workspace_bytes = self.workspace.numel()
+        return d
+
     def route(self, stream=None):
         moe_pw_route(self.cfg, self.logits, self.idx, self.gates, stream)
 
@@ -486,7 +520,7 @@ class Buffers:
 
     def pack(self, stream=None):
         moe_pw_pack(self.cfg, self.x, self.idx, self.slot_map, self.occ, self.pool_x,
-                    self.pool_hdr, self.counters, stream)
+                    self.pool_hdr, self.counters, stream, self.workspace)
 
     def bucket(self, stream=None):
         moe_pw_bucket(self.cfg, self.pool_hdr, self.occ, self.recv_row, self.bucket_slot,
@@ -661,33 +695,26 @@ class Pipeline:
         self.inputs_free = [None] * depth   # compute of the last batch in set b has read its inputs
         self.output_free = [None] * depth   # last output of set b is on the host
         self.h_counters = [torch.empty_like(b.counters, device="cpu").pin_memory() for b in self.bufs]
+        self.dev = [b.device_buffers() for b in self.bufs]
 
     def submit(self, h_logits, h_x, h_scale, h_out):
         """Queue one batch: pinned host logits f32 [T,E], x bf16 bits [T,D],
-        scale f32 [E]; the result lands in pinned host h_out f32 [T,D]."""
+        scale f32 [E]; the result lands in pinned host h_out f32 [T,D].  The
+        library's moe_pw_step_host enqueues the upload, the path and the
+        download; this only orders the reuse of each buffer set."""
         k = self.n % self.depth
         b, sc = self.bufs[k], self.s_comp[k]
-        with torch.cuda.stream(self.s_in):
-            if self.inputs_free[k] is not None:
-                self.s_in.wait_event(self.inputs_free[k])
-            b.logits.copy_(h_logits, non_blocking=True)
-            b.x.copy_(h_x, non_blocking=True)
-            b.scale.copy_(h_scale, non_blocking=True)
-            landed = torch.cuda.Event()
-            landed.record(self.s_in)
-        sc.wait_event(landed)
+        if self.inputs_free[k] is not None:
+            self.s_in.wait_event(self.inputs_free[k])   # inputs read by the last compute
         if self.output_free[k] is not None:
-            sc.wait_event(self.output_free[k])
-        b.run_step(sc)
+            sc.wait_event(self.output_free[k])          # output read by the last download
+        moe_pw_step_host(self.cfg, h_logits, h_x, h_scale, h_out, self.h_counters[k],
+                         self.dev[k], sc, self.s_in, self.s_out)
         done = torch.cuda.Event()
         done.record(sc)
         self.inputs_free[k] = done
-        with torch.cuda.stream(self.s_out):
-            self.s_out.wait_event(done)
-            h_out.copy_(b.out, non_blocking=True)
-            self.h_counters[k].copy_(b.counters, non_blocking=True)
-            out_done = torch.cuda.Event()
-            out_done.record(self.s_out)
+        out_done = torch.cuda.Event()
+        out_done.record(self.s_out)
         self.output_free[k] = out_done
         self.n += 1
         return k

@@ -205,16 +205,24 @@ int moe_pw_assign(const moe_pw_config *cfg, const int32_t *idx, int32_t *slot_ma
  * Pack (section 二: expert id in the payload).  Copies each kept row x[t] into
  * its slot with TMA bulk copies through shared memory (one read of x[t], up to
  * k writes), writes the expert id into the slot header, and fills the empty
- * tail of every pool (positions >= occ) with zeros and header -1.  Ragged
- * mode: rows only, no empty slots.  A slot_map entry >= n_slots is skipped
- * and flagged in counters->error (which moe_pw_assign zeroed).  The empty
- * tails are handed out to the kernel's warps through counters->work, which
- * this call resets on `stream` before the kernel; two packs that share a
- * counters struct must not run at the same time.
+ * tail of every pool (positions >= occ) with zeros and header -1.  A
+ * slot_map entry >= n_slots is skipped and flagged in counters->error (which
+ * moe_pw_assign zeroed).  The empty tails are handed out to the kernel's warps
+ * through counters->work, which this call resets on `stream` before the
+ * kernel; two packs that share a counters struct must not run at the same
+ * time.
+ * Ragged mode: rows only, no empty slots.  Given the workspace moe_pw_assign
+ * used (unchanged since, at least moe_pw_sizes.workspace_bytes), the rows are
+ * written in their own order, block of tokens by block, expert by expert (its
+ * per-chunk bases tell where each block's run of an expert starts); the
+ * header array serves as the row -> token map until each row is copied.
+ * Without it (NULL, or too small) the kernel sweeps the tokens.  Same bytes
+ * either way.  Pooled mode ignores the workspace (it may be NULL).
  */
 int moe_pw_pack(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
                 const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
-                int32_t *pool_hdr, moe_pw_counters *counters, cudaStream_t stream);
+                int32_t *pool_hdr, moe_pw_counters *counters, void *workspace,
+                size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Exchange + receiver bucketing (section 二: receiver factor; huxiu: first
@@ -392,6 +400,52 @@ int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint1
 int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
                  const int32_t *expert_counts, moe_pw_drop_stats *host_out,
                  int32_t *host_expert_counts, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* One step from host memory to host memory.                                 */
+/* ------------------------------------------------------------------------ */
+
+/* The device arrays of one step (caller-allocated, sizes from moe_pw_plan). */
+typedef struct moe_pw_device_buffers {
+    float *logits;           /* f32 [T, E] */
+    uint16_t *x;             /* bf16 [T, D] */
+    float *scale;            /* f32 [E] */
+    int32_t *idx;            /* i32 [T, k] */
+    float *gates;            /* f32 [T, k] */
+    int32_t *slot_map;       /* i32 [T, k] */
+    int32_t *occ;            /* i32 [occ_len] */
+    uint16_t *pool_x;        /* bf16 [n_slots, D] */
+    int32_t *pool_hdr;       /* i32 [n_slots] */
+    int32_t *recv_row;       /* i32 [n_slots] */
+    int32_t *bucket_slot;    /* i32 [bucket_len] (pooled) */
+    int32_t *expert_counts;  /* i32 [2, E] */
+    uint16_t *ret_x;         /* bf16 [n_slots, D] */
+    int32_t *ret_hdr;        /* i32 [n_slots] */
+    float *out;              /* f32 [T, D] */
+    moe_pw_counters *counters;
+    void *workspace;
+    size_t workspace_bytes;
+} moe_pw_device_buffers;
+
+/*
+ * One whole step with host buffers in and out, all of it enqueued, nothing
+ * waited for: on copy_in the host inputs (logits f32 [T, E], x bf16 [T, D],
+ * scale f32 [E]) go to dev; compute waits for them and runs route, dispatch,
+ * the per-expert op and the combine; copy_out waits for the combine and
+ * brings out (f32 [T, D] into h_out) and the counters (into *h_counters)
+ * back.  The three streams may be the same stream.  For the copies to run
+ * beside the kernels, the host buffers must be pinned (cudaHostAlloc /
+ * cudaHostRegister) and the streams distinct; then the upload of one batch,
+ * the compute of the previous one and the download of the one before can
+ * overlap when the caller alternates two sets of device buffers and orders
+ * each set's reuse (its inputs after the compute that read them, its output
+ * after the download that read it) with events on these streams.  Returns
+ * once everything is enqueued; synchronise copy_out before reading h_out.
+ */
+int moe_pw_step_host(const moe_pw_config *cfg, const float *h_logits, const uint16_t *h_x,
+                     const float *h_scale, float *h_out, moe_pw_counters *h_counters,
+                     const moe_pw_device_buffers *dev, cudaStream_t compute,
+                     cudaStream_t copy_in, cudaStream_t copy_out);
 
 /* ------------------------------------------------------------------------ */
 /* Expert parallelism over several GPUs.                                     */

@@ -378,6 +378,32 @@ def test_pipeline_matches_single_steps():
     assert last.error == 0 and last.kept > 0
 
 
+def test_step_host_equals_device_step():
+    """moe_pw_step_host (host buffers in and out, one C call): the same
+    output and counters as the step on device buffers, on one stream and on
+    three."""
+    for name in ("tiny", "tiny_ragged"):
+        w = SMALL_CASES[name]
+        lg, x, s = _inputs(w)
+        ref, st = run_gpu(w, lg, x, s)
+        cfg = mp.Config.from_workload(w)
+        b = mp.Buffers(cfg)
+        h_lg = torch.from_numpy(lg).pin_memory()
+        h_x = torch.from_numpy(x.view(np.int16)).pin_memory()
+        h_s = torch.from_numpy(s).pin_memory()
+        for streams in (1, 3):
+            h_out = torch.full((w.T, w.D), 7.0, dtype=torch.float32).pin_memory()
+            h_ctr = torch.zeros((mp.COUNTERS_BYTES // 8,), dtype=torch.int64).pin_memory()
+            extra = [torch.cuda.Stream(), torch.cuda.Stream()] if streams == 3 else [None, None]
+            mp.moe_pw_step_host(cfg, h_lg, h_x, h_s, h_out, h_ctr, b.device_buffers(),
+                                torch.cuda.current_stream(), *extra)
+            torch.cuda.synchronize()
+            assert torch.equal(h_out, ref.out.cpu())
+            c = mp.moe_pw_counters.from_buffer_copy(h_ctr.numpy().tobytes())
+            assert (c.kept, c.sender_dropped, c.receiver_dropped, c.error) == (
+                st.kept, st.sender_dropped, st.receiver_dropped, 0)
+
+
 def test_captured_step_replays_bit_identical():
     """The forward step recorded as a CUDA graph: a replay equals an eager
     step byte for byte, and after new inputs are copied into the same
