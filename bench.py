@@ -385,12 +385,15 @@ def config_of(w):
 NVLINK_PEER_GBS = 770.0  # measured peer copy per direction on this machine (900 nominal)
 
 
-def ep_link_bytes(share, D: int, n: int) -> int:
-    """Bytes one GPU sends to the other GPUs per step, per direction: its
-    pools' rows and headers (fixed shape, zero tails included) to the
-    destinations' GPUs, and the same volume of returned rows back; the pools
-    for its own experts stay in its memory (1/n of them)."""
-    return share.n_slots * (2 * D + 4) * (n - 1) // n
+def ep_link_bytes(share, D: int, n: int, kept_send: int, kept_recv: int) -> int:
+    """Bytes one GPU sends to the other GPUs per step (and, by symmetry,
+    receives): the rows it keeps for other GPUs' experts plus every slot's
+    header, and the rows and headers it returns to other GPUs' sources; a
+    slot with header -1 sends its header only.  (n - 1) / n of the traffic
+    leaves the GPU (its own experts' pools stay local).  kept_send /
+    kept_recv: this GPU's share of the rows the senders and receivers kept."""
+    rows = (kept_send + kept_recv) * 2 * D + 2 * share.n_slots * 4
+    return rows * (n - 1) // n
 
 
 def run_ep_bench(a, world: int, rank: int, local: int):
@@ -454,7 +457,7 @@ def run_ep_bench(a, world: int, rank: int, local: int):
     ms, ms_one = max_over_ranks([ms, ms_one], world, dev)
     TK, kept, sd, rd, err = [int(v) for v in counts.tolist()]
     value = TK / (ms / 1e3)
-    link = ep_link_bytes(b.share, w.D, world)
+    link = ep_link_bytes(b.share, w.D, world, (TK - sd) // world, kept // world)
 
     # end to end: this GPU's inputs from pinned host memory, its output back
     h_lg = b.logits.cpu().pin_memory()

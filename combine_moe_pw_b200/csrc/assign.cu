@@ -23,6 +23,8 @@
 // touch only shared memory (the latency of one global read per chunk instead
 // of one per 32 assignments of a warp).
 // Ragged mode adds a one-block scan of the per-expert totals into offsets.
+#include <cstring>
+
 #include "common.cuh"
 
 namespace moe_pw {
@@ -30,6 +32,7 @@ namespace moe_pw {
 namespace {
 
 constexpr int AW = 8;  // warps per block in count/rank
+constexpr int MAX_FUSED_CHUNKS = 32;
 
 struct RankArgs {
     const int32_t *idx;
@@ -39,6 +42,7 @@ struct RankArgs {
     int32_t *totals;   // [n_groups][NB]
     moe_pw_counters *ctr;
     Geo g;
+    int32_t fused_scan;  // pooled, few chunks per group: assign_rank takes the scan's part
 };
 
 __device__ __forceinline__ int32_t bin_of_expert(const Geo &g, int32_t e)
@@ -260,14 +264,32 @@ __global__ void __launch_bounds__(AW * 32) assign_rank(RankArgs p)
     const int w0 = n * warp / AW, w1 = n * (warp + 1) / AW;
     warp_hist(p, s, w0, w1, warp, lane);
     __syncthreads();
-    // turn per-warp counts into per-warp starting ranks
-    const int32_t *base = p.counts + int64_t(blockIdx.x) * p.g.NB;
+    // turn per-warp counts into per-warp starting ranks.  The chunk's base
+    // is the scan pass's output, or (few chunks per group) the sum of the
+    // earlier chunks' raw counts, taken here; then the group's last chunk
+    // also settles the pools' occupancy and drops, which the scan pass
+    // would have done.
+    const int cpg = p.g.chunks_per_group;
+    const int ci = int(blockIdx.x) - group * cpg;
     for (int b = threadIdx.x; b < p.g.NB; b += blockDim.x) {
-        int32_t run = base[b];
+        int32_t run = 0;
+        if (p.fused_scan) {
+            const int32_t *col = p.counts + int64_t(group) * cpg * p.g.NB + b;
+            for (int c = 0; c < ci; ++c) run += col[int64_t(c) * p.g.NB];
+        } else {
+            run = p.counts[int64_t(blockIdx.x) * p.g.NB + b];
+        }
         for (int w = 0; w < AW; ++w) {
             const int32_t v = s.hist[w * p.g.NB + b];
             s.hist[w * p.g.NB + b] = run;
             run += v;
+        }
+        if (p.fused_scan && ci == cpg - 1) {
+            // run = the pool's total over the whole group
+            const int64_t kept = run < p.g.C_s ? run : p.g.C_s;
+            p.occ[int64_t(group) * p.g.NB + b] = int32_t(kept);
+            if (run > kept) atomicAdd(&p.ctr->sender_dropped, (unsigned long long)(run - kept));
+            atomicMax(&p.ctr->max_occ, int32_t(kept));
         }
     }
     __syncthreads();
@@ -312,6 +334,7 @@ cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, i
     if (g.T == 0) return cudaMemsetAsync(occ, 0, sizeof(int32_t) * occ_len, st);
 
     RankArgs p;
+    memset(&p, 0, sizeof(p));
     p.idx = idx;
     p.slot_map = slot_map;
     p.occ = occ;
@@ -332,11 +355,16 @@ cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, i
                                         di.smem_optin)) != cudaSuccess)
             return err;
     }
+    // with at most MAX_FUSED_CHUNKS chunks per source the rank pass sums the
+    // earlier chunks' counts itself and the scan pass is skipped (pooled mode)
+    p.fused_scan = g.mode == MOE_PW_POOLED && g.chunks_per_group <= MAX_FUSED_CHUNKS;
     assign_count<<<g.n_chunks, AW * 32, smem, st>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    dim3 sgrid((g.NB + 31) / 32, g.n_groups);
-    assign_scan<<<sgrid, 1024, 0, st>>>(p);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (!p.fused_scan) {
+        dim3 sgrid((g.NB + 31) / 32, g.n_groups);
+        assign_scan<<<sgrid, 1024, 0, st>>>(p);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
     if (g.mode == MOE_PW_RAGGED) {
         ragged_offsets<<<1, 1024, 0, st>>>(p);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;

@@ -54,18 +54,10 @@ cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, i
                           moe_pw_counters *ctr, void *ws, cudaStream_t st);
 // ep (optional): the receive pools of every GPU of an expert-parallel run;
 // rows then go to the destination's GPU, only for waves in wave_mask.
-// ws (optional, ragged mode): the assignment pass's workspace, unchanged since;
-// with it the dropless pack writes rows in their own order (pack_ragged.cu).
 cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
                         const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
                         int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st,
-                        const EpRows *ep = nullptr, uint32_t wave_mask = ~0u,
-                        void *ws = nullptr);
-// the dropless pack in row order; cudaErrorNotSupported when rows are too
-// wide for its ring (the caller then sweeps the tokens instead)
-cudaError_t launch_pack_ragged(const Geo &g, const uint16_t *x, const int32_t *slot_map,
-                               const int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr,
-                               moe_pw_counters *ctr, void *ws, cudaStream_t st);
+                        const EpRows *ep = nullptr, uint32_t wave_mask = ~0u);
 // occ == nullptr: an empty slot is one whose header is -1 (expert-parallel
 // receive pools, where no counts are exchanged).
 cudaError_t launch_bucket(const Geo &g, const int32_t *pool_hdr, const int32_t *occ,
@@ -96,28 +88,11 @@ cudaError_t launch_gemm(const uint16_t *A, const uint16_t *Bt, int64_t M, int32_
                         int64_t n_slots, moe_pw_counters *ctr, cudaStream_t st,
                         const uint16_t *add = nullptr);
 
-// Workspace layout: the ranking pass's per-chunk counts (then bases) and
-// per-group totals; in ragged mode also the dropless pack's per-block run
-// prefix (blocks of about RAGGED_BLOCK_BYTES of x, whole chunks each).
-constexpr int64_t RAGGED_BLOCK_BYTES = int64_t(24) << 20;
+// Workspace layout of the ranking pass.
 inline int64_t align256(int64_t b) { return (b + 255) & ~int64_t(255); }
 inline int64_t ws_counts_bytes(const Geo &g) { return align256(4 * int64_t(g.n_chunks) * g.NB); }
 inline int64_t ws_totals_bytes(const Geo &g) { return align256(4 * int64_t(g.n_groups) * g.NB); }
-inline int64_t ragged_chunks_per_block(const Geo &g)
-{
-    const int64_t c = RAGGED_BLOCK_BYTES / (2 * int64_t(g.D) * (g.chunk_tokens > 0 ? g.chunk_tokens : 1));
-    return c > 0 ? c : 1;
-}
-inline int64_t ws_ragged_bytes(const Geo &g)
-{
-    if (g.mode != MOE_PW_RAGGED) return 0;
-    const int64_t cpb = ragged_chunks_per_block(g);
-    return align256(4 * ((g.n_chunks + cpb - 1) / cpb) * (int64_t(g.E) + 1));
-}
-inline int64_t ws_bytes(const Geo &g)
-{
-    return ws_counts_bytes(g) + ws_totals_bytes(g) + ws_ragged_bytes(g);
-}
+inline int64_t ws_bytes(const Geo &g) { return ws_counts_bytes(g) + ws_totals_bytes(g); }
 
 // ---------------------------------------------------------------------------
 // Device helpers: mbarrier and bulk (TMA) copies, inline PTX for sm_100a.

@@ -93,7 +93,8 @@ __global__ void __launch_bounds__(256) expert_kernel(ExpertArgs a)
                 y.w = scale_pair(v.w, s);
                 __stcs(dst + c, y);
             }
-        } else {
+        } else if (!EP) {
+            // (across GPUs the header -1 alone goes back: nothing reads the row)
             for (int c = lane; c < cpr; c += 32) __stcs(dst + c, make_uint4(0, 0, 0, 0));
         }
         if (lane == 0) *dst_hdr = keep ? e : -1;

@@ -222,8 +222,7 @@ int moe_pw_assign(const moe_pw_config *cfg, const int32_t *idx, int32_t *slot_ma
 
 int moe_pw_pack(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
                 const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr,
-                moe_pw_counters *counters, void *workspace, size_t workspace_bytes,
-                cudaStream_t stream)
+                moe_pw_counters *counters, cudaStream_t stream)
 {
     Geo g;
     int rc = make_geo(cfg, &g);
@@ -233,15 +232,7 @@ int moe_pw_pack(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
     if (!aligned(x, 16) || !aligned(pool_x, 16) || !aligned(idx, 4) || !aligned(slot_map, 4) ||
         !aligned(occ, 4) || !aligned(pool_hdr, 4) || !aligned(counters, 8))
         return MOE_PW_EUNSUPPORTED;
-    // the workspace only serves the dropless mode; too small or absent, the
-    // pack sweeps the tokens instead
-    void *ws = nullptr;
-    if (g.mode == MOE_PW_RAGGED && workspace && int64_t(workspace_bytes) >= ws_bytes(g)) {
-        if (!aligned(workspace, 256)) return MOE_PW_EUNSUPPORTED;
-        ws = workspace;
-    }
-    return cuda_rc(launch_pack(g, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream,
-                               nullptr, ~0u, ws));
+    return cuda_rc(launch_pack(g, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream));
 }
 
 int moe_pw_bucket(const moe_pw_config *cfg, const int32_t *pool_hdr, const int32_t *occ,
@@ -269,8 +260,7 @@ int moe_pw_dispatch(const moe_pw_config *cfg, const uint16_t *x, const int32_t *
 {
     int rc = moe_pw_assign(cfg, idx, slot_map, occ, counters, workspace, workspace_bytes, stream);
     if (rc != MOE_PW_OK) return rc;
-    rc = moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, workspace,
-                     workspace_bytes, stream);
+    rc = moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream);
     if (rc != MOE_PW_OK) return rc;
     return moe_pw_bucket(cfg, pool_hdr, occ, recv_row, bucket_slot, expert_counts, counters,
                          stream);

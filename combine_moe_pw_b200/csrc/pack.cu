@@ -28,7 +28,6 @@
 // The defaults below came from a sweep on the 262,144-token batch: deeper
 // rings with fewer warps beat more warps with shallow rings; the lag between
 // 8 and 20 made no measurable difference.
-#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -206,16 +205,13 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
         if (filled < 0) filled = 0;
         if (filled > p.C_s) filled = p.C_s;
         if (EP) {
-            // the tail is contiguous in the destination's receive pool too
+            // across GPUs only the headers of the empty tail travel: -1 marks
+            // the slot empty and nothing reads an empty slot's row, so the
+            // zero rows would be link bytes without information
             int h, w;
             const uint32_t rq0 = ep_send_to_recv(p.geo, uint32_t(q * p.C_s), h, w);
             if (!((p.wave_mask >> w) & 1u)) continue;
-            for (int64_t c = filled + lane; c < p.C_s; c += 32) {
-                bulk_s2g(p.ep.x[h] + (int64_t(rq0) + c) * D, zero, rb, pol_pool);
-                p.ep.hdr[h][rq0 + c] = -1;
-            }
-            bulk_commit();
-            bulk_wait_read<8>();
+            for (int64_t c = filled + lane; c < p.C_s; c += 32) p.ep.hdr[h][rq0 + c] = -1;
             continue;
         }
 #if MOE_PW_PACK_ZERO_TMA
@@ -276,30 +272,14 @@ cudaError_t launch_ep(const PackArgs &p, const DevInfo &di, const Geo &g, int nw
     return launch_lag<2, EP>(p, di, g, nw, smem, st);
 }
 
-// MOE_PW_RAGGED_PACK=sweep in the environment (read once) keeps the dropless
-// mode on the token sweep of this file; by default it writes rows in their
-// own order (pack_ragged.cu).  Both give the same bytes.
-bool ragged_pack_enabled()
-{
-    static const bool on = [] {
-        const char *v = getenv("MOE_PW_RAGGED_PACK");
-        return !(v && strcmp(v, "sweep") == 0);
-    }();
-    return on;
-}
-
 }  // namespace
 
 cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
                         const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
                         int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st,
-                        const EpRows *ep, uint32_t wave_mask, void *ws)
+                        const EpRows *ep, uint32_t wave_mask)
 {
     if (g.T == 0 && g.n_pools == 0) return cudaSuccess;
-    if (g.mode == MOE_PW_RAGGED && ws && !ep && ragged_pack_enabled()) {
-        const cudaError_t e = launch_pack_ragged(g, x, slot_map, occ, pool_x, pool_hdr, ctr, ws, st);
-        if (e != cudaErrorNotSupported) return e;
-    }
     DevInfo di;
     if (dev_info(&di) != 0) return cudaErrorUnknown;
     PackArgs p;

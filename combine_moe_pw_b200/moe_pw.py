@@ -100,7 +100,7 @@ SIGNATURES = {
     "moe_pw_route": [_CFG, _VP, _VP, _VP, _VP],
     "moe_pw_assign": [_CFG, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_assign_noalloc": [_CFG, _VP, _VP, _VP, _VP, _VP],
-    "moe_pw_pack": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "moe_pw_pack": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_bucket": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_dispatch": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_expert": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
@@ -241,13 +241,11 @@ def moe_pw_assign_noalloc(cfg, idx, slot_map, occ, counters, stream=None):
         ctypes.byref(c), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(counters), _stream(stream)))
 
 
-def moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream=None,
-                workspace=None):
+def moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream=None):
     c = _cfg(cfg)
-    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("moe_pw_pack", load_library().moe_pw_pack(
         ctypes.byref(c), _ptr(x), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(pool_x),
-        _ptr(pool_hdr), _ptr(counters), _ptr(workspace), wsb, _stream(stream)))
+        _ptr(pool_hdr), _ptr(counters), _stream(stream)))
 
 
 def moe_pw_bucket(cfg, pool_hdr, occ, recv_row, bucket_slot, expert_counts, counters, stream=None):
@@ -520,7 +518,7 @@ class Buffers:
 
     def pack(self, stream=None):
         moe_pw_pack(self.cfg, self.x, self.idx, self.slot_map, self.occ, self.pool_x,
-                    self.pool_hdr, self.counters, stream, self.workspace)
+                    self.pool_hdr, self.counters, stream)
 
     def bucket(self, stream=None):
         moe_pw_bucket(self.cfg, self.pool_hdr, self.occ, self.recv_row, self.bucket_slot,

@@ -205,24 +205,16 @@ int moe_pw_assign(const moe_pw_config *cfg, const int32_t *idx, int32_t *slot_ma
  * Pack (section 二: expert id in the payload).  Copies each kept row x[t] into
  * its slot with TMA bulk copies through shared memory (one read of x[t], up to
  * k writes), writes the expert id into the slot header, and fills the empty
- * tail of every pool (positions >= occ) with zeros and header -1.  A
- * slot_map entry >= n_slots is skipped and flagged in counters->error (which
- * moe_pw_assign zeroed).  The empty tails are handed out to the kernel's warps
- * through counters->work, which this call resets on `stream` before the
- * kernel; two packs that share a counters struct must not run at the same
- * time.
- * Ragged mode: rows only, no empty slots.  Given the workspace moe_pw_assign
- * used (unchanged since, at least moe_pw_sizes.workspace_bytes), the rows are
- * written in their own order, block of tokens by block, expert by expert (its
- * per-chunk bases tell where each block's run of an expert starts); the
- * header array serves as the row -> token map until each row is copied.
- * Without it (NULL, or too small) the kernel sweeps the tokens.  Same bytes
- * either way.  Pooled mode ignores the workspace (it may be NULL).
+ * tail of every pool (positions >= occ) with zeros and header -1.  Ragged
+ * mode: rows only, no empty slots.  A slot_map entry >= n_slots is skipped
+ * and flagged in counters->error (which moe_pw_assign zeroed).  The empty
+ * tails are handed out to the kernel's warps through counters->work, which
+ * this call resets on `stream` before the kernel; two packs that share a
+ * counters struct must not run at the same time.
  */
 int moe_pw_pack(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
                 const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
-                int32_t *pool_hdr, moe_pw_counters *counters, void *workspace,
-                size_t workspace_bytes, cudaStream_t stream);
+                int32_t *pool_hdr, moe_pw_counters *counters, cudaStream_t stream);
 
 /*
  * Exchange + receiver bucketing (section 二: receiver factor; huxiu: first
@@ -492,6 +484,11 @@ int moe_pw_step_host(const moe_pw_config *cfg, const float *h_logits, const uint
  * Waves: wave_mask (bit w = wave w; (1 << W) - 1 = all) selects the waves a
  * pack, bucket or expert call handles, so wave w can be exchanged while the
  * expert op of wave w - 1 runs.  Pooled mode only.
+ *
+ * Only what is read crosses GPUs: an empty send slot and a slot the receiver
+ * did not keep travel as their header -1 alone; their rows in the receive
+ * and return pools are left as they were (the single-GPU calls write zeros
+ * there).  Every consumer skips such rows by the header.
  */
 #define MOE_PW_EP_MAX_GPUS 64
 
@@ -543,8 +540,8 @@ int moe_pw_ep_assign(const moe_pw_config *cfg, const moe_pw_ep *ep, const int32_
  * (loaded once into shared memory) is bulk-stored into the receive pool of
  * the destination's GPU (peers->recv_x[d / Rn]) at its receive slot, with the
  * expert id as its header; the empty tails (c >= occ) of this GPU's pools of
- * those waves get zero rows and header -1 there.  Uses counters->work like
- * moe_pw_pack.  x bf16 [tokens, D].
+ * those waves get header -1 there (their rows are not sent).  Uses
+ * counters->work like moe_pw_pack.  x bf16 [tokens, D].
  */
 int moe_pw_ep_pack(const moe_pw_config *cfg, const moe_pw_ep *ep, const moe_pw_ep_peers *peers,
                    const uint16_t *x, const int32_t *idx, const int32_t *slot_map,
@@ -566,9 +563,9 @@ int moe_pw_ep_bucket(const moe_pw_config *cfg, const moe_pw_ep *ep, const int32_
 /*
  * Per-expert op and return trip (huxiu: results come back by a second
  * all-to-all).  For every receive slot of the waves in wave_mask: if the
- * receiver kept it, bf16_rn(scale[e] * row) and header e, else zeros and -1,
- * stored into the return pool of the source's GPU (peers->ret_x[s / Rn]) at
- * the source's send slot.
+ * receiver kept it, bf16_rn(scale[e] * row) and header e, else header -1
+ * alone, stored into the return pool of the source's GPU (peers->ret_x[s /
+ * Rn]) at the source's send slot.
  */
 int moe_pw_ep_expert(const moe_pw_config *cfg, const moe_pw_ep *ep, const moe_pw_ep_peers *peers,
                      const uint16_t *recv_x, const int32_t *recv_hdr, const int32_t *recv_row,

@@ -1,7 +1,10 @@
 """Reassembling the per-GPU shares of an expert-parallel run into the
 single-batch layout, so the oracle's arrays can be compared with them
 directly.  Only index relabelling lives here (the layouts of include/moe_pw.h,
-"Expert parallelism over several GPUs"); no arithmetic of the method.
+"Expert parallelism over several GPUs"); no arithmetic of the method.  Across
+GPUs the rows of slots whose header is -1 are not sent, so their payload is
+not defined there: those rows are set to the single-GPU reading (zeros)
+before the comparison, and the headers, compared in full, must mark them.
 """
 from types import SimpleNamespace
 
@@ -54,6 +57,9 @@ def assemble(cfg, shares, stats):
         bucket[h * Rn * L:(h + 1) * Rn * L] = np.where(bs >= 0, m[np.maximum(bs, 0)], -1)
         counts[:, h * Rn * L:(h + 1) * Rn * L] = _n(s.expert_counts)
         host_counts[:, h * Rn * L:(h + 1) * Rn * L] = s.host_expert_counts
+    # across GPUs the rows of empty and of receiver-dropped slots are not
+    # sent (their headers say so); the single-GPU reading has zeros there
+    pool_x[pool_hdr < 0] = 0
     b.pool_x = pool_x.reshape(S, D)
     b.pool_hdr = pool_hdr.reshape(S)
     b.recv_row = recv_row.reshape(S)
@@ -62,6 +68,7 @@ def assemble(cfg, shares, stats):
     b.host_expert_counts = host_counts
     b.ret_x = cat("ret_x")
     b.ret_hdr = cat("ret_hdr")
+    b.ret_x[b.ret_hdr < 0] = 0
     b.out = cat("out")
     for k, v in list(vars(b).items()):
         if isinstance(v, np.ndarray) and k != "host_expert_counts":

@@ -180,6 +180,10 @@ SMALL_CASES = {
     "ragged_tail_ragged": TINY.with_(T=8 * 37, seq_len=37, mode=synth.MODE_RAGGED,
                                      cf_send_pct=0, cf_recv_pct=0),
     "many_chunks": TINY.with_(T=8 * 1000 + 0, seq_len=1000, D=64),
+    # 40 chunks per source: the assignment's separate scan pass (at most 32
+    # chunks per source are summed inside the rank pass instead)
+    "long_sources": synth.Workload("long_sources", T=2 * 10000, R=2, L=6, W=3, P=2, k=8, D=16,
+                                   seq_len=10000, logit_kind=synth.LOGIT_SEQBIAS),
     "wide_E": synth.Workload("wide_E", T=64 * 24, R=64, L=16, W=4, P=4, k=8, D=64, seq_len=24,
                              logit_kind=synth.LOGIT_SEQBIAS),
     "E2048": synth.Workload("E2048", T=256 * 8, R=256, L=8, W=4, P=2, k=8, D=32, seq_len=64,
