@@ -112,6 +112,7 @@ def _configure(lib):
     lib.orc_dispatch_backward.argtypes = [gp, vp, vp, vp, vp]
     lib.orc_backward_tokens.argtypes = [gp, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp]
     lib.orc_project.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp]
+    lib.orc_seq_balance.argtypes = [gp, i64, ctypes.c_double, vp, vp, vp, vp, vp, vp]
     lib.orc_bf16_round.argtypes = [vp, vp, i64]
     lib.orc_expert_product.argtypes = [vp, vp, vp, i64]
     return lib
@@ -401,6 +402,22 @@ def project(A: np.ndarray, Bt: np.ndarray, exact: bool = False, add: np.ndarray 
     _load().orc_project(_p(A), _p(Bt), M, N, K, _p(add) if add is not None else None, _p(C),
                         _p(Ce) if exact else None, _p(mag) if exact else None)
     return (C, Ce, mag) if exact else C
+
+
+def seq_balance(g: Geom, seq_len: int, alpha: float, logits, idx, with_grad: bool = True):
+    """Sequence-level balance term (see orc_seq_balance): f, P [n_seq, E],
+    loss [n_seq] and, with_grad, dlogits [T, E]."""
+    lg = _c(logits, np.float32).reshape(g.T, g.E)
+    ix = _c(idx, np.int32).reshape(g.T, g.k)
+    n_seq = g.T // seq_len
+    f = np.empty((n_seq, g.E), np.float64)
+    P = np.empty((n_seq, g.E), np.float64)
+    loss = np.empty((n_seq,), np.float64)
+    dl = np.empty((g.T, g.E), np.float64) if with_grad else None
+    gc = g.c()
+    _load().orc_seq_balance(ctypes.byref(gc), seq_len, alpha, _p(lg), _p(ix), _p(f), _p(P),
+                            _p(loss), _p(dl) if with_grad else None)
+    return (f, P, loss, dl) if with_grad else (f, P, loss)
 
 
 def bf16_round(a: np.ndarray) -> np.ndarray:

@@ -677,3 +677,69 @@ void orc_project(const uint16_t *A, const uint16_t *Bt, int64_t M, int64_t N, in
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Sequence-level balancing.                                                 */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * "Marin 开始公开训练 535B 参数 MoE 模型", section 四: if drops stay too high,
+ * one remedy is sequence-level balancing, which "may force the experts to
+ * re-specialise during training".  The pages give no formula.  READING: a
+ * balance term of the training loss computed per sequence, the product of
+ * how often each expert is chosen and how much router probability it gets,
+ * within one sequence:
+ *   p[t][e]  = softmax over all E logits of token t
+ *   f[s][e]  = E / (k * L) * #{ t in s, j : idx[t][j] == e }
+ *   P[s][e]  = 1 / L * sum over t in s of p[t][e]
+ *   loss[s]  = alpha * sum_e f[s][e] * P[s][e]
+ * with L = seq_len tokens per sequence (T % L == 0).  Perfect balance
+ * (f = 1 for every expert) gives loss = alpha whatever the probabilities.
+ * The gradient treats f as constant (the top-k choice is piecewise constant
+ * in the logits):
+ *   dlogits[t][e] = alpha / L * p[t][e] * (f[s][e] - sum_i f[s][i] * p[t][i]).
+ * All in double.  f, P: [T / L, E]; loss: [T / L]; dlogits [T, E] may be NULL.
+ */
+void orc_seq_balance(const orc_geom *g, int64_t seq_len, double alpha, const float *logits,
+                     const int32_t *idx, double *f, double *P, double *loss, double *dlogits)
+{
+    const int32_t E = g->E, k = g->k;
+    const int64_t n_seq = g->T / seq_len;
+    double *p = (double *)malloc(sizeof(double) * (size_t)E);
+    for (int64_t s = 0; s < n_seq; ++s) {
+        double *fs = f + s * E, *Ps = P + s * E;
+        for (int32_t e = 0; e < E; ++e) fs[e] = Ps[e] = 0.0;
+        for (int64_t t = s * seq_len; t < (s + 1) * seq_len; ++t) {
+            for (int32_t j = 0; j < k; ++j) fs[idx[t * k + j]] += 1.0;
+            const float *l = logits + t * E;
+            double mx = l[0];
+            for (int32_t e = 1; e < E; ++e) if (l[e] > mx) mx = l[e];
+            double den = 0.0;
+            for (int32_t e = 0; e < E; ++e) den += exp((double)l[e] - mx);
+            for (int32_t e = 0; e < E; ++e) Ps[e] += exp((double)l[e] - mx) / den;
+        }
+        double acc = 0.0;
+        for (int32_t e = 0; e < E; ++e) {
+            fs[e] *= (double)E / ((double)k * (double)seq_len);
+            Ps[e] /= (double)seq_len;
+            acc += fs[e] * Ps[e];
+        }
+        loss[s] = alpha * acc;
+        if (!dlogits) continue;
+        for (int64_t t = s * seq_len; t < (s + 1) * seq_len; ++t) {
+            const float *l = logits + t * E;
+            double mx = l[0];
+            for (int32_t e = 1; e < E; ++e) if (l[e] > mx) mx = l[e];
+            double den = 0.0;
+            for (int32_t e = 0; e < E; ++e) den += exp((double)l[e] - mx);
+            double dot = 0.0;
+            for (int32_t e = 0; e < E; ++e) {
+                p[e] = exp((double)l[e] - mx) / den;
+                dot += fs[e] * p[e];
+            }
+            for (int32_t e = 0; e < E; ++e)
+                dlogits[t * E + e] = alpha / (double)seq_len * p[e] * (fs[e] - dot);
+        }
+    }
+    free(p);
+}

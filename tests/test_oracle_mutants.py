@@ -18,6 +18,7 @@ import test_oracle_combine as tc
 import test_oracle_dispatch as td
 import test_oracle_headers as th
 import test_oracle_route as tr
+import test_oracle_seq_balance as tsb
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "oracle.c")
 
@@ -92,6 +93,13 @@ MUTANTS = [
     ("ragged_receiver_counts_from_one", "recv_row[q] = arrivals[e]++;",
      "recv_row[q] = ++arrivals[e];",
      lambda: th.test_ragged_receiver_rows_brute_force()),
+    ("balance_share_not_scaled", "fs[e] *= (double)E / ((double)k * (double)seq_len);",
+     "fs[e] /= (double)seq_len;",
+     lambda: tsb.test_perfect_balance_gives_alpha_for_any_logits()),
+    ("balance_prob_not_averaged", "Ps[e] /= (double)seq_len;", "Ps[e] /= 1.0;",
+     lambda: tsb.test_f_and_P_against_library_routines()),
+    ("balance_gradient_sign", "p[e] * (fs[e] - dot);", "p[e] * (dot - fs[e]);",
+     lambda: tsb.test_gradient_matches_autograd_and_rows_sum_to_zero()),
     ("ragged_rows_by_token_desc", "const int32_t row = next[e]++;",
      "const int32_t row = row_off[e] + row_cnt[e] - 1 - (next[e]++ - row_off[e]);",
      lambda: td.test_ragged_assignment()),
