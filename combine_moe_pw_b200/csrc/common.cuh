@@ -82,6 +82,11 @@ cudaError_t launch_combine_backward(const Geo &g, const float *dout, const uint1
                                     float *dgates, float *dlogits, moe_pw_counters *ctr,
                                     cudaStream_t st);
 
+int64_t balance_ws_bytes(int64_t T, int64_t L, int32_t E);
+cudaError_t launch_balance(const Geo &g, int64_t seq_len, float alpha, const float *logits,
+                           const int32_t *idx, float *f, float *P, float *loss, float *dlogits,
+                           int32_t accumulate, void *ws, cudaStream_t st);
+
 cudaError_t launch_gemm(const uint16_t *A, const uint16_t *Bt, int64_t M, int32_t N, int32_t K,
                         int32_t mode, uint16_t *C, int64_t ldc, const int32_t *slot_map,
                         const int32_t *idx, int32_t topk, uint16_t *pool_x, int32_t *pool_hdr,

@@ -427,6 +427,36 @@ int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint1
     return cuda_rc(e);
 }
 
+int moe_pw_seq_balance_plan(const moe_pw_config *cfg, int64_t seq_len, int64_t *workspace_bytes)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!workspace_bytes || seq_len < 1 || g.T % seq_len != 0) return MOE_PW_EINVAL;
+    *workspace_bytes = balance_ws_bytes(g.T, seq_len, g.E);
+    return MOE_PW_OK;
+}
+
+int moe_pw_seq_balance(const moe_pw_config *cfg, int64_t seq_len, float alpha,
+                       const float *logits, const int32_t *idx, float *f, float *P, float *loss,
+                       float *dlogits, int32_t accumulate, void *workspace,
+                       size_t workspace_bytes, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (seq_len < 1 || g.T % seq_len != 0) return MOE_PW_EINVAL;
+    if (g.E % 4 != 0) return MOE_PW_EUNSUPPORTED;
+    if (g.T == 0) return MOE_PW_OK;
+    if (!logits || !idx || !f || !P || !loss || !workspace) return MOE_PW_EINVAL;
+    if (int64_t(workspace_bytes) < balance_ws_bytes(g.T, seq_len, g.E)) return MOE_PW_EINVAL;
+    if (!aligned(logits, 16) || !aligned(idx, 4) || !aligned(f, 4) || !aligned(P, 4) ||
+        !aligned(loss, 4) || !aligned(workspace, 256) || (dlogits && !aligned(dlogits, 16)))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_balance(g, seq_len, alpha, logits, idx, f, P, loss, dlogits, accumulate,
+                                  workspace, stream));
+}
+
 int moe_pw_stats(const moe_pw_config *cfg, const moe_pw_counters *counters,
                  const int32_t *expert_counts, moe_pw_drop_stats *host_out,
                  int32_t *host_expert_counts, cudaStream_t stream)

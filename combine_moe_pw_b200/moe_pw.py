@@ -114,6 +114,9 @@ SIGNATURES = {
     "moe_pw_project_pack": [_CFG, _VP, _VP, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_stats": [_CFG, _VP, _VP, ctypes.POINTER(moe_pw_drop_stats), _VP, _VP],
     "moe_pw_selftest_wait_timeout": [_VP, ctypes.c_int32, _VP],
+    "moe_pw_seq_balance_plan": [_CFG, _I64, ctypes.POINTER(ctypes.c_int64)],
+    "moe_pw_seq_balance": [_CFG, _I64, ctypes.c_float, _VP, _VP, _VP, _VP, _VP, _VP,
+                           ctypes.c_int32, _VP, _SZ, _VP],
     "moe_pw_step_host": [_CFG, _VP, _VP, _VP, _VP, _VP, ctypes.POINTER(moe_pw_device_buffers),
                          _VP, _VP, _VP],
     "moe_pw_ep_plan": [_CFG, ctypes.POINTER(moe_pw_ep), _I64, ctypes.POINTER(moe_pw_ep_sizes)],
@@ -354,6 +357,25 @@ def moe_pw_selftest_wait_timeout(counters, polls: int = 4096, stream=None):
     """Run the bounded-wait self-test (see include/moe_pw.h)."""
     _check("moe_pw_selftest_wait_timeout", load_library().moe_pw_selftest_wait_timeout(
         _ptr(counters), polls, _stream(stream)))
+
+
+def moe_pw_seq_balance_plan(cfg, seq_len: int) -> int:
+    c = _cfg(cfg)
+    n = ctypes.c_int64()
+    _check("moe_pw_seq_balance_plan", load_library().moe_pw_seq_balance_plan(
+        ctypes.byref(c), seq_len, ctypes.byref(n)))
+    return int(n.value)
+
+
+def moe_pw_seq_balance(cfg, seq_len: int, alpha: float, logits, idx, f, P, loss, workspace,
+                       dlogits=None, accumulate: bool = False, stream=None):
+    """Sequence-level balance term and (with dlogits) its gradient; see
+    include/moe_pw.h."""
+    c = _cfg(cfg)
+    _check("moe_pw_seq_balance", load_library().moe_pw_seq_balance(
+        ctypes.byref(c), seq_len, alpha, _ptr(logits), _ptr(idx), _ptr(f), _ptr(P), _ptr(loss),
+        _ptr(dlogits), 1 if accumulate else 0, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def moe_pw_step_host(cfg, h_logits, h_x, h_scale, h_out, h_counters,

@@ -381,6 +381,31 @@ int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint1
                         moe_pw_counters *counters, cudaStream_t stream);
 
 /*
+ * Sequence-level balancing ("Marin 开始公开训练 535B 参数 MoE 模型", section 四:
+ * the third remedy named for high drop rates, one that may make the experts
+ * re-specialise during training; the pages give no formula).  This library's
+ * reading is a per-sequence balance term of the training loss.  For each
+ * sequence s of seq_len = L consecutive tokens (T % L == 0):
+ *   p[t][e] = softmax over all E logits of token t
+ *   f[s][e] = E / (k L) * (assignments of s to e in idx)   (1 at balance)
+ *   P[s][e] = (1 / L) * sum over t in s of p[t][e]
+ *   loss[s] = alpha * sum_e f[s][e] * P[s][e]               (alpha at balance)
+ * and, when dlogits is not NULL, its gradient with the routing held fixed,
+ *   dlogits[t][e] = alpha / L * p[t][e] * (f[s][e] - sum_i f[s][i] p[t][i]),
+ * written (accumulate = 0) or added to dlogits (accumulate != 0, e.g. onto
+ * the top-k softmax gradient of moe_pw_combine_backward).  logits f32 [T, E]
+ * (16-byte aligned), idx i32 [T, k]; f, P f32 [T / L, E]; loss f32 [T / L];
+ * dlogits f32 [T, E] (16-byte aligned).  Sums in fp32 in a fixed order
+ * (deterministic).  workspace: at least the bytes moe_pw_seq_balance_plan
+ * gives, 256-byte aligned.  E % 4 == 0.
+ */
+int moe_pw_seq_balance_plan(const moe_pw_config *cfg, int64_t seq_len, int64_t *workspace_bytes);
+int moe_pw_seq_balance(const moe_pw_config *cfg, int64_t seq_len, float alpha,
+                       const float *logits, const int32_t *idx, float *f, float *P, float *loss,
+                       float *dlogits, int32_t accumulate, void *workspace,
+                       size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Drop statistics (section 二: the two kinds of drop are reported apart).
  * Copies *counters (device) to *host_out (host memory) and, when both
  * expert_counts (device, i32 [2, E] as written by moe_pw_bucket) and
