@@ -22,6 +22,10 @@ def test_drop_study_trends_and_oracle_point():
             r = by[(L, cf)]
             assert r["kept"] + r["sender_dropped"] + r["receiver_dropped"] == r["assignments"]
     assert by[(16384, 1.1)]["drop_total"] > by[(1024, 1.1)]["drop_total"]
+    # the balance term is above 1 (skewed sequences) and the same for every factor
+    for L in (1024, 16384):
+        vals = {by[(L, cf)]["sequence_balance"] for cf in (1.0, 1.1, 1.5, 0.0)}
+        assert len(vals) == 1 and vals.pop() > 1.0
     # one grid point against the oracle, bit for bit
     w = synth.WORKLOADS["rack"].with_(T=T, D=8, seq_len=16384, cf_send_pct=110, cf_recv_pct=115)
     r = oracle.run_headers(w, synth.logits(w))
