@@ -716,6 +716,41 @@ def main():
         del b.d_ret, b.d_pool, b.dout, b.dlogits, b.dx
         torch.cuda.empty_cache()
 
+    # sequence-level balance term and its gradient (reported apart): logits
+    # read twice (statistics, gradient), dlogits written once
+    bal = None
+    if not a.no_backward and w.T % w.seq_len == 0:
+        n_seq = w.T // w.seq_len
+        bf = torch.empty((n_seq, w.E), dtype=torch.float32, device=dev)
+        bP = torch.empty_like(bf)
+        bl = torch.empty((n_seq,), dtype=torch.float32, device=dev)
+        bd = torch.empty((w.T, w.E), dtype=torch.float32, device=dev)
+        bws = torch.empty((max(mp.moe_pw_seq_balance_plan(cfg, w.seq_len), 256),),
+                          dtype=torch.uint8, device=dev)
+
+        def bal_step():
+            mp.moe_pw_seq_balance(cfg, w.seq_len, 0.01, b.logits, b.idx, bf, bP, bl, bws,
+                                  dlogits=bd, stream=stream)
+        for _ in range(3):
+            bal_step()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(a.steps):
+            bal_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        (bms,) = max_over_ranks([e0.elapsed_time(e1) / a.steps], world, dev)
+        bbytes = 2 * 4 * w.T * w.E + 4 * w.T * w.k + 4 * w.T * w.E
+        bal = {"ms_per_step": bms, "alg_bytes_per_step": bbytes,
+               "hbm_gbs": bbytes / (bms / 1e3) / 1e9,
+               "hbm_frac_of_peak": bbytes / (bms / 1e3) / 1e9 / measured_peaks()[0],
+               "mean_term_alpha_1": float(bl.double().mean().item()) / 0.01,
+               "scope": "balance term per sequence and its gradient (logits read twice, "
+                        "dlogits written)"}
+        del bf, bP, bl, bd, bws
+        torch.cuda.empty_cache()
+
     proj = None
     if not a.no_projection:
         proj = time_projection(w, dev, stream, min(a.steps, 10), b)
@@ -817,6 +852,7 @@ def main():
             "gpu_launches": launches_per_step * a.steps,
             "graph": graph,
             "backward": bwd,
+            "seq_balance": bal,
             "projection": proj,
             "clocks": clocks,
             "e2e": e2e,
