@@ -61,6 +61,8 @@ def parse():
                     help="time only the tensor-core projections (profiling)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the batch's token count (profiling a smaller case)")
+    ap.add_argument("--balance-only", action="store_true",
+                    help="time only the sequence balance term and its gradient (profiling)")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism over the GPUs even at one GPU (the default for "
                          "more than one): the R ranks split over the GPUs, the pools "
@@ -154,6 +156,43 @@ def time_projection(w, dev, stream, steps: int, b=None):
     del h, wd, wu, xl, y
     torch.cuda.empty_cache()
     return out
+
+
+def time_balance(w, cfg, b, dev, stream, steps: int, world: int):
+    """The sequence-level balance term and its gradient on the routed batch
+    in b: logits read twice (statistics, gradient), dlogits written once."""
+    import torch
+    from combine_moe_pw_b200 import moe_pw as mp
+    if w.T % w.seq_len != 0:
+        return None
+    n_seq = w.T // w.seq_len
+    bf = torch.empty((n_seq, w.E), dtype=torch.float32, device=dev)
+    bP = torch.empty_like(bf)
+    bl = torch.empty((n_seq,), dtype=torch.float32, device=dev)
+    bd = torch.empty((w.T, w.E), dtype=torch.float32, device=dev)
+    bws = torch.empty((max(mp.moe_pw_seq_balance_plan(cfg, w.seq_len), 256),),
+                      dtype=torch.uint8, device=dev)
+
+    def bal_step():
+        mp.moe_pw_seq_balance(cfg, w.seq_len, 0.01, b.logits, b.idx, bf, bP, bl, bws,
+                              dlogits=bd, stream=stream)
+    for _ in range(3):
+        bal_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        bal_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    (bms,) = max_over_ranks([e0.elapsed_time(e1) / steps], world, dev)
+    bbytes = 2 * 4 * w.T * w.E + 4 * w.T * w.k + 4 * w.T * w.E
+    return {"ms_per_step": bms, "alg_bytes_per_step": bbytes,
+            "hbm_gbs": bbytes / (bms / 1e3) / 1e9,
+            "hbm_frac_of_peak": bbytes / (bms / 1e3) / 1e9 / measured_peaks()[0],
+            "mean_term_alpha_1": float(bl.double().mean().item()) / 0.01,
+            "scope": "balance term per sequence and its gradient (logits read twice, "
+                     "dlogits written)"}
 
 
 def rank_workload(base, rank: int):
@@ -563,6 +602,19 @@ def main():
         base = base.with_(T=a.tokens, seq_len=min(base.seq_len, a.tokens // base.R * base.R))
     w = rank_workload(base, rank)
     cfg = mp.Config.from_workload(w)
+    if a.balance_only:
+        # only what the balance term reads: logits and the routing
+        from types import SimpleNamespace
+        nb = SimpleNamespace(
+            logits=torch.from_numpy(synth.logits(w)).to(dev),
+            idx=torch.empty((w.T, w.k), dtype=torch.int32, device=dev),
+            gates=torch.empty((w.T, w.k), dtype=torch.float32, device=dev))
+        stream = torch.cuda.current_stream(dev)
+        mp.moe_pw_route(cfg, nb.logits, nb.idx, nb.gates, stream)
+        out = time_balance(w, cfg, nb, dev, stream, a.steps, world)
+        if rank == 0:
+            print(json.dumps({"seq_balance": out, "config": config_of(w)}), flush=True)
+        return
     b = mp.Buffers(cfg, device=dev)
     sizes = b.sizes
     lg = synth.logits(w)
@@ -608,7 +660,13 @@ def main():
     for _ in range(max(a.warmup, 3)):
         step()
     st = b.stats(stream)
-    launches_per_step = 8 if w.mode == 0 else 9
+    # kernels of ours per step: route; assignment count (+ scan when a source
+    # has more than 32 chunks of 2048 assignments, + row offsets in ragged
+    # mode) and rank; pack; bucket; expert; combine
+    chunk_tokens = min(max(2048 // w.k, 1), w.T // w.R if w.mode == 0 else w.T)
+    chunks_per_source = -(-(w.T // w.R) // chunk_tokens)
+    assign_kernels = (2 if chunks_per_source <= 32 else 3) if w.mode == 0 else 4
+    launches_per_step = 5 + assign_kernels
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(a.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -716,40 +774,10 @@ def main():
         del b.d_ret, b.d_pool, b.dout, b.dlogits, b.dx
         torch.cuda.empty_cache()
 
-    # sequence-level balance term and its gradient (reported apart): logits
-    # read twice (statistics, gradient), dlogits written once
+    # sequence-level balance term and its gradient (reported apart)
     bal = None
-    if not a.no_backward and w.T % w.seq_len == 0:
-        n_seq = w.T // w.seq_len
-        bf = torch.empty((n_seq, w.E), dtype=torch.float32, device=dev)
-        bP = torch.empty_like(bf)
-        bl = torch.empty((n_seq,), dtype=torch.float32, device=dev)
-        bd = torch.empty((w.T, w.E), dtype=torch.float32, device=dev)
-        bws = torch.empty((max(mp.moe_pw_seq_balance_plan(cfg, w.seq_len), 256),),
-                          dtype=torch.uint8, device=dev)
-
-        def bal_step():
-            mp.moe_pw_seq_balance(cfg, w.seq_len, 0.01, b.logits, b.idx, bf, bP, bl, bws,
-                                  dlogits=bd, stream=stream)
-        for _ in range(3):
-            bal_step()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(a.steps):
-            bal_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        (bms,) = max_over_ranks([e0.elapsed_time(e1) / a.steps], world, dev)
-        bbytes = 2 * 4 * w.T * w.E + 4 * w.T * w.k + 4 * w.T * w.E
-        bal = {"ms_per_step": bms, "alg_bytes_per_step": bbytes,
-               "hbm_gbs": bbytes / (bms / 1e3) / 1e9,
-               "hbm_frac_of_peak": bbytes / (bms / 1e3) / 1e9 / measured_peaks()[0],
-               "mean_term_alpha_1": float(bl.double().mean().item()) / 0.01,
-               "scope": "balance term per sequence and its gradient (logits read twice, "
-                        "dlogits written)"}
-        del bf, bP, bl, bd, bws
-        torch.cuda.empty_cache()
+    if not a.no_backward:
+        bal = time_balance(w, cfg, b, dev, stream, a.steps, world)
 
     proj = None
     if not a.no_projection:
