@@ -14,15 +14,16 @@
 //
 // Three kernels, all deterministic (fixed summation orders, integer counts):
 //   1. stats: block per (sequence, chunk of BAL_CHUNK tokens); a warp per
-//      token computes the row's max and sum of exponentials (warp reductions)
-//      and adds p into per-lane accumulators of the experts it holds, tokens
-//      in order; the block sums its warps in order and writes the chunk's
-//      partial sums; the chunk's expert counts come from shared-memory
-//      atomics on idx (integers: order does not matter);
+//      token (the next row loaded while this one is reduced) computes the
+//      row's max and sum of exponentials (warp reductions) and adds p into
+//      per-lane accumulators of the experts it holds, tokens in order; the
+//      block sums its warps in order and writes the chunk's partial sums; the
+//      chunk's expert counts come from shared-memory atomics on idx
+//      (integers: order does not matter);
 //   2. finish: block per sequence; partial sums over chunks in order, f, P and
 //      the loss (a fixed-order block reduction over experts);
-//   3. grad (optional): a warp per token, p again, dot = sum_i f_i p_i by a
-//      fixed xor tree, dlogits written or added.
+//   3. grad (optional): a warp per token (next row in flight), p again,
+//      dot = sum_i f_i p_i by a fixed xor tree, dlogits written or added.
 // Reads the logits once per pass (HBM-bound); no tensor cores.
 #include "common.cuh"
 
@@ -32,7 +33,7 @@ namespace {
 
 constexpr int BAL_THREADS = 256;
 constexpr int BAL_WARPS = BAL_THREADS / 32;
-constexpr int BAL_CHUNK = 256;  // tokens per stats block
+constexpr int BAL_CHUNK = 128;  // tokens per stats block
 
 struct BalArgs {
     const float *logits;
@@ -106,9 +107,14 @@ __global__ void __launch_bounds__(BAL_THREADS) balance_stats(BalArgs a)
     float acc[NV * 4];
 #pragma unroll
     for (int i = 0; i < NV * 4; ++i) acc[i] = 0.0f;
+    // the next token's row is loaded while the current one is reduced
+    float nx[NV * 4];
+    if (t0 + warp < t1) load_row<NV>(a, t0 + warp, lane, nx);
     for (int64_t t = t0 + warp; t < t1; t += BAL_WARPS) {
         float x[NV * 4];
-        load_row<NV>(a, t, lane, x);
+#pragma unroll
+        for (int i = 0; i < NV * 4; ++i) x[i] = nx[i];
+        if (t + BAL_WARPS < t1) load_row<NV>(a, t + BAL_WARPS, lane, nx);
         softmax_row<NV>(x);
 #pragma unroll
         for (int i = 0; i < NV * 4; ++i) acc[i] += x[i];
@@ -166,10 +172,14 @@ __global__ void __launch_bounds__(BAL_THREADS) balance_grad(BalArgs a)
     const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarp = (int64_t(gridDim.x) * blockDim.x) >> 5;
     const int E4 = a.E >> 2;
+    float nx[NV * 4];
+    if (warp < a.T) load_row<NV>(a, warp, lane, nx);
     for (int64_t t = warp; t < a.T; t += nwarp) {
         const int64_t s = t / a.L;
         float x[NV * 4], fv[NV * 4];
-        load_row<NV>(a, t, lane, x);
+#pragma unroll
+        for (int i = 0; i < NV * 4; ++i) x[i] = nx[i];
+        if (t + nwarp < a.T) load_row<NV>(a, t + nwarp, lane, nx);  // next row in flight
         softmax_row<NV>(x);
         float dot = 0.0f;
 #pragma unroll

@@ -4,8 +4,9 @@ oracle's definition (orc_seq_balance), through the C ABI.
 Bounds (derived from the fp32 arithmetic; u = 2^-24):
 - f: an integer count times E/(kL): two roundings, 2u relative.
 - P: each probability (expf and one division) within 4u; a lane adds at most
-  32 of them per chunk, the block 8 warps, then the chunks in order: within
-  (32 + 8 + chunks + 8) u of the positive sum, doubled for margin.
+  32 of them per chunk (of 128 tokens: 16 per warp), the block 8 warps, then
+  the chunks in order: within (32 + 8 + chunks + 8) u of the positive sum,
+  doubled for margin.
 - loss: P's bound plus the fixed-order sum over E positive terms,
   (E/256 + 8) u.
 - dlogits = alpha/L * p (f - dot): dot is a sum of E positive products
@@ -50,7 +51,7 @@ def run(w, L, accumulate_on=None):
 
 def check(w, L, g, lg, idx, f, P, loss, dl, base=None):
     fr, Pr, lr, dr = oracle.seq_balance(g, L, ALPHA, lg, idx)
-    chunks = (L + 255) // 256
+    chunks = (L + 127) // 128
     np.testing.assert_allclose(f, fr, rtol=2 * U, atol=0)
     rp = 2 * (32 + 8 + chunks + 8) * U
     assert np.all(np.abs(P - Pr) <= rp * Pr + 1e-30)
