@@ -146,9 +146,11 @@ __global__ void __launch_bounds__(BAL_THREADS) balance_finish(BalArgs a)
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
         float sum = 0.0f;
         int64_t n = 0;
+        // chunks in order; unrolled so the loads of 8 chunks are in flight together
+#pragma unroll 8
         for (int c = 0; c < a.chunks; ++c) {
-            sum += a.part[(s * a.chunks + c) * a.E + e];
-            n += a.cnt[(s * a.chunks + c) * a.E + e];
+            sum += __ldcg(a.part + (s * a.chunks + c) * a.E + e);
+            n += __ldcg(a.cnt + (s * a.chunks + c) * a.E + e);
         }
         const float P = sum / float(a.L);
         const float f = float(n) * scale_f;
@@ -182,14 +184,17 @@ __global__ void __launch_bounds__(BAL_THREADS) balance_grad(BalArgs a)
         if (t + nwarp < a.T) load_row<NV>(a, t + nwarp, lane, nx);  // next row in flight
         softmax_row<NV>(x);
         float dot = 0.0f;
+        const float4 *frow = reinterpret_cast<const float4 *>(a.f + s * a.E);
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
             const int q = lane + 32 * v;
+            const float4 f4 = q < E4 ? __ldg(frow + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            fv[4 * v + 0] = f4.x;
+            fv[4 * v + 1] = f4.y;
+            fv[4 * v + 2] = f4.z;
+            fv[4 * v + 3] = f4.w;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                fv[4 * v + cc] = q < E4 ? a.f[s * a.E + 4 * q + cc] : 0.0f;
-                dot = fmaf(fv[4 * v + cc], x[4 * v + cc], dot);
-            }
+            for (int cc = 0; cc < 4; ++cc) dot = fmaf(fv[4 * v + cc], x[4 * v + cc], dot);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(FULL_MASK, dot, o);

@@ -450,7 +450,7 @@ int moe_pw_seq_balance(const moe_pw_config *cfg, int64_t seq_len, float alpha,
     if (g.T == 0) return MOE_PW_OK;
     if (!logits || !idx || !f || !P || !loss || !workspace) return MOE_PW_EINVAL;
     if (int64_t(workspace_bytes) < balance_ws_bytes(g.T, seq_len, g.E)) return MOE_PW_EINVAL;
-    if (!aligned(logits, 16) || !aligned(idx, 4) || !aligned(f, 4) || !aligned(P, 4) ||
+    if (!aligned(logits, 16) || !aligned(idx, 4) || !aligned(f, 16) || !aligned(P, 4) ||
         !aligned(loss, 4) || !aligned(workspace, 256) || (dlogits && !aligned(dlogits, 16)))
         return MOE_PW_EUNSUPPORTED;
     return cuda_rc(launch_balance(g, seq_len, alpha, logits, idx, f, P, loss, dlogits, accumulate,

@@ -394,7 +394,8 @@ int moe_pw_project_pack(const moe_pw_config *cfg, const uint16_t *h, const uint1
  *   dlogits[t][e] = alpha / L * p[t][e] * (f[s][e] - sum_i f[s][i] p[t][i]),
  * written (accumulate = 0) or added to dlogits (accumulate != 0, e.g. onto
  * the top-k softmax gradient of moe_pw_combine_backward).  logits f32 [T, E]
- * (16-byte aligned), idx i32 [T, k]; f, P f32 [T / L, E]; loss f32 [T / L];
+ * (16-byte aligned), idx i32 [T, k]; f (16-byte aligned), P f32 [T / L, E];
+ * loss f32 [T / L];
  * dlogits f32 [T, E] (16-byte aligned).  Sums in fp32 in a fixed order
  * (deterministic).  workspace: at least the bytes moe_pw_seq_balance_plan
  * gives, 256-byte aligned.  E % 4 == 0.
