@@ -155,10 +155,17 @@ __global__ void __launch_bounds__(BK_THREADS, 2) bucket_pooled(BucketArgs p)
             run[4 * v + 3] = x.w;
         }
         for (int pp = 0; pp < P; ++pp) {
-            uint32_t mine = 0;  // bit i: run position i holds local expert pp
+            // bit i: run position i holds local expert pp.  Four positions per
+            // word: a bytewise compare, then the four byte flags gathered into
+            // bits 28..31 by one multiply (the other partial products stay
+            // below bit 24, so nothing carries into them)
+            uint32_t mine = 0;
+            const uint32_t key = uint32_t(pp) * 0x01010101u;
 #pragma unroll
-            for (int i = 0; i < BK_ITEMS; ++i)
-                mine |= uint32_t(int8_t(run[i >> 2] >> (8 * (i & 3))) == pp) << i;
+            for (int wi = 0; wi < BK_ITEMS / 4; ++wi) {
+                const uint32_t eq = __vcmpeq4(run[wi], key) & 0x01010101u;
+                mine |= ((eq * 0x10204080u) >> 28) << (4 * wi);
+            }
             int32_t total;
             const int32_t first = block_exclusive_scan(__popc(mine), wsum, &total);
             int32_t r = carry[pp] + first;

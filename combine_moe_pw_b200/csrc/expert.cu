@@ -51,7 +51,16 @@ __global__ void __launch_bounds__(256) expert_kernel(ExpertArgs a)
     const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarp = (int64_t(gridDim.x) * blockDim.x) >> 5;
     const int cpr = a.cpr;
-    for (int64_t slot = warp; slot < a.n_slots; slot += nwarp) {
+    // one wave only (expert-parallel runs overlap the waves): walk just that
+    // wave's slots, every W-th run of C_s slots of the receive pool
+    const int one_wave = EP && __popc(a.wave_mask) == 1 ? __ffs(a.wave_mask) - 1 : -1;
+    const int64_t n_walk = one_wave >= 0 ? a.n_slots / a.geo.W : a.n_slots;
+    for (int64_t i = warp; i < n_walk; i += nwarp) {
+        int64_t slot = i;
+        if (one_wave >= 0) {
+            const int64_t run = i / a.geo.C_s;
+            slot = (run * a.geo.W + one_wave) * a.geo.C_s + (i - run * a.geo.C_s);
+        }
         uint4 *dst;
         int32_t *dst_hdr;
         if (EP) {

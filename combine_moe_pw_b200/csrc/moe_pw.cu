@@ -153,7 +153,7 @@ const char *moe_pw_strerror(int code)
     switch (code) {
     case MOE_PW_OK: return "ok";
     case MOE_PW_EINVAL: return "invalid argument or config";
-    case MOE_PW_EUNSUPPORTED: return "shape or alignment not supported by this build";
+    case MOE_PW_EUNSUPPORTED: return "shape or alignment not supported by this library";
     case MOE_PW_ECUDA: return "CUDA runtime or launch error";
     case MOE_PW_EDEVICE: return "a kernel flagged a violation (see counters.error)";
     case MOE_PW_ENOMEM: return "buffers exceed the memory budget or the built-in scratch limit";
@@ -760,8 +760,8 @@ int moe_pw_ep_bucket(const moe_pw_config *cfg, const moe_pw_ep *ep, const int32_
     Geo g;
     int rc = make_geo_ep(cfg, ep, &g);
     if (rc != MOE_PW_OK) return rc;
-    if (!counters || !expert_counts || !recv_hdr || !recv_row || !bucket_slot)
-        return MOE_PW_EINVAL;
+    if (!counters || !expert_counts) return MOE_PW_EINVAL;
+    if (g.n_slots > 0 && (!recv_hdr || !recv_row || !bucket_slot)) return MOE_PW_EINVAL;
     if (!aligned(counters, 8) || !aligned(expert_counts, 4) || !aligned(recv_hdr, 4) ||
         !aligned(recv_row, 4) || !aligned(bucket_slot, 4))
         return MOE_PW_EUNSUPPORTED;

@@ -184,15 +184,24 @@ route_kernel(const float *__restrict__ logits, int32_t *__restrict__ idx,
             }
         }
 
-        // softmax over the chosen logits, summed in choice order: lane j holds choice j
+        // softmax over the chosen logits: lane j holds choice j
         const float val = key_value(sel_key);
         const float top = __shfl_sync(FULL_MASK, val, 0);
         const float ex = (lane < k) ? expf(val - top) : 0.0f;
         float sum = 0.0f;
+        if (KC == 8) {
+            // butterfly over lanes 0..7: every lane of the group ends with the
+            // same bits (each add's operands only swap places)
+            sum = ex;
+            sum += __shfl_xor_sync(FULL_MASK, sum, 1);
+            sum += __shfl_xor_sync(FULL_MASK, sum, 2);
+            sum += __shfl_xor_sync(FULL_MASK, sum, 4);
+        } else {
 #pragma unroll
-        for (int j = 0; j < (KC ? KC : 1); ++j) sum += __shfl_sync(FULL_MASK, ex, j);
-        if (!KC)
-            for (int j = 1; j < k; ++j) sum += __shfl_sync(FULL_MASK, ex, j);
+            for (int j = 0; j < (KC ? KC : 1); ++j) sum += __shfl_sync(FULL_MASK, ex, j);
+            if (!KC)
+                for (int j = 1; j < k; ++j) sum += __shfl_sync(FULL_MASK, ex, j);
+        }
         if (lane < k) {
             idx[t * k + lane] = sel_idx;
             gates[t * k + lane] = ex / sum;

@@ -29,7 +29,9 @@
  *     {P*w, ..., P*w + P - 1} (P = L / W);
  *   - top-k order is (logit descending, expert id ascending): equal logits go
  *     to the lower id (float comparison: -0.0 equals +0.0); gates are the
- *     softmax over the k chosen logits, max-subtracted, summed in j order;
+ *     softmax over the k chosen logits, max-subtracted (the device sums the
+ *     k exponentials in a fixed order: a butterfly for k = 8, j order
+ *     otherwise; gates agree with the exact softmax within 1e-6);
  *   - sender order: assignments (t, j) of a source in lexicographic order; the
  *     slot of (t, j) in pool (s, d, w) is the number of earlier ones in that
  *     pool; kept iff slot < C_s;
@@ -91,7 +93,7 @@ extern "C" {
 
 #define MOE_PW_OK 0
 #define MOE_PW_EINVAL (-1)        /* null pointer, bad config, inconsistent sizes */
-#define MOE_PW_EUNSUPPORTED (-2)  /* shape or alignment this build does not handle */
+#define MOE_PW_EUNSUPPORTED (-2)  /* shape or alignment this library does not handle */
 #define MOE_PW_ECUDA (-3)         /* a CUDA runtime call or a launch failed */
 #define MOE_PW_EDEVICE (-4)       /* a kernel flagged a violation (moe_pw_stats) */
 #define MOE_PW_ENOMEM (-5)        /* buffers exceed the caller's budget (moe_pw_plan) or the
@@ -111,7 +113,7 @@ extern "C" {
                                        the context) as suspect and re-run the step */
 #define MOE_PW_DEVERR_SLOT 8        /* slot_map entry outside [-1, n_slots) */
 
-/* Problem description.  Limits of this build: 1 <= k <= 32, k <= E,
+/* Problem description.  Limits of this library: 1 <= k <= 32, k <= E,
  * E == R * L, L == W * P, E <= 2048 (and E % 4 == 0 for moe_pw_route),
  * T % R == 0, 8 <= D <= 12288 with D % 8 == 0, R * W <= 2048. */
 typedef struct moe_pw_config {

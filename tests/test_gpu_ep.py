@@ -125,3 +125,17 @@ def test_ep_rejects_bad_shares():
     b = ep.EpBuffers(cfg, 2, 0)
     with pytest.raises(mp.MoePwError):
         b.pack()                              # GPU 1's receive pool is not in the table
+
+
+def test_ep_empty_batch():
+    """No tokens: every share's step runs and reports nothing kept or dropped."""
+    w = TINY.with_(T=0)
+    cfg = mp.Config.from_workload(w)
+    shares = [ep.EpBuffers(cfg, 2, g) for g in range(2)]
+    for b in shares:
+        b.expert_counts.fill_(7)
+    ep.emulate_step(shares)
+    for b in shares:
+        st = b.stats()
+        assert (st.assignments, st.kept, st.sender_dropped, st.receiver_dropped) == (0, 0, 0, 0)
+        assert int(b.expert_counts.abs().sum()) == 0
