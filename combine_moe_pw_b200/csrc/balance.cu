@@ -174,28 +174,40 @@ __global__ void __launch_bounds__(BAL_THREADS) balance_grad(BalArgs a)
     const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarp = (int64_t(gridDim.x) * blockDim.x) >> 5;
     const int E4 = a.E >> 2;
-    float nx[NV * 4];
-    if (warp < a.T) load_row<NV>(a, warp, lane, nx);
-    for (int64_t t = warp; t < a.T; t += nwarp) {
-        const int64_t s = t / a.L;
-        float x[NV * 4], fv[NV * 4];
-#pragma unroll
-        for (int i = 0; i < NV * 4; ++i) x[i] = nx[i];
-        if (t + nwarp < a.T) load_row<NV>(a, t + nwarp, lane, nx);  // next row in flight
-        softmax_row<NV>(x);
-        float dot = 0.0f;
-        const float4 *frow = reinterpret_cast<const float4 *>(a.f + s * a.E);
+    // the next token's logits and its sequence's f row are loaded while the
+    // current token is worked on
+    float nx[NV * 4], nf[NV * 4];
+    auto load_f = [&](int64_t t, float (&fo)[NV * 4]) {
+        const float4 *frow = reinterpret_cast<const float4 *>(a.f + (t / a.L) * a.E);
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
             const int q = lane + 32 * v;
             const float4 f4 = q < E4 ? __ldg(frow + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-            fv[4 * v + 0] = f4.x;
-            fv[4 * v + 1] = f4.y;
-            fv[4 * v + 2] = f4.z;
-            fv[4 * v + 3] = f4.w;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) dot = fmaf(fv[4 * v + cc], x[4 * v + cc], dot);
+            fo[4 * v + 0] = f4.x;
+            fo[4 * v + 1] = f4.y;
+            fo[4 * v + 2] = f4.z;
+            fo[4 * v + 3] = f4.w;
         }
+    };
+    if (warp < a.T) {
+        load_row<NV>(a, warp, lane, nx);
+        load_f(warp, nf);
+    }
+    for (int64_t t = warp; t < a.T; t += nwarp) {
+        float x[NV * 4], fv[NV * 4];
+#pragma unroll
+        for (int i = 0; i < NV * 4; ++i) {
+            x[i] = nx[i];
+            fv[i] = nf[i];
+        }
+        if (t + nwarp < a.T) {
+            load_row<NV>(a, t + nwarp, lane, nx);
+            load_f(t + nwarp, nf);
+        }
+        softmax_row<NV>(x);
+        float dot = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NV * 4; ++i) dot = fmaf(fv[i], x[i], dot);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(FULL_MASK, dot, o);
         const float g = a.alpha / float(a.L);
