@@ -139,12 +139,16 @@ def time_projection(w, dev, stream, steps: int, b=None):
         out["project_then_pack_ms"] = timed(two_step)
         # the whole routed branch, model width to model width
         lat = torch.empty(T, D, dtype=torch.int16, device=dev)
-        out["routed_layer_ms"] = timed(lambda: b.run_routed_layer(h, wd, wu, Dm, lat, y, stream))
+        out["routed_layer_ms"] = timed(lambda: b.run_routed_layer(h, wd, wu, Dm, lat, y, stream,
+                                                                  overlap=False))
         out["routed_layer_tokens_per_s"] = T / (out["routed_layer_ms"] / 1e3)
         # merged with a shared-path output, sequential and with the combine
         # and up-projection overlapped in 8192-token blocks
         sh = torch.randn(T, Dm, device=dev, generator=g).to(torch.bfloat16).view(torch.int16)
         out["routed_layer_merged_ms"] = timed(
+            lambda: b.run_routed_layer(h, wd, wu, Dm, lat, y, stream, shared_out=sh,
+                                       overlap=False))
+        out["routed_layer_merged_default_ms"] = timed(
             lambda: b.run_routed_layer(h, wd, wu, Dm, lat, y, stream, shared_out=sh))
         for chunk in (4096, 8192, 16384):
             out[f"routed_layer_merged_pipelined_{chunk}_ms"] = timed(

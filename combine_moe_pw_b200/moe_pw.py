@@ -584,16 +584,28 @@ class Buffers:
         moe_pw_dispatch_backward(self.cfg, self.d_pool, self.recv_row, self.slot_map, self.dx,
                                  self.counters, stream)
 
+    OVERLAP_BLOCK_TOKENS = 16384  # the fastest block size measured on the rack batch
+
     def run_routed_layer(self, h, w_down_t, w_up_t, model_width: int, latent_bf16, out_model,
-                         stream=None, shared_out=None):
+                         stream=None, shared_out=None, overlap: bool = True):
         """The whole routed branch from model width back to model width:
         route -> assign -> down-projection fused with the pack -> bucket ->
         expert op -> combine (bf16 latent) -> up-projection.  h: bf16 [T, Dm],
         w_down_t: bf16 [D, Dm], w_up_t: bf16 [Dm, D], latent_bf16: bf16 [T, D]
         (scratch), out_model: bf16 [T, Dm].  With shared_out (bf16 [T, Dm],
         the shared experts' output) the up-projection's epilogue adds it: the
-        merge of the two paths."""
+        merge of the two paths.  With overlap (and at least two blocks of
+        OVERLAP_BLOCK_TOKENS tokens) the combine and the up-projection run
+        block by block on two streams (run_routed_layer_pipelined), the two
+        block buffers taken from latent_bf16; the bytes are the same."""
         cfg = self.cfg
+        blk = self.OVERLAP_BLOCK_TOKENS
+        if overlap and cfg.T >= 2 * blk:
+            self.run_routed_layer_pipelined(h, w_down_t, w_up_t, model_width, out_model,
+                                            shared_out=shared_out, chunk_tokens=blk,
+                                            stream=stream,
+                                            latent_chunks=[latent_bf16[:blk], latent_bf16[blk:2 * blk]])
+            return
         self.route(stream)
         self.assign(stream)
         moe_pw_project_pack(cfg, h, w_down_t, model_width, self.idx, self.slot_map, self.occ,

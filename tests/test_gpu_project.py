@@ -259,7 +259,7 @@ def test_pipelined_routed_layer_equals_sequential(chunk):
     lat = torch.empty((w.T, w.D), dtype=torch.int16, device="cuda")
     for shared in (None, S):
         ref = torch.empty((w.T, Dm), dtype=torch.int16, device="cuda")
-        b.run_routed_layer(h, wd, wu, Dm, lat, ref, shared_out=shared)
+        b.run_routed_layer(h, wd, wu, Dm, lat, ref, shared_out=shared, overlap=False)
         got = torch.full((w.T, Dm), 0x7FC0, dtype=torch.int16, device="cuda")
         b.run_routed_layer_pipelined(h, wd, wu, Dm, got, shared_out=shared, chunk_tokens=chunk)
         torch.cuda.synchronize()
@@ -326,3 +326,25 @@ def test_one_sm_fallback_matches_pair_kernel(tmp_path):
         C, _ = gpu_project(A, Bt)
         check_project(A, Bt, C)
         np.testing.assert_array_equal(C, one_sm[f"{M}_{N}_{K}"].view(np.uint16))
+
+
+def test_routed_layer_default_overlaps_large_batches():
+    """At two or more blocks of 16,384 tokens run_routed_layer overlaps the
+    combine and the up-projection by default, using its latent scratch for
+    the two block buffers: the same bytes as the sequential chain."""
+    w = synth.Workload("two_blocks", T=64 * 600, R=64, L=6, W=3, P=2, k=8, D=256, seq_len=600,
+                       logit_kind=synth.LOGIT_SEQBIAS)
+    Dm = 512
+    h, wd, wu = (torch.from_numpy(a.view(np.int16)).cuda() for a in synth.projection_inputs(w, Dm))
+    S = torch.from_numpy(synth.matrix_bf16(w.T, Dm, 1.0, 65).view(np.int16)).cuda()
+    b = mp.Buffers(mp.Config.from_workload(w))
+    b.logits.copy_(torch.from_numpy(synth.logits(w)))
+    b.scale.copy_(torch.from_numpy(synth.scales(w)))
+    lat = torch.empty((w.T, w.D), dtype=torch.int16, device="cuda")
+    ref = torch.empty((w.T, Dm), dtype=torch.int16, device="cuda")
+    b.run_routed_layer(h, wd, wu, Dm, lat, ref, shared_out=S, overlap=False)
+    got = torch.full((w.T, Dm), 0x7FC0, dtype=torch.int16, device="cuda")
+    assert w.T >= 2 * b.OVERLAP_BLOCK_TOKENS
+    b.run_routed_layer(h, wd, wu, Dm, lat, got, shared_out=S)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
