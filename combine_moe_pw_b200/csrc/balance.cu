@@ -82,8 +82,11 @@ __device__ __forceinline__ void softmax_row(float (&x)[NV * 4])
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL_MASK, sum, o);
+    // one IEEE division per lane, then products (within 2 ulp of x / sum):
+    // the per-element divisions made the pass issue-bound
+    const float inv = 1.0f / sum;
 #pragma unroll
-    for (int i = 0; i < NV * 4; ++i) x[i] = x[i] / sum;
+    for (int i = 0; i < NV * 4; ++i) x[i] = x[i] * inv;
 }
 
 template <int NV>

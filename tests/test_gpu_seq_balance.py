@@ -3,7 +3,7 @@ oracle's definition (orc_seq_balance), through the C ABI.
 
 Bounds (derived from the fp32 arithmetic; u = 2^-24):
 - f: an integer count times E/(kL): two roundings, 2u relative.
-- P: each probability (expf and one division) within 4u; a lane adds at most
+- P: each probability (expf, a reciprocal and a product) within 5u; a lane adds at most
   32 of them per chunk (of 128 tokens: 16 per warp), the block 8 warps, then
   the chunks in order: within (32 + 8 + chunks + 8) u of the positive sum,
   doubled for margin.
