@@ -148,8 +148,9 @@ def time_projection(w, dev, stream, steps: int, b=None):
         out["routed_layer_merged_ms"] = timed(
             lambda: b.run_routed_layer(h, wd, wu, Dm, lat, y, stream, shared_out=sh,
                                        overlap=False))
-        out["routed_layer_merged_default_ms"] = timed(
-            lambda: b.run_routed_layer(h, wd, wu, Dm, lat, y, stream, shared_out=sh))
+        out["routed_layer_merged_overlap_ms"] = timed(
+            lambda: b.run_routed_layer(h, wd, wu, Dm, lat, y, stream, shared_out=sh,
+                                       overlap=True))
         for chunk in (4096, 8192, 16384):
             out[f"routed_layer_merged_pipelined_{chunk}_ms"] = timed(
                 lambda: b.run_routed_layer_pipelined(h, wd, wu, Dm, y, shared_out=sh,

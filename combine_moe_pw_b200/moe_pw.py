@@ -584,10 +584,10 @@ class Buffers:
         moe_pw_dispatch_backward(self.cfg, self.d_pool, self.recv_row, self.slot_map, self.dx,
                                  self.counters, stream)
 
-    OVERLAP_BLOCK_TOKENS = 16384  # the fastest block size measured on the rack batch
+    OVERLAP_BLOCK_TOKENS = 16384  # block size for the overlapped routed layer
 
     def run_routed_layer(self, h, w_down_t, w_up_t, model_width: int, latent_bf16, out_model,
-                         stream=None, shared_out=None, overlap: bool = True):
+                         stream=None, shared_out=None, overlap: bool = False):
         """The whole routed branch from model width back to model width:
         route -> assign -> down-projection fused with the pack -> bucket ->
         expert op -> combine (bf16 latent) -> up-projection.  h: bf16 [T, Dm],
@@ -597,7 +597,10 @@ class Buffers:
         merge of the two paths.  With overlap (and at least two blocks of
         OVERLAP_BLOCK_TOKENS tokens) the combine and the up-projection run
         block by block on two streams (run_routed_layer_pipelined), the two
-        block buffers taken from latent_bf16; the bytes are the same."""
+        block buffers taken from latent_bf16; the bytes are the same.  Off by
+        default: on the rack batch the GEMMs run at the power cap, and with the
+        combine beside them the overlap gained 1 ms in one run and lost 0.5 ms
+        in another."""
         cfg = self.cfg
         blk = self.OVERLAP_BLOCK_TOKENS
         if overlap and cfg.T >= 2 * blk:
@@ -628,9 +631,9 @@ class Buffers:
         block by block: the combine of token block c + 1 (HBM-bound) runs on
         one stream while the up-projection of block c (tensor-bound) runs on
         another, and the bf16 latent passes through two buffers of
-        chunk_tokens rows (latent_chunks, allocated here if not given) that
-        are rewritten before they can leave L2.  Same kernels, same per-row
-        arithmetic: the output equals run_routed_layer's bit for bit."""
+        chunk_tokens rows (latent_chunks, allocated here if not given) instead
+        of a whole-batch array.  Same kernels, same per-row arithmetic: the
+        output equals run_routed_layer's bit for bit."""
         cfg = self.cfg
         dev = self.out.device
         s0 = stream if stream is not None else torch.cuda.current_stream(dev)

@@ -328,9 +328,9 @@ def test_one_sm_fallback_matches_pair_kernel(tmp_path):
         np.testing.assert_array_equal(C, one_sm[f"{M}_{N}_{K}"].view(np.uint16))
 
 
-def test_routed_layer_default_overlaps_large_batches():
-    """At two or more blocks of 16,384 tokens run_routed_layer overlaps the
-    combine and the up-projection by default, using its latent scratch for
+def test_routed_layer_overlap_on_large_batches():
+    """At two or more blocks of 16,384 tokens run_routed_layer(overlap=True)
+    overlaps the combine and the up-projection, using its latent scratch for
     the two block buffers: the same bytes as the sequential chain."""
     w = synth.Workload("two_blocks", T=64 * 600, R=64, L=6, W=3, P=2, k=8, D=256, seq_len=600,
                        logit_kind=synth.LOGIT_SEQBIAS)
@@ -345,6 +345,6 @@ def test_routed_layer_default_overlaps_large_batches():
     b.run_routed_layer(h, wd, wu, Dm, lat, ref, shared_out=S, overlap=False)
     got = torch.full((w.T, Dm), 0x7FC0, dtype=torch.int16, device="cuda")
     assert w.T >= 2 * b.OVERLAP_BLOCK_TOKENS
-    b.run_routed_layer(h, wd, wu, Dm, lat, got, shared_out=S)
+    b.run_routed_layer(h, wd, wu, Dm, lat, got, shared_out=S, overlap=True)
     torch.cuda.synchronize()
     assert torch.equal(got, ref)
