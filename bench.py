@@ -4,11 +4,12 @@
     python bench.py --impl reference ...        # the CPU oracle as the reference arm
     torchrun --nproc-per-node N bench.py --gpus N ...
 
-One step = route -> dispatch (assign, pack, bucket) -> per-expert op ->
-combine -> drop statistics, on one synthetic batch already resident in HBM.
-The metric is routed assignments per second for dispatch + combine: T*k
-divided by the device time of route + assign + pack + bucket + combine, each
-timed with CUDA events on the launching stream inside the K timed steps (the
+One step = route -> dispatch (assign, then pack and bucketing in one launch;
+dropless ragged mode: assign, pack, bucket) -> per-expert op -> combine ->
+drop statistics, on one synthetic batch already resident in HBM.  The metric
+is routed assignments per second for dispatch + combine: T*k divided by the
+device time of route + assign + pack/bucket + combine, each timed with CUDA
+events on the launching stream inside the K timed steps (the
 per-expert op runs in every step but is timed apart, since it stands in for
 the expert network).  HBM GB/s and the fraction of the measured copy peak use
 the algorithmic bytes of those stages.
@@ -48,6 +49,9 @@ def parse():
     ap.add_argument("--workload", default="rack")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--separate-dispatch", action="store_true",
+                    help="pooled mode: pack and bucketing as two launches (the fused launch "
+                         "is the default)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
     ap.add_argument("--cpu-sample-sources", type=int, default=16)
@@ -253,7 +257,13 @@ def alg_bytes(w, stats, C_s):
     pack = 2 * T * D + 8 * T * k + S * (2 * D + 4)      # x rows, slot_map + idx, pool rows + headers
     bucket = 8 * S                                      # read headers, write receiver rows
     combine = 8 * T * k + 4 * K_s + 2 * D * K + 4 * T * D
+    # fused dispatch: the assignment writes the kept slots' headers; the
+    # pack + bucketing launch reads the slot map (not the ids), writes rows
+    # and the empty slots' headers, and buckets
+    assign_headers = assign + 4 * K_s
+    pack_bucket = 2 * T * D + 4 * T * k + S * 2 * D + 4 * (S - K_s) + bucket
     return {"route": route, "assign": assign, "pack": pack, "bucket": bucket, "combine": combine,
+            "assign_headers": assign_headers, "pack_bucket": pack_bucket,
             "expert": 2 * D * K + 8 * S + S * (2 * D + 4)}
 
 
@@ -644,25 +654,22 @@ def main():
             print(json.dumps({"projection": proj}), flush=True)
         return
 
-    stages = ["route", "assign", "pack", "bucket", "expert", "combine"]
+    fused = w.mode == 0 and not a.separate_dispatch
+    if fused:
+        stages = ["route", "assign_headers", "pack_bucket", "expert", "combine"]
+        dispatch_calls = [b.assign_headers, b.pack_bucket]
+    else:
+        stages = ["route", "assign", "pack", "bucket", "expert", "combine"]
+        dispatch_calls = [b.assign, b.pack, b.bucket]
+    calls = [b.route, *dispatch_calls, b.expert, b.combine]
 
     def step(evs=None):
-        def mark(i):
+        for i, f in enumerate(calls):
             if evs is not None:
                 evs[i].record(stream)
-        mark(0)
-        b.route(stream)
-        mark(1)
-        b.assign(stream)
-        mark(2)
-        b.pack(stream)
-        mark(3)
-        b.bucket(stream)
-        mark(4)
-        b.expert(stream)
-        mark(5)
-        b.combine(stream)
-        mark(6)
+            f(stream)
+        if evs is not None:
+            evs[len(calls)].record(stream)
 
     # the counters are read after the loops, not per step: a per-step read
     # synchronises the host, and the GPU would then wait for the next step's
@@ -677,9 +684,10 @@ def main():
     chunk_tokens = min(max(2048 // w.k, 1), w.T // w.R if w.mode == 0 else w.T)
     chunks_per_source = -(-(w.T // w.R) // chunk_tokens)
     assign_kernels = (2 if chunks_per_source <= 32 else 3) if w.mode == 0 else 4
-    launches_per_step = 5 + assign_kernels
+    launches_per_step = (4 if fused else 5) + assign_kernels
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(a.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+           for _ in range(a.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     sampler.start()
@@ -726,7 +734,7 @@ def main():
     total_ms = start.elapsed_time(end)
     per_stage = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(a.steps)]
                  for j, n in enumerate(stages)}
-    dc_stages = ["route", "assign", "pack", "bucket", "combine"]
+    dc_stages = [n for n in stages if n != "expert"]
     dc_ms = sum(sum(per_stage[n]) for n in dc_stages)  # over K steps
     total_ms, dc_ms = max_over_ranks([total_ms, dc_ms], world, dev)
     value = throughput(w.T * w.k, a.steps, world, dc_ms)
@@ -735,8 +743,10 @@ def main():
     peak, peak_kind = measured_peaks()
     gbs = b_alg * a.steps / (dc_ms / 1e3) / 1e9
     stage_ms = {n: statistics.mean(v) for n, v in per_stage.items()}
-    dom = max(["pack", "combine"], key=lambda n: stage_ms[n])
-    kname = {"pack": "pack_kernel", "combine": "combine_kernel"}[dom]
+    pack_stage = "pack_bucket" if fused else "pack"
+    dom = max([pack_stage, "combine"], key=lambda n: stage_ms[n])
+    kname = {"pack": "pack_kernel", "pack_bucket": "pack_bucket_kernel",
+             "combine": "combine_kernel"}[dom]
     achieved = ab[dom] / (stage_ms[dom] / 1e3) / 1e9
     traffic = traffic_from_profiles(kname, ab[dom])
 

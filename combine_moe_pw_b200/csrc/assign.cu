@@ -43,6 +43,7 @@ struct RankArgs {
     moe_pw_counters *ctr;
     Geo g;
     int32_t fused_scan;  // pooled, few chunks per group: assign_rank takes the scan's part
+    int32_t *pool_hdr;   // optional: the kept slots' headers (the expert id)
 };
 
 __device__ __forceinline__ int32_t bin_of_expert(const Geo &g, int32_t e)
@@ -313,6 +314,7 @@ __global__ void __launch_bounds__(AW * 32) assign_rank(RankArgs p)
                     slot = int32_t((pool_base + b) * p.g.C_s + r);
             }
             p.slot_map[a0 + i] = slot;
+            if (p.pool_hdr && slot >= 0) p.pool_hdr[slot] = p.idx[a0 + i];
         }
     }
 }
@@ -326,7 +328,7 @@ size_t rank_smem_bytes(const Geo &g)
 }  // namespace
 
 cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, int32_t *occ,
-                          moe_pw_counters *ctr, void *ws, cudaStream_t st)
+                          moe_pw_counters *ctr, void *ws, cudaStream_t st, int32_t *pool_hdr)
 {
     cudaError_t err = cudaMemsetAsync(ctr, 0, sizeof(moe_pw_counters), st);
     if (err != cudaSuccess) return err;
@@ -342,6 +344,7 @@ cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, i
     p.totals = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + ws_counts_bytes(g));
     p.ctr = ctr;
     p.g = g;
+    p.pool_hdr = pool_hdr;
 
     const size_t smem = rank_smem_bytes(g);
     if (smem > 48 * 1024) {

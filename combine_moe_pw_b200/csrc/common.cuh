@@ -50,14 +50,25 @@ int dev_info(DevInfo *out);
 // Kernel launchers (asynchronous; return cudaError_t of the launch).
 cudaError_t launch_route(const Geo &g, const float *logits, int32_t *idx, float *gates,
                          cudaStream_t st);
+// pool_hdr (optional): also write the kept slots' headers (the expert id),
+// as the fused pack + bucketing launch expects.
 cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, int32_t *occ,
-                          moe_pw_counters *ctr, void *ws, cudaStream_t st);
+                          moe_pw_counters *ctr, void *ws, cudaStream_t st,
+                          int32_t *pool_hdr = nullptr);
 // ep (optional): the receive pools of every GPU of an expert-parallel run;
 // rows then go to the destination's GPU, only for waves in wave_mask.
 cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
                         const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
                         int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st,
                         const EpRows *ep = nullptr, uint32_t wave_mask = ~0u);
+// Pack and receiver bucketing in one launch (one GPU, pooled mode, T > 0):
+// the kept slots' headers must already be in pool_hdr (launch_assign with
+// pool_hdr); the launch writes the rows, the empty slots' headers and the
+// bucketing's outputs.
+cudaError_t launch_pack_bucket(const Geo &g, const uint16_t *x, const int32_t *idx,
+                               const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
+                               int32_t *pool_hdr, int32_t *recv_row, int32_t *bucket_slot,
+                               int32_t *expert_counts, moe_pw_counters *ctr, cudaStream_t st);
 // occ == nullptr: an empty slot is one whose header is -1 (expert-parallel
 // receive pools, where no counts are exchanged).
 cudaError_t launch_bucket(const Geo &g, const int32_t *pool_hdr, const int32_t *occ,

@@ -252,12 +252,63 @@ int moe_pw_bucket(const moe_pw_config *cfg, const int32_t *pool_hdr, const int32
                                  stream));
 }
 
+int moe_pw_assign_headers(const moe_pw_config *cfg, const int32_t *idx, int32_t *slot_map,
+                          int32_t *occ, int32_t *pool_hdr, moe_pw_counters *counters,
+                          void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.mode != MOE_PW_POOLED) return MOE_PW_EUNSUPPORTED;
+    if (!counters || !occ) return MOE_PW_EINVAL;
+    if (g.T > 0 && (!idx || !slot_map || !workspace || !pool_hdr)) return MOE_PW_EINVAL;
+    if (g.T > 0 && int64_t(workspace_bytes) < ws_bytes(g)) return MOE_PW_EINVAL;
+    if (!aligned(counters, 8) || !aligned(occ, 4) || (g.T > 0 && (!aligned(idx, 4) ||
+        !aligned(slot_map, 4) || !aligned(pool_hdr, 4) || !aligned(workspace, 256))))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_assign(g, idx, slot_map, occ, counters, workspace, stream, pool_hdr));
+}
+
+int moe_pw_pack_bucket(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
+                       const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
+                       int32_t *pool_hdr, int32_t *recv_row, int32_t *bucket_slot,
+                       int32_t *expert_counts, moe_pw_counters *counters, cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.mode != MOE_PW_POOLED) return MOE_PW_EUNSUPPORTED;
+    if (g.T == 0) {
+        rc = moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream);
+        if (rc != MOE_PW_OK) return rc;
+        return moe_pw_bucket(cfg, pool_hdr, occ, recv_row, bucket_slot, expert_counts, counters,
+                             stream);
+    }
+    if (!x || !idx || !slot_map || !occ || !pool_x || !pool_hdr || !recv_row || !bucket_slot ||
+        !expert_counts || !counters)
+        return MOE_PW_EINVAL;
+    if (!aligned(x, 16) || !aligned(pool_x, 16) || !aligned(idx, 4) || !aligned(slot_map, 4) ||
+        !aligned(occ, 4) || !aligned(pool_hdr, 4) || !aligned(recv_row, 4) ||
+        !aligned(bucket_slot, 4) || !aligned(expert_counts, 4) || !aligned(counters, 8))
+        return MOE_PW_EUNSUPPORTED;
+    return cuda_rc(launch_pack_bucket(g, x, idx, slot_map, occ, pool_x, pool_hdr, recv_row,
+                                      bucket_slot, expert_counts, counters, stream));
+}
+
 int moe_pw_dispatch(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
                     int32_t *slot_map, int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr,
                     int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,
                     moe_pw_counters *counters, void *workspace, size_t workspace_bytes,
                     cudaStream_t stream)
 {
+    if (cfg && cfg->mode == MOE_PW_POOLED) {
+        // the bucketing runs beside the row copies (same outputs)
+        int rc = moe_pw_assign_headers(cfg, idx, slot_map, occ, pool_hdr, counters, workspace,
+                                       workspace_bytes, stream);
+        if (rc != MOE_PW_OK) return rc;
+        return moe_pw_pack_bucket(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, recv_row,
+                                  bucket_slot, expert_counts, counters, stream);
+    }
     int rc = moe_pw_assign(cfg, idx, slot_map, occ, counters, workspace, workspace_bytes, stream);
     if (rc != MOE_PW_OK) return rc;
     rc = moe_pw_pack(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, counters, stream);

@@ -30,6 +30,7 @@
 // 8 and 20 made no measurable difference.
 #include <cstring>
 
+#include "bucket_body.cuh"
 #include "common.cuh"
 
 namespace moe_pw {
@@ -82,26 +83,43 @@ struct PackArgs {
     EpRows ep;
 };
 
-// EP: rows and tails go to the destination GPUs' receive pools (peer stores).
-template <int LAG, bool EP>
-__global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
+// Shared memory of the pack: one mbarrier per stage of every warp, the zero
+// row, then the warps' rings of row stages.
+__host__ __device__ inline size_t pack_bar_bytes(int warps, int stages)
 {
-    extern __shared__ __align__(128) unsigned char smem[];
+    return (size_t(warps) * stages * sizeof(uint64_t) + 127) & ~size_t(127);
+}
+
+// Zero row and barriers, by the first `nthreads` threads of the block (the
+// caller then synchronises them).
+__device__ __forceinline__ void pack_init(const PackArgs &p, unsigned char *smem, int pack_warps,
+                                          int nthreads)
+{
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int PACK_WARPS = blockDim.x >> 5;
     const int NS = p.stages;
-    const uint32_t rb = p.rowbytes;
-
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
-    unsigned char *zero = smem + ((PACK_WARPS * NS * sizeof(uint64_t) + 127) & ~size_t(127));
-    unsigned char *bufs = zero + rb;
-
-    for (uint32_t i = threadIdx.x; i < rb / 16; i += blockDim.x)
+    unsigned char *zero = smem + pack_bar_bytes(pack_warps, NS);
+    for (uint32_t i = threadIdx.x; i < p.rowbytes / 16; i += nthreads)
         reinterpret_cast<uint4 *>(zero)[i] = make_uint4(0, 0, 0, 0);
-    if (lane == 0)
+    if (lane == 0 && warp < pack_warps)
         for (int s = 0; s < NS; ++s) mbar_init(&bars[warp * NS + s], 1);
     fence_init_and_proxy();
-    __syncthreads();
+}
+
+// One pack warp (warp of PACK_WARPS per block) after pack_init.
+// EP: rows and tails go to the destination GPUs' receive pools (peer stores).
+// HDR: the pack writes the slot headers (kept: the expert; empty tail: -1);
+// without it (fused with the bucketing) the assignment pass has written the
+// kept slots' headers and the bucketing writes the empty ones.
+template <int LAG, bool EP, bool HDR>
+__device__ __forceinline__ void pack_warp(const PackArgs &p, unsigned char *smem, int warp,
+                                          int lane, int PACK_WARPS)
+{
+    const int NS = p.stages;
+    const uint32_t rb = p.rowbytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+    unsigned char *zero = smem + pack_bar_bytes(PACK_WARPS, NS);
+    unsigned char *bufs = zero + rb;
 
     const uint64_t pol_x = policy_evict_first();
 #if MOE_PW_PACK_STORE_EVICT_FIRST
@@ -138,7 +156,7 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
     int32_t nslot = -1, nexp = -1;
     if (n > 0 && lane < k) {
         nslot = p.slot_map[t0 * k + lane];
-        nexp = p.idx[t0 * k + lane];
+        if (HDR) nexp = p.idx[t0 * k + lane];
     }
     bool ok = true;
     for (int64_t i = 0; i < n; ++i) {
@@ -146,7 +164,7 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
         if (i + 1 < n && lane < k) {
             const int64_t tn = t0 + (i + 1) * tstride;
             nslot = p.slot_map[tn * k + lane];
-            nexp = p.idx[tn * k + lane];
+            if (HDR) nexp = p.idx[tn * k + lane];
         }
         const int s = int(i % NS);
         const uint32_t parity = uint32_t((i / NS) & 1);
@@ -176,7 +194,7 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
                 }
             } else {
                 bulk_s2g(p.pool_x + int64_t(slot) * D, buf + size_t(s) * rb, rb, pol_pool);
-                p.pool_hdr[slot] = e;
+                if (HDR) p.pool_hdr[slot] = e;
             }
         }
         bulk_commit();
@@ -218,7 +236,7 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
         for (int64_t c = filled + lane; c < p.C_s; c += 32) {
             const int64_t slot = q * p.C_s + c;
             bulk_s2g(p.pool_x + slot * D, zero, rb, pol_pool);
-            p.pool_hdr[slot] = -1;
+            if (HDR) p.pool_hdr[slot] = -1;
         }
         bulk_commit();
         bulk_wait_read<8>();
@@ -227,7 +245,8 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
         uint4 *tail = reinterpret_cast<uint4 *>(p.pool_x + (q * p.C_s + filled) * D);
         const int64_t n16 = (p.C_s - filled) * (rb / 16);
         for (int64_t i = lane; i < n16; i += 32) __stcs(tail + i, make_uint4(0, 0, 0, 0));
-        for (int64_t c = filled + lane; c < p.C_s; c += 32) p.pool_hdr[q * p.C_s + c] = -1;
+        if (HDR)
+            for (int64_t c = filled + lane; c < p.C_s; c += 32) p.pool_hdr[q * p.C_s + c] = -1;
 #endif
     }
     bulk_wait_all();
@@ -239,23 +258,73 @@ __global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
     }
 }
 
+template <int LAG, bool EP>
+__global__ void __launch_bounds__(MAX_PACK_WARPS * 32) pack_kernel(PackArgs p)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int PACK_WARPS = blockDim.x >> 5;
+    pack_init(p, smem, PACK_WARPS, blockDim.x);
+    __syncthreads();
+    pack_warp<LAG, EP, true>(p, smem, threadIdx.x >> 5, threadIdx.x & 31, PACK_WARPS);
+}
+
+// Pack and receiver bucketing in one launch (one GPU, pooled mode).  The
+// bucketing needs only the occupancies and the kept slots' headers, which
+// the assignment pass has written, so it does not wait for the rows: warp 0
+// of every block runs the pack pipeline (the HBM-bound copy, which leaves
+// the SM's issue slots nearly idle), and the block's other BKF_THREADS
+// threads take bucket items (d, w) blockIdx.x, blockIdx.x + gridDim.x, ...
+// meanwhile.  The two roles write disjoint words: the pack the rows, the
+// bucketing recv_row, bucket_slot, the counts and the empty slots' headers.
+constexpr int BKF_THREADS = 128;
+constexpr int BKF_BAR = 1;  // named barrier of the bucketing threads
+
+template <int LAG>
+__global__ void __launch_bounds__(32 + BKF_THREADS) pack_bucket_kernel(PackArgs p, BucketArgs b,
+                                                                      uint32_t bucket_off)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    pack_init(p, smem, 1, blockDim.x);
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        pack_warp<LAG, false, false>(p, smem, 0, threadIdx.x, 1);
+        return;
+    }
+    int32_t *bsm = reinterpret_cast<int32_t *>(smem + bucket_off);
+    const int items = b.g.Rn * b.g.W;
+    for (int dw = blockIdx.x; dw < items; dw += gridDim.x)
+        bucket_item<BKF_THREADS, BKF_BAR, true>(b, dw, int(threadIdx.x) - 32, bsm);
+}
+
+// Blocks of a persistent launch: one wave of resident blocks, no more than
+// `need`.
+template <typename Kern>
+cudaError_t persistent_blocks(Kern kern, int threads, size_t smem, const DevInfo &di,
+                              int64_t need, int64_t *blocks)
+{
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (err != cudaSuccess) return err;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) per_sm = 1;
+    int64_t n = int64_t(di.sms) * per_sm;
+    if (n > need) n = need;
+    if (n < 1) n = 1;
+    *blocks = n;
+    return cudaSuccess;
+}
+
 template <int LAGT, bool EP>
 cudaError_t launch_lag(const PackArgs &p, const DevInfo &di, const Geo &g, int nw, size_t smem,
                        cudaStream_t st)
 {
-    cudaError_t err = cudaFuncSetAttribute(pack_kernel<LAGT, EP>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (err != cudaSuccess) return err;
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pack_kernel<LAGT, EP>, nw * 32,
-                                                        smem);
-    if (err != cudaSuccess) return err;
-    if (per_sm < 1) per_sm = 1;
-    int64_t blocks = int64_t(di.sms) * per_sm;
     const int64_t units = (g.T > g.n_pools ? g.T : g.n_pools);
-    const int64_t need = (units + nw - 1) / nw;
-    if (blocks > need) blocks = need;
-    if (blocks < 1) blocks = 1;
+    int64_t blocks = 0;
+    cudaError_t err =
+        persistent_blocks(pack_kernel<LAGT, EP>, nw * 32, smem, di, (units + nw - 1) / nw, &blocks);
+    if (err != cudaSuccess) return err;
     // the zero-fill phase's pool counter starts at 0 for every launch
     if ((err = cudaMemsetAsync(&p.ctr->work, 0, sizeof(int32_t), st)) != cudaSuccess) return err;
     pack_kernel<LAGT, EP><<<unsigned(blocks), nw * 32, smem, st>>>(p);
@@ -272,16 +341,24 @@ cudaError_t launch_ep(const PackArgs &p, const DevInfo &di, const Geo &g, int nw
     return launch_lag<2, EP>(p, di, g, nw, smem, st);
 }
 
-}  // namespace
-
-cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
-                        const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
-                        int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st,
-                        const EpRows *ep, uint32_t wave_mask)
+template <int LAGT>
+cudaError_t launch_fused_lag(const PackArgs &p, const BucketArgs &b, uint32_t bucket_off,
+                             const DevInfo &di, const Geo &g, size_t smem, cudaStream_t st)
 {
-    if (g.T == 0 && g.n_pools == 0) return cudaSuccess;
-    DevInfo di;
-    if (dev_info(&di) != 0) return cudaErrorUnknown;
+    const int64_t units = (g.T > g.n_pools ? g.T : g.n_pools);
+    int64_t blocks = 0;
+    cudaError_t err =
+        persistent_blocks(pack_bucket_kernel<LAGT>, 32 + BKF_THREADS, smem, di, units, &blocks);
+    if (err != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(&p.ctr->work, 0, sizeof(int32_t), st)) != cudaSuccess) return err;
+    pack_bucket_kernel<LAGT><<<unsigned(blocks), 32 + BKF_THREADS, smem, st>>>(p, b, bucket_off);
+    return cudaGetLastError();
+}
+
+PackArgs pack_args(const Geo &g, const uint16_t *x, const int32_t *idx, const int32_t *slot_map,
+                   const int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr, moe_pw_counters *ctr,
+                   const EpRows *ep, uint32_t wave_mask)
+{
     PackArgs p;
     p.x = x;
     p.idx = idx;
@@ -297,28 +374,90 @@ cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
     p.k = g.k;
     p.D = g.D;
     p.rowbytes = uint32_t(g.D) * 2u;
+    p.stages = 0;
     p.geo = g;
     p.wave_mask = wave_mask;
     if (ep) p.ep = *ep;
     else std::memset(&p.ep, 0, sizeof(p.ep));
+    return p;
+}
 
-    // warps and stages per warp: as many rows as fit next to the zero row,
-    // MIN_STAGES .. MOE_PW_PACK_MAX_STAGES, dropping warps for very wide rows
-    const size_t budget = size_t(di.smem_optin) - 1024 - p.rowbytes;
-    constexpr int MIN_STAGES = 4;
-    int nw = MAX_PACK_WARPS;
-    while (nw > 1 && budget / (size_t(nw) * p.rowbytes) < size_t(MIN_STAGES)) --nw;
-    int stages = int(budget / (size_t(nw) * p.rowbytes));
+constexpr int MIN_STAGES = 4;
+
+// Warps and stages per warp: as many rows as fit next to the zero row and
+// `extra` bytes of other shared memory, MIN_STAGES .. MOE_PW_PACK_MAX_STAGES,
+// dropping warps for very wide rows.  Returns false if even one warp's
+// MIN_STAGES do not fit.
+bool ring_shape(const DevInfo &di, uint32_t rowbytes, int max_warps, size_t extra, int *nw_out,
+                int *stages_out)
+{
+    const size_t fixed = size_t(1024) + rowbytes + extra;
+    if (size_t(di.smem_optin) < fixed) return false;
+    const size_t budget = size_t(di.smem_optin) - fixed;
+    int nw = max_warps;
+    while (nw > 1 && budget / (size_t(nw) * rowbytes) < size_t(MIN_STAGES)) --nw;
+    int stages = int(budget / (size_t(nw) * rowbytes));
     if (stages > MOE_PW_PACK_MAX_STAGES) stages = MOE_PW_PACK_MAX_STAGES;
-    if (stages < MIN_STAGES) return cudaErrorInvalidValue;
+    if (stages < MIN_STAGES) return false;
+    *nw_out = nw;
+    *stages_out = stages;
+    return true;
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const Geo &g, const uint16_t *x, const int32_t *idx,
+                        const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
+                        int32_t *pool_hdr, moe_pw_counters *ctr, cudaStream_t st,
+                        const EpRows *ep, uint32_t wave_mask)
+{
+    if (g.T == 0 && g.n_pools == 0) return cudaSuccess;
+    DevInfo di;
+    if (dev_info(&di) != 0) return cudaErrorUnknown;
+    PackArgs p = pack_args(g, x, idx, slot_map, occ, pool_x, pool_hdr, ctr, ep, wave_mask);
+    int nw = 0, stages = 0;
+    if (!ring_shape(di, p.rowbytes, MAX_PACK_WARPS, 0, &nw, &stages)) return cudaErrorInvalidValue;
     p.stages = stages;
-    const int PACK_WARPS = nw;
-    const size_t bar_bytes = (PACK_WARPS * stages * sizeof(uint64_t) + 127) & ~size_t(127);
-    const size_t smem = bar_bytes + p.rowbytes + size_t(PACK_WARPS) * stages * p.rowbytes;
+    const size_t smem = pack_bar_bytes(nw, stages) + p.rowbytes + size_t(nw) * stages * p.rowbytes;
     // the deepest store lag (<= LAG) that leaves two stages for loads
     const int lag_cap = stages - 2 < LAG ? stages - 2 : LAG;
     return ep ? launch_ep<true>(p, di, g, nw, smem, lag_cap, st)
               : launch_ep<false>(p, di, g, nw, smem, lag_cap, st);
+}
+
+cudaError_t launch_pack_bucket(const Geo &g, const uint16_t *x, const int32_t *idx,
+                               const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
+                               int32_t *pool_hdr, int32_t *recv_row, int32_t *bucket_slot,
+                               int32_t *expert_counts, moe_pw_counters *ctr, cudaStream_t st)
+{
+    if (g.mode != MOE_PW_POOLED || g.ep_n != 1 || g.T == 0) return cudaErrorInvalidValue;
+    DevInfo di;
+    if (dev_info(&di) != 0) return cudaErrorUnknown;
+    PackArgs p = pack_args(g, x, idx, slot_map, occ, pool_x, pool_hdr, ctr, nullptr, ~0u);
+    const size_t bucket_bytes = (bucket_smem_bytes(BKF_THREADS, g.P) + 127) & ~size_t(127);
+    int nw = 0, stages = 0;
+    if (!ring_shape(di, p.rowbytes, 1, bucket_bytes, &nw, &stages)) return cudaErrorInvalidValue;
+    p.stages = stages;
+    const size_t pack_bytes = pack_bar_bytes(1, stages) + p.rowbytes + size_t(stages) * p.rowbytes;
+    const uint32_t bucket_off = uint32_t((pack_bytes + 127) & ~size_t(127));
+    const size_t smem = bucket_off + bucket_bytes;
+
+    BucketArgs b;
+    b.pool_hdr = pool_hdr;
+    b.occ = occ;
+    b.recv_row = recv_row;
+    b.bucket_slot = bucket_slot;
+    b.expert_counts = expert_counts;
+    b.ctr = ctr;
+    b.g = g;
+    b.wave_mask = ~0u;
+    b.hdr_out = pool_hdr;
+
+    const int lag_cap = stages - 2 < LAG ? stages - 2 : LAG;
+    if (lag_cap >= 12 && LAG >= 12) return launch_fused_lag<12>(p, b, bucket_off, di, g, smem, st);
+    if (lag_cap >= 8) return launch_fused_lag<8>(p, b, bucket_off, di, g, smem, st);
+    if (lag_cap >= 4) return launch_fused_lag<4>(p, b, bucket_off, di, g, smem, st);
+    return launch_fused_lag<2>(p, b, bucket_off, di, g, smem, st);
 }
 
 }  // namespace moe_pw

@@ -102,6 +102,8 @@ SIGNATURES = {
     "moe_pw_assign_noalloc": [_CFG, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_pack": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_bucket": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_assign_headers": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "moe_pw_pack_bucket": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_dispatch": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_expert": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_combine": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
@@ -256,6 +258,27 @@ def moe_pw_bucket(cfg, pool_hdr, occ, recv_row, bucket_slot, expert_counts, coun
     _check("moe_pw_bucket", load_library().moe_pw_bucket(
         ctypes.byref(c), _ptr(pool_hdr), _ptr(occ), _ptr(recv_row), _ptr(bucket_slot),
         _ptr(expert_counts), _ptr(counters), _stream(stream)))
+
+
+def moe_pw_assign_headers(cfg, idx, slot_map, occ, pool_hdr, counters, workspace,
+                          workspace_bytes=None, stream=None):
+    """moe_pw_assign that also writes the kept slots' headers (pooled mode)."""
+    c = _cfg(cfg)
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check("moe_pw_assign_headers", load_library().moe_pw_assign_headers(
+        ctypes.byref(c), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(pool_hdr), _ptr(counters),
+        _ptr(workspace), wsb, _stream(stream)))
+
+
+def moe_pw_pack_bucket(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, recv_row, bucket_slot,
+                       expert_counts, counters, stream=None):
+    """Pack and receiver bucketing in one launch; pool_hdr must hold the
+    kept slots' headers from moe_pw_assign_headers."""
+    c = _cfg(cfg)
+    _check("moe_pw_pack_bucket", load_library().moe_pw_pack_bucket(
+        ctypes.byref(c), _ptr(x), _ptr(idx), _ptr(slot_map), _ptr(occ), _ptr(pool_x),
+        _ptr(pool_hdr), _ptr(recv_row), _ptr(bucket_slot), _ptr(expert_counts), _ptr(counters),
+        _stream(stream)))
 
 
 def moe_pw_dispatch(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, recv_row, bucket_slot,
@@ -538,6 +561,15 @@ class Buffers:
         moe_pw_assign(self.cfg, self.idx, self.slot_map, self.occ, self.counters, self.workspace,
                       stream=stream)
 
+    def assign_headers(self, stream=None):
+        moe_pw_assign_headers(self.cfg, self.idx, self.slot_map, self.occ, self.pool_hdr,
+                              self.counters, self.workspace, stream=stream)
+
+    def pack_bucket(self, stream=None):
+        moe_pw_pack_bucket(self.cfg, self.x, self.idx, self.slot_map, self.occ, self.pool_x,
+                           self.pool_hdr, self.recv_row, self.bucket_slot, self.expert_counts,
+                           self.counters, stream)
+
     def pack(self, stream=None):
         moe_pw_pack(self.cfg, self.x, self.idx, self.slot_map, self.occ, self.pool_x,
                     self.pool_hdr, self.counters, stream)
@@ -683,7 +715,8 @@ class Buffers:
                 s0.wait_event(ev)
 
     def run_step(self, stream=None):
-        """route -> dispatch (assign, pack, bucket) -> expert -> combine."""
+        """route -> dispatch (assign, pack, bucket; pooled mode: the pack and
+        the bucketing in one launch) -> expert -> combine."""
         self.route(stream)
         self.dispatch(stream)
         self.expert(stream)

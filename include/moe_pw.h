@@ -259,7 +259,39 @@ int moe_pw_bucket(const moe_pw_config *cfg, const int32_t *pool_hdr, const int32
 int moe_pw_assign_noalloc(const moe_pw_config *cfg, const int32_t *idx, int32_t *slot_map,
                           int32_t *occ, moe_pw_counters *counters, cudaStream_t stream);
 
-/* moe_pw_assign, moe_pw_pack and moe_pw_bucket in one call. */
+/*
+ * moe_pw_assign that also writes the header (the expert id) of every slot the
+ * sender kept into pool_hdr [n_slots]; the other headers are left as they
+ * are.  Pooled mode only (MOE_PW_EUNSUPPORTED otherwise).  The first half of
+ * the fused dispatch: moe_pw_pack_bucket then needs no headers from the pack.
+ */
+int moe_pw_assign_headers(const moe_pw_config *cfg, const int32_t *idx, int32_t *slot_map,
+                          int32_t *occ, int32_t *pool_hdr, moe_pw_counters *counters,
+                          void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * moe_pw_pack and moe_pw_bucket in one launch (pooled mode, one GPU).  The
+ * bucketing reads only the occupancies and the kept slots' headers, so it
+ * runs beside the row copies instead of after them: the pack's copy warp of
+ * every block drives the TMA engine while the block's other warps bucket the
+ * (destination, wave) items.  Precondition: pool_hdr holds the kept slots'
+ * headers of this batch, written by moe_pw_assign_headers with the same
+ * idx, slot_map and occ (the pack writes no headers here).  Writes pool_x
+ * (kept rows; zero rows in the empty tails), the empty slots' headers (-1),
+ * recv_row, bucket_slot and expert_counts, and adds receiver drops and kept
+ * rows to *counters: every output equals moe_pw_pack followed by
+ * moe_pw_bucket.  Ragged mode: MOE_PW_EUNSUPPORTED.  T = 0: the two calls
+ * are made one after the other.  Uses counters->work like moe_pw_pack.
+ */
+int moe_pw_pack_bucket(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
+                       const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
+                       int32_t *pool_hdr, int32_t *recv_row, int32_t *bucket_slot,
+                       int32_t *expert_counts, moe_pw_counters *counters, cudaStream_t stream);
+
+/*
+ * moe_pw_assign, moe_pw_pack and moe_pw_bucket in one call.  Pooled mode:
+ * moe_pw_assign_headers then moe_pw_pack_bucket (same outputs).
+ */
 int moe_pw_dispatch(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
                     int32_t *slot_map, int32_t *occ, uint16_t *pool_x, int32_t *pool_hdr,
                     int32_t *recv_row, int32_t *bucket_slot, int32_t *expert_counts,

@@ -140,3 +140,31 @@ def test_workspace_follows_the_chunk_rule(lib, k, chunks_per_source):
     bins = cfg.R * cfg.W
     pad = lambda b: (b + 255) // 256 * 256
     assert s.workspace_bytes == pad(4 * cfg.R * chunks_per_source * bins) + pad(4 * cfg.R * bins)
+
+
+def test_fused_dispatch_entries_validate_before_any_launch(lib):
+    """The fused dispatch halves are pooled-mode calls: a ragged config is
+    refused, and so are missing or misaligned buffers, all on the host."""
+    tiny = mp.Config.from_workload(synth.WORKLOADS["tiny"])
+    ragged = mp.Config(**{**tiny.__dict__, "mode": synth.MODE_RAGGED, "cf_send_pct": 0,
+                          "cf_recv_pct": 0})
+    good, odd = 1 << 20, (1 << 20) + 4  # placeholder addresses, never dereferenced
+    ws = mp.moe_pw_plan(tiny).workspace_bytes
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_assign_headers(ragged, good, good, good, good, good, good, ws, stream=0)
+    assert ei.value.code == mp.MOE_PW_EUNSUPPORTED
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_pack_bucket(ragged, *[good] * 10, stream=0)
+    assert ei.value.code == mp.MOE_PW_EUNSUPPORTED
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_assign_headers(tiny, good, good, good, None, good, good, ws, stream=0)
+    assert ei.value.code == mp.MOE_PW_EINVAL
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_assign_headers(tiny, good, good, good, good, good, good, ws - 256, stream=0)
+    assert ei.value.code == mp.MOE_PW_EINVAL
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_pack_bucket(tiny, *[good] * 6, None, *[good] * 3, stream=0)  # no recv_row
+    assert ei.value.code == mp.MOE_PW_EINVAL
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_pack_bucket(tiny, odd + 8, *[good] * 9, stream=0)  # x needs 16 bytes
+    assert ei.value.code == mp.MOE_PW_EUNSUPPORTED

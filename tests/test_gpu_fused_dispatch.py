@@ -1,0 +1,120 @@
+"""The fused dispatch (assignment with headers, then pack and bucketing in one
+launch) against the three separate launches and the oracle.
+
+Every output buffer is poisoned before each path runs, so a word the fused
+launch fails to write shows up.  The cases cover bucket items of one and of
+several tiles (positions per (destination, wave) item above the fused
+launch's tile of 4096), more items than blocks (each block then takes
+several), one wave with 16 experts per rank, one expert per wave, heavy
+sender and receiver drops, and the pages' rank count.
+"""
+import numpy as np
+import pytest
+import torch
+
+from combine_moe_pw_b200 import moe_pw as mp
+from combine_moe_pw_b200 import synth
+from test_gpu_parity import SMALL_CASES, TINY, _inputs, check_full
+
+pytestmark = pytest.mark.gpu
+
+OUTPUTS = ["slot_map", "occ", "pool_x", "pool_hdr", "recv_row", "bucket_slot", "expert_counts"]
+
+CASES = {
+    "tiny": TINY,
+    "tiny_tight": SMALL_CASES["tiny_tight"],
+    "single_pool": SMALL_CASES["single_pool"],
+    "one_expert_per_wave": TINY.with_(W=6, P=1),
+    "wide_E": SMALL_CASES["wide_E"],
+    "E2048": SMALL_CASES["E2048"],              # 1024 items: several per block
+    "pages_ranks_small": SMALL_CASES["pages_ranks_small"],
+    # 2 sources of 10,000 tokens: ~29,000 positions per item, 8 tiles
+    "long_sources": SMALL_CASES["long_sources"],
+    "multi_tile_ragged_tail": synth.Workload("multi_tile", T=8 * 5001, R=8, L=6, W=3, P=2, k=8,
+                                             D=24, seq_len=5001,
+                                             logit_kind=synth.LOGIT_SEQBIAS),
+}
+
+
+def _fresh(w, lg, x, s):
+    b = mp.Buffers(mp.Config.from_workload(w))
+    b.logits.copy_(torch.from_numpy(lg))
+    b.x.copy_(torch.from_numpy(x.view(np.int16)))
+    b.scale.copy_(torch.from_numpy(s))
+    return b
+
+
+def _poison(b):
+    b.slot_map.fill_(-77)
+    b.occ.fill_(-77)
+    b.pool_x.fill_(0x2A2A)
+    b.pool_hdr.fill_(-55)
+    b.recv_row.fill_(-66)
+    b.bucket_slot.fill_(-88)
+    b.expert_counts.fill_(99)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_fused_equals_separate_launches(name):
+    w = CASES[name]
+    lg, x, s = _inputs(w)
+    ref = _fresh(w, lg, x, s)
+    ref.route()
+    _poison(ref)
+    ref.assign()
+    ref.pack()
+    ref.bucket()
+    st_ref = ref.stats()
+
+    b = _fresh(w, lg, x, s)
+    b.route()
+    _poison(b)
+    b.assign_headers()
+    b.pack_bucket()
+    st = b.stats()
+    torch.cuda.synchronize()
+    for n in OUTPUTS:
+        assert torch.equal(getattr(b, n), getattr(ref, n)), n
+    assert (st.kept, st.sender_dropped, st.receiver_dropped, st.error, st.max_fill) == (
+        st_ref.kept, st_ref.sender_dropped, st_ref.receiver_dropped, st_ref.error,
+        st_ref.max_fill)
+    np.testing.assert_array_equal(b.host_expert_counts, ref.host_expert_counts)
+
+
+@pytest.mark.parametrize("name", ["multi_tile_ragged_tail", "one_expert_per_wave"])
+def test_fused_step_full_parity(name):
+    """The whole step through moe_pw_dispatch (the fused path) against the
+    whole oracle, on buffers poisoned first."""
+    w = CASES[name]
+    lg, x, s = _inputs(w)
+    b = _fresh(w, lg, x, s)
+    _poison(b)
+    b.run_step()
+    st = b.stats(raise_on_device_error=False)
+    torch.cuda.synchronize()
+    check_full(w, lg, x, s, b, st)
+
+
+def test_fused_repeat_rebuilds_every_word():
+    """A second fused launch on poisoned pools (same assignment) rebuilds the
+    same bytes: headers of empty slots come from the bucketing, rows from the
+    pack's zero fill."""
+    w = TINY.with_(T=8 * 1024, seq_len=1024, D=256, logit_kind=synth.LOGIT_SEQBIAS)
+    lg, x, s = _inputs(w)
+    b = _fresh(w, lg, x, s)
+    b.run_step()
+    torch.cuda.synchronize()
+    keep = {n: getattr(b, n).clone() for n in OUTPUTS}
+    assert (keep["pool_hdr"] < 0).any()
+    for _ in range(2):
+        b.assign_headers()
+        b.pool_x.fill_(0x1357)
+        # the kept slots' headers stay (the assignment wrote them); the rest is poisoned
+        b.pool_hdr.masked_fill_(keep["pool_hdr"] < 0, -9)
+        b.recv_row.fill_(-66)
+        b.bucket_slot.fill_(-88)
+        b.pack_bucket()
+        torch.cuda.synchronize()
+        for n in OUTPUTS:
+            assert torch.equal(getattr(b, n), keep[n]), n
+    assert b.stats().error == 0
