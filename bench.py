@@ -4,12 +4,14 @@
     python bench.py --impl reference ...        # the CPU oracle as the reference arm
     torchrun --nproc-per-node N bench.py --gpus N ...
 
-One step = route -> dispatch (assign, then pack and bucketing in one launch;
-dropless ragged mode: assign, pack, bucket) -> per-expert op -> combine ->
-drop statistics, on one synthetic batch already resident in HBM.  The metric
-is routed assignments per second for dispatch + combine: T*k divided by the
-device time of route + assign + pack/bucket + combine, each timed with CUDA
-events on the launching stream inside the K timed steps (the
+One step = route -> dispatch (assign, pack, bucket) -> per-expert op ->
+combine -> drop statistics, on one synthetic batch already resident in HBM.
+Pooled mode runs route + assignment as one launch and pack + bucketing as
+one launch (--dispatch selects the split forms); dropless ragged mode runs
+route, assign, pack, bucket.  The metric is routed assignments per second for
+dispatch + combine: T*k divided by the device time of every stage but the
+expert op, each timed with CUDA events on the launching stream inside the K
+timed steps (the
 per-expert op runs in every step but is timed apart, since it stands in for
 the expert network).  HBM GB/s and the fraction of the measured copy peak use
 the algorithmic bytes of those stages.
@@ -49,9 +51,10 @@ def parse():
     ap.add_argument("--workload", default="rack")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--separate-dispatch", action="store_true",
-                    help="pooled mode: pack and bucketing as two launches (the fused launch "
-                         "is the default)")
+    ap.add_argument("--dispatch", default="fused", choices=["fused", "split-route", "separate"],
+                    help="pooled mode: fused = route+assignment and pack+bucketing as two "
+                         "launches; split-route = route, assignment, pack+bucketing; separate = "
+                         "route, assignment, pack, bucketing")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
     ap.add_argument("--cpu-sample-sources", type=int, default=16)
@@ -262,8 +265,11 @@ def alg_bytes(w, stats, C_s):
     # and the empty slots' headers, and buckets
     assign_headers = assign + 4 * K_s
     pack_bucket = 2 * T * D + 4 * T * k + S * 2 * D + 4 * (S - K_s) + bucket
+    # route + assignment in one launch: the ids stay on chip for the ranking
+    route_assign = route + 4 * T * k + 4 * K_s
     return {"route": route, "assign": assign, "pack": pack, "bucket": bucket, "combine": combine,
             "assign_headers": assign_headers, "pack_bucket": pack_bucket,
+            "route_assign": route_assign,
             "expert": 2 * D * K + 8 * S + S * (2 * D + 4)}
 
 
@@ -654,14 +660,17 @@ def main():
             print(json.dumps({"projection": proj}), flush=True)
         return
 
-    fused = w.mode == 0 and not a.separate_dispatch
-    if fused:
+    mode = a.dispatch if w.mode == 0 else "separate"
+    if mode == "fused":
+        stages = ["route_assign", "pack_bucket", "expert", "combine"]
+        calls = [b.route_assign, b.pack_bucket, b.expert, b.combine]
+    elif mode == "split-route":
         stages = ["route", "assign_headers", "pack_bucket", "expert", "combine"]
-        dispatch_calls = [b.assign_headers, b.pack_bucket]
+        calls = [b.route, b.assign_headers, b.pack_bucket, b.expert, b.combine]
     else:
         stages = ["route", "assign", "pack", "bucket", "expert", "combine"]
-        dispatch_calls = [b.assign, b.pack, b.bucket]
-    calls = [b.route, *dispatch_calls, b.expert, b.combine]
+        calls = [b.route, b.assign, b.pack, b.bucket, b.expert, b.combine]
+    fused = mode != "separate"
 
     def step(evs=None):
         for i, f in enumerate(calls):
@@ -678,13 +687,19 @@ def main():
     for _ in range(max(a.warmup, 3)):
         step()
     st = b.stats(stream)
-    # kernels of ours per step: route; assignment count (+ scan when a source
+    # kernels of ours per step.  fused: route + assignment (one clustered
+    # launch up to 1,024 tokens per SM, else route and the assignment
+    # passes), pack + bucketing, expert, combine.
+    # split-route / separate: route; assignment count (+ scan when a source
     # has more than 32 chunks of 2048 assignments, + row offsets in ragged
-    # mode) and rank; pack; bucket; expert; combine
+    # mode) and rank; pack + bucketing, or pack and bucketing; expert; combine
     chunk_tokens = min(max(2048 // w.k, 1), w.T // w.R if w.mode == 0 else w.T)
     chunks_per_source = -(-(w.T // w.R) // chunk_tokens)
     assign_kernels = (2 if chunks_per_source <= 32 else 3) if w.mode == 0 else 4
-    launches_per_step = (4 if fused else 5) + assign_kernels
+    one_launch = mode == "fused" and mp.moe_pw_route_assign_plan(cfg)
+    launches_per_step = {"fused": 4 if one_launch else 4 + assign_kernels,
+                         "split-route": 4 + assign_kernels,
+                         "separate": 5 + assign_kernels}[mode]
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
            for _ in range(a.steps)]

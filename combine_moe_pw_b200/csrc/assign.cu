@@ -46,11 +46,6 @@ struct RankArgs {
     int32_t *pool_hdr;   // optional: the kept slots' headers (the expert id)
 };
 
-__device__ __forceinline__ int32_t bin_of_expert(const Geo &g, int32_t e)
-{
-    return g.mode == MOE_PW_POOLED ? (e / g.L) * g.W + (e % g.L) / g.P : e;
-}
-
 // Flat assignment range [a0, a1) of this block's chunk and its group.
 __device__ __forceinline__ void chunk_range(const Geo &g, int chunk, int64_t &a0, int64_t &a1,
                                             int &group)
@@ -121,19 +116,6 @@ __device__ __forceinline__ void warp_hist(const RankArgs &p, const Smem &s, int 
         const int32_t b = s.bins[i];
         if (b >= 0) atomicAdd(&h[b], 1);
     }
-}
-
-// Lanes of the warp holding the same key as this lane (key in [0, 2^nbits)):
-// one ballot per key bit.  All lanes call it with the same nbits.
-__device__ __forceinline__ unsigned equal_lanes(uint32_t key, int nbits)
-{
-    unsigned m = FULL_MASK;
-    for (int i = 0; i < nbits; ++i) {
-        const bool bit = (key >> i) & 1u;
-        const unsigned bal = __ballot_sync(FULL_MASK, bit);
-        m &= bit ? bal : ~bal;
-    }
-    return m;
 }
 
 __device__ __forceinline__ void setup(const RankArgs &p, const Smem &s)

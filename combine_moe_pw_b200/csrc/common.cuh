@@ -50,6 +50,17 @@ int dev_info(DevInfo *out);
 // Kernel launchers (asynchronous; return cudaError_t of the launch).
 cudaError_t launch_route(const Geo &g, const float *logits, int32_t *idx, float *gates,
                          cudaStream_t st);
+// Route and sender assignment (with the kept slots' headers) in one launch,
+// pooled mode on one GPU; zeroes *ctr first.  cudaErrorNotSupported (nothing
+// enqueued) when the batch's shape does not fit the launch or the batch is
+// large enough for the separate kernels to be faster: the caller then runs
+// launch_route and launch_assign.
+cudaError_t launch_route_assign(const Geo &g, const float *logits, int32_t *idx, float *gates,
+                                int32_t *slot_map, int32_t *occ, int32_t *pool_hdr,
+                                moe_pw_counters *ctr, cudaStream_t st);
+// Whether launch_route_assign takes the one launch for this batch on the
+// current device (*one_launch 1) or returns cudaErrorNotSupported (0).
+cudaError_t route_assign_plan(const Geo &g, int *one_launch);
 // pool_hdr (optional): also write the kept slots' headers (the expert id),
 // as the fused pack + bucketing launch expects.
 cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, int32_t *occ,
@@ -262,6 +273,26 @@ __device__ __forceinline__ uint32_t ep_recv_to_send(const Geo &g, uint32_t rq, i
 __device__ __forceinline__ void set_error(moe_pw_counters *ctr, int bits)
 {
     atomicOr(&ctr->error, bits);
+}
+
+// Ranking bin of expert e: pooled, the pool (d, w) of its rank and wave
+// within a source, (e / L) * W + (e % L) / P; ragged, the expert itself.
+__device__ __forceinline__ int32_t bin_of_expert(const Geo &g, int32_t e)
+{
+    return g.mode == MOE_PW_POOLED ? (e / g.L) * g.W + (e % g.L) / g.P : e;
+}
+
+// Lanes of the warp holding the same key as this lane (key in [0, 2^nbits)):
+// one ballot per key bit.  All lanes call it with the same nbits.
+__device__ __forceinline__ unsigned equal_lanes(uint32_t key, int nbits)
+{
+    unsigned m = FULL_MASK;
+    for (int i = 0; i < nbits; ++i) {
+        const bool bit = (key >> i) & 1u;
+        const unsigned bal = __ballot_sync(FULL_MASK, bit);
+        m &= bit ? bal : ~bal;
+    }
+    return m;
 }
 
 __device__ __forceinline__ unsigned lanemask_lt()

@@ -269,6 +269,47 @@ int moe_pw_assign_headers(const moe_pw_config *cfg, const int32_t *idx, int32_t 
     return cuda_rc(launch_assign(g, idx, slot_map, occ, counters, workspace, stream, pool_hdr));
 }
 
+int moe_pw_route_assign(const moe_pw_config *cfg, const float *logits, int32_t *idx,
+                        float *gates, int32_t *slot_map, int32_t *occ, int32_t *pool_hdr,
+                        moe_pw_counters *counters, void *workspace, size_t workspace_bytes,
+                        cudaStream_t stream)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (g.mode != MOE_PW_POOLED || g.E % 4 != 0) return MOE_PW_EUNSUPPORTED;
+    if (!counters || !occ) return MOE_PW_EINVAL;
+    if (g.T > 0 && (!logits || !idx || !gates || !slot_map || !pool_hdr || !workspace))
+        return MOE_PW_EINVAL;
+    if (g.T > 0 && int64_t(workspace_bytes) < ws_bytes(g)) return MOE_PW_EINVAL;
+    if (!aligned(counters, 8) || !aligned(occ, 4) ||
+        (g.T > 0 && (!aligned(logits, 16) || !aligned(idx, 4) || !aligned(gates, 4) ||
+                     !aligned(slot_map, 4) || !aligned(pool_hdr, 4) ||
+                     !aligned(workspace, 256))))
+        return MOE_PW_EUNSUPPORTED;
+    if (g.T > 0) {
+        const cudaError_t e =
+            launch_route_assign(g, logits, idx, gates, slot_map, occ, pool_hdr, counters, stream);
+        if (e != cudaErrorNotSupported) return cuda_rc(e);
+    }
+    rc = moe_pw_route(cfg, logits, idx, gates, stream);
+    if (rc != MOE_PW_OK) return rc;
+    return moe_pw_assign_headers(cfg, idx, slot_map, occ, pool_hdr, counters, workspace,
+                                 workspace_bytes, stream);
+}
+
+int moe_pw_route_assign_plan(const moe_pw_config *cfg, int32_t *one_launch)
+{
+    Geo g;
+    int rc = make_geo(cfg, &g);
+    if (rc != MOE_PW_OK) return rc;
+    if (!one_launch) return MOE_PW_EINVAL;
+    int one = 0;
+    const cudaError_t e = route_assign_plan(g, &one);
+    *one_launch = one;
+    return cuda_rc(e);
+}
+
 int moe_pw_pack_bucket(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
                        const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,
                        int32_t *pool_hdr, int32_t *recv_row, int32_t *bucket_slot,
@@ -673,13 +714,24 @@ extern "C" int moe_pw_step_host(const moe_pw_config *cfg, const float *h_logits,
         return MOE_PW_ECUDA;
     if (order(copy_in, compute) != cudaSuccess) return MOE_PW_ECUDA;
     // the path, every step in this library's kernels
-    if ((rc = moe_pw_route(cfg, dev->logits, dev->idx, dev->gates, compute)) != MOE_PW_OK)
-        return rc;
-    if ((rc = moe_pw_dispatch(cfg, dev->x, dev->idx, dev->slot_map, dev->occ, dev->pool_x,
-                              dev->pool_hdr, dev->recv_row, dev->bucket_slot, dev->expert_counts,
-                              dev->counters, dev->workspace, dev->workspace_bytes, compute)) !=
-        MOE_PW_OK)
-        return rc;
+    if (g.mode == MOE_PW_POOLED) {
+        if ((rc = moe_pw_route_assign(cfg, dev->logits, dev->idx, dev->gates, dev->slot_map,
+                                      dev->occ, dev->pool_hdr, dev->counters, dev->workspace,
+                                      dev->workspace_bytes, compute)) != MOE_PW_OK)
+            return rc;
+        if ((rc = moe_pw_pack_bucket(cfg, dev->x, dev->idx, dev->slot_map, dev->occ, dev->pool_x,
+                                     dev->pool_hdr, dev->recv_row, dev->bucket_slot,
+                                     dev->expert_counts, dev->counters, compute)) != MOE_PW_OK)
+            return rc;
+    } else {
+        if ((rc = moe_pw_route(cfg, dev->logits, dev->idx, dev->gates, compute)) != MOE_PW_OK)
+            return rc;
+        if ((rc = moe_pw_dispatch(cfg, dev->x, dev->idx, dev->slot_map, dev->occ, dev->pool_x,
+                                  dev->pool_hdr, dev->recv_row, dev->bucket_slot,
+                                  dev->expert_counts, dev->counters, dev->workspace,
+                                  dev->workspace_bytes, compute)) != MOE_PW_OK)
+            return rc;
+    }
     if ((rc = moe_pw_expert(cfg, dev->pool_x, dev->pool_hdr, dev->recv_row, dev->scale,
                             dev->ret_x, dev->ret_hdr, compute)) != MOE_PW_OK)
         return rc;

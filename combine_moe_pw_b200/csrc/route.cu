@@ -1,58 +1,19 @@
 // route.cu - top-k expert selection and softmax gates, one warp per token.
 //
 // "Marin 开始公开训练 535B 参数 MoE 模型", section 二: the router picks 8 of the
-// 384 routed experts for every token.  Order (logit descending, expert id
-// ascending) and softmax gates over the chosen logits are this library's
-// reading.
-//
-// Layout: lane l holds float4 number l + 32*v of the row (v < NV), i.e. the
-// logits of experts 4*(l + 32*v) + c.  Each logit becomes an order-preserving
-// unsigned key (0 marks "taken or absent").  For ranking, a candidate carries
-// the compound 64-bit key (logit key, ~expert id), so one unsigned comparison
-// orders by logit descending, then id ascending.
-// Selection: tau = the k-th largest of the 32 lane maxima bounds the top k
-// from below; the logits >= tau (typically ~k of them) are compacted into
-// shared memory and ranked exactly by (key descending, id ascending).  When
-// more than 32 logits pass (many equal values), k exact rounds run instead:
-// a warp-wide max of the keys (redux.sync), then a warp-wide min of the ids
-// holding it.  The next token's row is loaded while the current one is
+// 384 routed experts for every token.  The selection itself is in
+// route_body.cuh.  The next token's row is loaded while the current one is
 // being selected.
 // The kernel is issue-bound (a few hundred warp instructions per token), so
 // the common shapes are compiled with k = 8 and E = 128*NV fixed, and the
 // grid is one wave of resident blocks at 64 registers (4 blocks per SM):
 // on B200 that measured 17% faster than the same selection with run-time k
 // and 60 registers over two waves.
-#include "common.cuh"
+#include "route_body.cuh"
 
 namespace moe_pw {
 
 namespace {
-
-// Order-preserving map float -> uint32; -0.0 is folded onto +0.0 first, so
-// the two compare equal as floats do.  Finite floats map to keys >=
-// 0x007FFFFF, so 0 never collides with a logit.
-__device__ __forceinline__ uint32_t order_key(float f)
-{
-    const uint32_t u = __float_as_uint(f + 0.0f);  // -0.0 + 0.0 = +0.0
-    return u ^ (uint32_t(int32_t(u) >> 31) | 0x80000000u);
-}
-
-__device__ __forceinline__ float key_value(uint32_t key)
-{
-    return __uint_as_float(key ^ ((key & 0x80000000u) ? 0x80000000u : 0xFFFFFFFFu));
-}
-
-template <int NV, bool FULL>
-__device__ __forceinline__ void load_row(const float *__restrict__ logits, int64_t t, int E4,
-                                         int lane, float4 (&f)[NV])
-{
-    const float4 *row = reinterpret_cast<const float4 *>(logits) + t * E4;
-#pragma unroll
-    for (int v = 0; v < NV; ++v) {
-        const int q = lane + 32 * v;
-        if (FULL || q < E4) f[v] = __ldcs(row + q);
-    }
-}
 
 constexpr int ROUTE_WARPS = 8;
 constexpr int ROUTE_MIN_BLOCKS = 4;  // caps registers at 64
@@ -73,139 +34,22 @@ route_kernel(const float *__restrict__ logits, int32_t *__restrict__ idx,
     const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarp = (int64_t(gridDim.x) * blockDim.x) >> 5;
     const int E4 = E >> 2;
-    const uint32_t base = 4u * lane;
 
-    float4 cur[NV], nxt[NV];
-    if (warp < T) load_row<NV, FULL>(logits, warp, E4, lane, cur);
-
-    for (int64_t t = warp; t < T; t += nwarp) {
-        if (t + nwarp < T) load_row<NV, FULL>(logits, t + nwarp, E4, lane, nxt);
-
-        uint32_t key[NV][4];
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            const bool in = FULL || lane + 32 * v < E4;
-            key[v][0] = in ? order_key(cur[v].x) : 0u;
-            key[v][1] = in ? order_key(cur[v].y) : 0u;
-            key[v][2] = in ? order_key(cur[v].z) : 0u;
-            key[v][3] = in ? order_key(cur[v].w) : 0u;
-        }
-        uint32_t lm = 0;
-#pragma unroll
-        for (int v = 0; v < NV; ++v)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) lm = max(lm, key[v][c]);
-
-        // tau = k-th largest lane maximum: at least k logits are >= tau, so
-        // every one of the top k is >= tau.  Usually few logits pass.
-        uint32_t rem = lm, tau = 0;
-#pragma unroll
-        for (int j = 0; j < (KC ? KC : 1); ++j) {
-            tau = __reduce_max_sync(FULL_MASK, rem);
-            rem = (rem == tau) ? 0u : rem;
-        }
-        if (!KC)
-            for (int j = 1; j < k; ++j) {
-                tau = __reduce_max_sync(FULL_MASK, rem);
-                rem = (rem == tau) ? 0u : rem;
-            }
-        int cnt = 0;
-#pragma unroll
-        for (int v = 0; v < NV; ++v)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) cnt += key[v][c] >= tau;
-        const int C = tau ? int(__reduce_add_sync(FULL_MASK, unsigned(cnt))) : 1 << 30;
-
-        uint32_t sel_key = 0;
-        int32_t sel_idx = 0;
-        if (C <= 32) {
-            // compact the candidates (lane order, then element order) ...
-            int pos = cnt;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int u = __shfl_up_sync(FULL_MASK, pos, o);
-                if (lane >= o) pos += u;
-            }
-            pos -= cnt;
-#pragma unroll
-            for (int v = 0; v < NV; ++v)
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    if (key[v][c] >= tau)
-                        cand_sm[wib][pos++] = (static_cast<unsigned long long>(key[v][c]) << 32) |
-                                              ~(base + 128u * v + c);
-            if (lane >= C) cand_sm[wib][lane] = 0ull;  // ranks below every candidate
-            __syncwarp();
-            // ... and rank each one against all of them
-            const unsigned long long me = cand_sm[wib][lane];
-            int rank = 0;
-            const int C4 = (C + 3) & ~3;
-            for (int i = 0; i < C4; i += 4) {
-                rank += cand_sm[wib][i] > me;
-                rank += cand_sm[wib][i + 1] > me;
-                rank += cand_sm[wib][i + 2] > me;
-                rank += cand_sm[wib][i + 3] > me;
-            }
-            if (lane < C && rank < k) sel_sm[wib][rank] = me;
-            __syncwarp();
-            if (lane < k) {
-                const unsigned long long s = sel_sm[wib][lane];
-                sel_key = uint32_t(s >> 32);
-                sel_idx = int32_t(~uint32_t(s));
-            }
-            __syncwarp();
-        } else {
-            // many equal logits: k exact rounds over every logit
-            for (int j = 0; j < k; ++j) {
-                uint32_t mx = 0;
-#pragma unroll
-                for (int v = 0; v < NV; ++v)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) mx = max(mx, key[v][c]);
-                const uint32_t m = __reduce_max_sync(FULL_MASK, mx);
-                // lowest expert id in this lane whose key equals the maximum
-                int32_t cand = 0x7FFFFFFF;
-#pragma unroll
-                for (int v = NV - 1; v >= 0; --v)
-#pragma unroll
-                    for (int c = 3; c >= 0; --c)
-                        if (key[v][c] == m) cand = base + 128 * v + c;
-                const int32_t gi = __reduce_min_sync(FULL_MASK, cand);
-                const int32_t rel = gi - int32_t(base);  // 128*v + c only in the owning lane
-#pragma unroll
-                for (int v = 0; v < NV; ++v)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        if (rel == 128 * v + c) key[v][c] = 0u;
-                if (lane == j) {
-                    sel_key = m;
-                    sel_idx = gi;
-                }
-            }
-        }
-
-        // softmax over the chosen logits: lane j holds choice j
-        const float val = key_value(sel_key);
-        const float top = __shfl_sync(FULL_MASK, val, 0);
-        const float ex = (lane < k) ? expf(val - top) : 0.0f;
-        float sum = 0.0f;
-        if (KC == 8) {
-            // butterfly over lanes 0..7: every lane of the group ends with the
-            // same bits (each add's operands only swap places)
-            sum = ex;
-            sum += __shfl_xor_sync(FULL_MASK, sum, 1);
-            sum += __shfl_xor_sync(FULL_MASK, sum, 2);
-            sum += __shfl_xor_sync(FULL_MASK, sum, 4);
-        } else {
-#pragma unroll
-            for (int j = 0; j < (KC ? KC : 1); ++j) sum += __shfl_sync(FULL_MASK, ex, j);
-            if (!KC)
-                for (int j = 1; j < k; ++j) sum += __shfl_sync(FULL_MASK, ex, j);
-        }
+    auto one = [&](int64_t t, const float4 (&row)[NV]) {
+        int32_t sel_idx;
+        float ex, sum;
+        route_select<NV, FULL, KC, ROUTE_WARPS>(row, k, E4, lane, wib, cand_sm, sel_sm, sel_idx,
+                                                ex, sum);
         if (lane < k) {
             idx[t * k + lane] = sel_idx;
             gates[t * k + lane] = ex / sum;
         }
+    };
+    float4 cur[NV], nxt[NV];
+    if (warp < T) load_row<NV, FULL>(logits, warp, E4, lane, cur);
+    for (int64_t t = warp; t < T; t += nwarp) {
+        if (t + nwarp < T) load_row<NV, FULL>(logits, t + nwarp, E4, lane, nxt);
+        one(t, cur);
 #pragma unroll
         for (int v = 0; v < NV; ++v) cur[v] = nxt[v];
     }

@@ -102,6 +102,8 @@ SIGNATURES = {
     "moe_pw_assign_noalloc": [_CFG, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_pack": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_bucket": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_route_assign": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "moe_pw_route_assign_plan": [_CFG, ctypes.POINTER(ctypes.c_int32)],
     "moe_pw_assign_headers": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_pack_bucket": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_dispatch": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
@@ -258,6 +260,27 @@ def moe_pw_bucket(cfg, pool_hdr, occ, recv_row, bucket_slot, expert_counts, coun
     _check("moe_pw_bucket", load_library().moe_pw_bucket(
         ctypes.byref(c), _ptr(pool_hdr), _ptr(occ), _ptr(recv_row), _ptr(bucket_slot),
         _ptr(expert_counts), _ptr(counters), _stream(stream)))
+
+
+def moe_pw_route_assign(cfg, logits, idx, gates, slot_map, occ, pool_hdr, counters, workspace,
+                        workspace_bytes=None, stream=None):
+    """moe_pw_route + moe_pw_assign_headers, one clustered launch where the
+    batch allows (pooled mode)."""
+    c = _cfg(cfg)
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check("moe_pw_route_assign", load_library().moe_pw_route_assign(
+        ctypes.byref(c), _ptr(logits), _ptr(idx), _ptr(gates), _ptr(slot_map), _ptr(occ),
+        _ptr(pool_hdr), _ptr(counters), _ptr(workspace), wsb, _stream(stream)))
+
+
+def moe_pw_route_assign_plan(cfg) -> bool:
+    """True if moe_pw_route_assign takes its one clustered launch for this
+    batch on the current device."""
+    c = _cfg(cfg)
+    one = ctypes.c_int32(0)
+    _check("moe_pw_route_assign_plan",
+           load_library().moe_pw_route_assign_plan(ctypes.byref(c), ctypes.byref(one)))
+    return bool(one.value)
 
 
 def moe_pw_assign_headers(cfg, idx, slot_map, occ, pool_hdr, counters, workspace,
@@ -561,6 +584,10 @@ class Buffers:
         moe_pw_assign(self.cfg, self.idx, self.slot_map, self.occ, self.counters, self.workspace,
                       stream=stream)
 
+    def route_assign(self, stream=None):
+        moe_pw_route_assign(self.cfg, self.logits, self.idx, self.gates, self.slot_map, self.occ,
+                            self.pool_hdr, self.counters, self.workspace, stream=stream)
+
     def assign_headers(self, stream=None):
         moe_pw_assign_headers(self.cfg, self.idx, self.slot_map, self.occ, self.pool_hdr,
                               self.counters, self.workspace, stream=stream)
@@ -715,10 +742,15 @@ class Buffers:
                 s0.wait_event(ev)
 
     def run_step(self, stream=None):
-        """route -> dispatch (assign, pack, bucket; pooled mode: the pack and
-        the bucketing in one launch) -> expert -> combine."""
-        self.route(stream)
-        self.dispatch(stream)
+        """route -> dispatch (assign, pack, bucket) -> expert -> combine.
+        Pooled mode: route and assignment in one launch, then the pack and the
+        bucketing in one launch."""
+        if self.cfg.mode == MOE_PW_POOLED:
+            self.route_assign(stream)
+            self.pack_bucket(stream)
+        else:
+            self.route(stream)
+            self.dispatch(stream)
         self.expert(stream)
         self.combine(stream)
 

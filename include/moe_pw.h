@@ -260,6 +260,37 @@ int moe_pw_assign_noalloc(const moe_pw_config *cfg, const int32_t *idx, int32_t 
                           int32_t *occ, moe_pw_counters *counters, cudaStream_t stream);
 
 /*
+ * moe_pw_route followed by moe_pw_assign_headers, in one launch where the
+ * batch allows (pooled mode, one GPU, and moe_pw_route_assign_plan below):
+ * one thread-block cluster per source
+ * shard routes the shard's tokens, exchanges the per-pool counts of its
+ * blocks through distributed shared memory and ranks the choices, so the
+ * assignment needs no separate count, scan and rank kernels and no global
+ * workspace.  Outputs (idx, gates, slot_map, occ, the kept slots' headers in
+ * pool_hdr, *counters zeroed and then the sender drops) equal those of the
+ * two calls.  Where the one launch does not apply (shared memory per block,
+ * no cluster placement on this device, or a batch large enough for the two
+ * calls to be faster) the two calls are made, which is why workspace and
+ * workspace_bytes are needed as for moe_pw_assign.  Pooled mode only
+ * (MOE_PW_EUNSUPPORTED otherwise).
+ */
+int moe_pw_route_assign(const moe_pw_config *cfg, const float *logits, int32_t *idx,
+                        float *gates, int32_t *slot_map, int32_t *occ, int32_t *pool_hdr,
+                        moe_pw_counters *counters, void *workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
+/*
+ * Which form moe_pw_route_assign takes for this batch on the current device:
+ * *one_launch = 1 for the one clustered launch, 0 for moe_pw_route followed
+ * by moe_pw_assign_headers.  The one launch is taken where it applies (see
+ * above) and the batch has at most 1,024 tokens per SM: a cluster is tied to
+ * one source shard, so the route's token work cannot spread evenly over the
+ * SMs, and on larger batches that costs more than the separate assignment
+ * kernels' fixed latency.  Needs a CUDA device (occupancy queries; no launch).
+ */
+int moe_pw_route_assign_plan(const moe_pw_config *cfg, int32_t *one_launch);
+
+/*
  * moe_pw_assign that also writes the header (the expert id) of every slot the
  * sender kept into pool_hdr [n_slots]; the other headers are left as they
  * are.  Pooled mode only (MOE_PW_EUNSUPPORTED otherwise).  The first half of

@@ -1,5 +1,7 @@
-"""The fused dispatch (assignment with headers, then pack and bucketing in one
-launch) against the three separate launches and the oracle.
+"""The fused dispatch against the separate launches and the oracle: route and
+assignment in one clustered launch (moe_pw_route_assign), the assignment with
+headers (moe_pw_assign_headers), and pack and bucketing in one launch
+(moe_pw_pack_bucket).
 
 Every output buffer is poisoned before each path runs, so a word the fused
 launch fails to write shows up.  The cases cover bucket items of one and of
@@ -118,3 +120,88 @@ def test_fused_repeat_rebuilds_every_word():
         for n in OUTPUTS:
             assert torch.equal(getattr(b, n), keep[n]), n
     assert b.stats().error == 0
+
+
+RA_OUTPUTS = ["idx", "gates", "slot_map", "occ", "pool_hdr"]
+
+RA_CASES = {
+    **{n: CASES[n] for n in ["tiny", "tiny_tight", "single_pool", "one_expert_per_wave",
+                             "wide_E", "E2048", "pages_ranks_small", "long_sources",
+                             "multi_tile_ragged_tail"]},
+    "k1": SMALL_CASES["k1"],
+    "k16": SMALL_CASES["k16"],
+    "k32": SMALL_CASES["k32"],
+    "odd_E": synth.Workload("odd_E", T=4 * 300, R=4, L=5, W=1, P=5, k=6, D=8, seq_len=300,
+                            logit_kind=synth.LOGIT_ZIPF),   # E = 20: NV = 1, not full
+    "one_token_sources": synth.Workload("one_token", T=16, R=16, L=4, W=2, P=2, k=3, D=8,
+                                       seq_len=1, logit_kind=synth.LOGIT_IID),
+    # 48,000 tokens per source: the one-launch form's shared memory would pass
+    # its limit, so the call runs route + assignment instead (same outputs)
+    "fallback_long_sources": synth.Workload("fallback", T=2 * 48000, R=2, L=6, W=3, P=2, k=8,
+                                            D=8, seq_len=48000,
+                                            logit_kind=synth.LOGIT_SEQBIAS),
+}
+
+
+RA_SEPARATE = {"fallback_long_sources", "E2048"}
+
+
+def _poison_route(b):
+    b.idx.fill_(-5)
+    b.gates.fill_(float("nan"))
+    b.slot_map.fill_(-77)
+    b.occ.fill_(-77)
+    b.pool_hdr.fill_(-55)
+
+
+@pytest.mark.parametrize("name", list(RA_CASES))
+def test_route_assign_equals_separate_launches(name):
+    """moe_pw_route_assign against moe_pw_route + moe_pw_assign_headers: ids,
+    gates (bit for bit: the same selection code), slots, occupancies, the
+    kept slots' headers and the sender counters."""
+    w = RA_CASES[name]
+    lg, x, s = _inputs(w)
+    ref = _fresh(w, lg, x, s)
+    _poison_route(ref)
+    ref.route()
+    ref.assign_headers()
+    st_ref = ref.stats()
+
+    b = _fresh(w, lg, x, s)
+    # every case runs the one clustered launch but two whose shared memory
+    # per block would pass the launch's limit: 48,000 tokens per source, and
+    # 1,024 pools per source (E2048: the per-warp pool counts alone take 32 KB)
+    assert mp.moe_pw_route_assign_plan(b.cfg) == (name not in RA_SEPARATE)
+    _poison_route(b)
+    b.counters.fill_(-1)  # the call zeroes the counters itself
+    b.route_assign()
+    st = b.stats()
+    torch.cuda.synchronize()
+    for n in RA_OUTPUTS:
+        assert torch.equal(getattr(b, n), getattr(ref, n)), n
+    assert (st.assignments, st.sender_dropped, st.max_occ, st.error) == (
+        st_ref.assignments, st_ref.sender_dropped, st_ref.max_occ, st_ref.error)
+
+
+@pytest.mark.parametrize("name", ["k16", "E2048", "fallback_long_sources"])
+def test_route_assign_step_full_parity(name):
+    """The whole step (run_step: route + assignment, pack + bucketing, expert
+    op, combine) against the whole oracle."""
+    w = RA_CASES[name]
+    lg, x, s = _inputs(w)
+    b = _fresh(w, lg, x, s)
+    _poison(b)
+    b.run_step()
+    st = b.stats(raise_on_device_error=False)
+    torch.cuda.synchronize()
+    check_full(w, lg, x, s, b, st)
+
+
+def test_route_assign_plan_follows_tokens_per_sm():
+    """One launch up to 1,024 tokens per SM: the 65,536-token layer batch
+    takes it, the 262,144-token rack batch (above 148 * 1,024) does not."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for name in ["layer", "rack"]:
+        w = synth.WORKLOADS[name]
+        expect = w.T <= 1024 * sms
+        assert mp.moe_pw_route_assign_plan(mp.Config.from_workload(w)) == expect, name
