@@ -352,7 +352,7 @@ def traffic_from_profiles(kernel: str, alg_bytes: float):
     over that launch's algorithmic bytes, times this launch's algorithmic
     bytes (the kernel streams its rows once, so its traffic grows in
     proportion).  None unless the kernel source is unchanged since the capture
-    (its sha256 is recorded there)."""
+    (the sha256 of every source file is recorded there)."""
     import hashlib
     import re
     prof = os.path.join(ROOT, "profiles", f"{kernel}_small_case_traffic.txt")
@@ -360,13 +360,14 @@ def traffic_from_profiles(kernel: str, alg_bytes: float):
         return None
     text = open(prof).read()
     m_r = re.search(r"^traffic_per_algorithmic_byte:\s*([0-9.eE+]+)", text, re.M)
-    m_h = re.search(r"^source_sha256:\s*([0-9a-f]+)", text, re.M)
-    m_f = re.search(r"^source_file:\s*(\S+)", text, re.M)
-    if not (m_r and m_h and m_f):
+    files = re.findall(r"^source_file:\s*(\S+)", text, re.M)
+    hashes = re.findall(r"^source_sha256:\s*([0-9a-f]+)", text, re.M)
+    if not (m_r and files and len(files) == len(hashes)):
         return None
-    src = os.path.join(ROOT, m_f.group(1))
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != m_h.group(1):
-        return None
+    for f, h in zip(files, hashes):  # every source of the kernel unchanged
+        src = os.path.join(ROOT, f)
+        if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != h:
+            return None
     return float(m_r.group(1)) * alg_bytes
 
 
