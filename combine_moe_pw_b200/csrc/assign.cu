@@ -32,6 +32,11 @@ namespace moe_pw {
 namespace {
 
 constexpr int AW = 8;  // warps per block in count/rank
+// Blocks per SM the count and rank passes are compiled for (32 registers): a
+// rack-size batch has 1024 chunks, which then all run in one wave on 148 SMs
+// (at 38-40 registers only 6 blocks fit, and a seventh block per SM started
+// one block's time late).
+constexpr int AW_MIN_BLOCKS = 8;
 constexpr int MAX_FUSED_CHUNKS = 32;
 
 struct RankArgs {
@@ -65,8 +70,12 @@ struct Smem {
     int32_t *bin_tab;  // [E]
     int32_t *hist;     // [AW][NB]
     int32_t *off;      // [E + 1] (ragged rank pass)
-    int32_t *bins;     // [chunk_tokens * k]: bin of each assignment of the chunk, -1 if invalid
+    // [chunk_tokens * k]: each assignment of the chunk as (expert << 16) | bin,
+    // -1 if its id is invalid (bins and ids are below 2^11, so both fit)
+    int32_t *bins;
 };
+
+__device__ __forceinline__ int32_t bin_part(int32_t v) { return v >= 0 ? (v & 0xFFFF) : -1; }
 
 __device__ __forceinline__ Smem carve(const Geo &g, int32_t *sm)
 {
@@ -79,7 +88,9 @@ __device__ __forceinline__ Smem carve(const Geo &g, int32_t *sm)
 }
 
 // bins[i] for the chunk's assignments a0 + i, i < n; the loads of one thread
-// are issued together.  flag: report ids outside [0, E) (rank pass).
+// are issued together.  flag: report ids outside [0, E) (rank pass).  The
+// expert id stays beside the bin, so the rank walk's header stores need no
+// second global read.
 __device__ __forceinline__ void load_bins(const RankArgs &p, const Smem &s, int64_t a0, int n,
                                           bool flag)
 {
@@ -95,12 +106,12 @@ __device__ __forceinline__ void load_bins(const RankArgs &p, const Smem &s, int6
         for (int u = 0; u < U; ++u) {
             const int i = i0 + u * int(blockDim.x);
             if (i < n) {
-                int32_t b = -1;
+                int32_t v = -1;
                 if (e[u] >= 0 && e[u] < p.g.E)
-                    b = s.bin_tab[e[u]];
+                    v = (e[u] << 16) | s.bin_tab[e[u]];
                 else if (flag)
                     set_error(p.ctr, MOE_PW_DEVERR_EXPERT_ID);
-                s.bins[i] = b;
+                s.bins[i] = v;
             }
         }
     }
@@ -113,7 +124,7 @@ __device__ __forceinline__ void warp_hist(const RankArgs &p, const Smem &s, int 
 {
     int32_t *h = s.hist + warp * p.g.NB;
     for (int i = w0 + lane; i < w1; i += 32) {
-        const int32_t b = s.bins[i];
+        const int32_t b = bin_part(s.bins[i]);
         if (b >= 0) atomicAdd(&h[b], 1);
     }
 }
@@ -124,7 +135,7 @@ __device__ __forceinline__ void setup(const RankArgs &p, const Smem &s)
     for (int i = threadIdx.x; i < AW * p.g.NB; i += blockDim.x) s.hist[i] = 0;
 }
 
-__global__ void __launch_bounds__(AW * 32) assign_count(RankArgs p)
+__global__ void __launch_bounds__(AW * 32, AW_MIN_BLOCKS) assign_count(RankArgs p)
 {
     extern __shared__ int32_t sm[];
     const Smem s = carve(p.g, sm);
@@ -228,7 +239,7 @@ __global__ void __launch_bounds__(1024) ragged_offsets(RankArgs p)
     if (threadIdx.x == blockDim.x - 1) p.occ[E] = run;
 }
 
-__global__ void __launch_bounds__(AW * 32) assign_rank(RankArgs p)
+__global__ void __launch_bounds__(AW * 32, AW_MIN_BLOCKS) assign_rank(RankArgs p)
 {
     extern __shared__ int32_t sm[];
     const Smem s = carve(p.g, sm);
@@ -281,7 +292,8 @@ __global__ void __launch_bounds__(AW * 32) assign_rank(RankArgs p)
     const int nbits = 32 - __clz(p.g.NB);  // keys b + 1 in [0, NB]
     for (int a = w0; a < w1; a += 32) {
         const int i = a + lane;
-        const int32_t b = i < w1 ? s.bins[i] : -1;
+        const int32_t v = i < w1 ? s.bins[i] : -1;
+        const int32_t b = bin_part(v);
         const unsigned same = equal_lanes(uint32_t(b + 1), nbits);
         const int32_t r = (b >= 0 ? h[b] : 0) + __popc(same & lanemask_lt());
         __syncwarp();
@@ -296,7 +308,7 @@ __global__ void __launch_bounds__(AW * 32) assign_rank(RankArgs p)
                     slot = int32_t((pool_base + b) * p.g.C_s + r);
             }
             p.slot_map[a0 + i] = slot;
-            if (p.pool_hdr && slot >= 0) p.pool_hdr[slot] = p.idx[a0 + i];
+            if (p.pool_hdr && slot >= 0) p.pool_hdr[slot] = v >> 16;
         }
     }
 }
