@@ -697,7 +697,7 @@ def main():
     chunk_tokens = min(max(2048 // w.k, 1), w.T // w.R if w.mode == 0 else w.T)
     chunks_per_source = -(-(w.T // w.R) // chunk_tokens)
     assign_kernels = (2 if chunks_per_source <= 32 else 3) if w.mode == 0 else 4
-    one_launch = mode == "fused" and mp.moe_pw_route_assign_plan(cfg)
+    one_launch = mode == "fused" and mp.moe_pw_route_assign_plan(cfg) != mp.RA_SEPARATE
     launches_per_step = {"fused": 4 if one_launch else 4 + assign_kernels,
                          "split-route": 4 + assign_kernels,
                          "separate": 5 + assign_kernels}[mode]

@@ -16,8 +16,9 @@
 //   2. scan  : per (group, bin), exclusive prefix over the group's chunks;
 //   3. rank  : per chunk, recount, per-warp bases = chunk base + earlier warps,
 //              then each warp walks its assignments 32 at a time: lanes with
-//              the same bin find each other (one ballot per bit of the bin
-//              id) and take ranks in lane order.
+//              the same bin find each other (each sets its bit in a per-warp
+//              mask word of the bin in shared memory and reads it back) and
+//              take ranks in lane order.
 // Passes 1 and 3 first read the chunk's expert ids with every thread's loads
 // in flight at once and keep their bins in shared memory, so the walks above
 // touch only shared memory (the latency of one global read per chunk instead
@@ -73,6 +74,7 @@ struct Smem {
     // [chunk_tokens * k]: each assignment of the chunk as (expert << 16) | bin,
     // -1 if its id is invalid (bins and ids are below 2^11, so both fit)
     int32_t *bins;
+    uint32_t *wmask;   // [AW][NB]: the rank walk's lane masks, zero between steps
 };
 
 __device__ __forceinline__ int32_t bin_part(int32_t v) { return v >= 0 ? (v & 0xFFFF) : -1; }
@@ -84,6 +86,7 @@ __device__ __forceinline__ Smem carve(const Geo &g, int32_t *sm)
     s.hist = sm + g.E;
     s.off = s.hist + AW * g.NB;
     s.bins = s.off + g.E + 1;
+    s.wmask = reinterpret_cast<uint32_t *>(s.bins + g.chunk_tokens * g.k);
     return s;
 }
 
@@ -132,8 +135,94 @@ __device__ __forceinline__ void warp_hist(const RankArgs &p, const Smem &s, int 
 __device__ __forceinline__ void setup(const RankArgs &p, const Smem &s)
 {
     for (int e = threadIdx.x; e < p.g.E; e += blockDim.x) s.bin_tab[e] = bin_of_expert(p.g, e);
-    for (int i = threadIdx.x; i < AW * p.g.NB; i += blockDim.x) s.hist[i] = 0;
+    for (int i = threadIdx.x; i < AW * p.g.NB; i += blockDim.x) {
+        s.hist[i] = 0;
+        s.wmask[i] = 0u;
+    }
 }
+
+size_t rank_smem_bytes(const Geo &g)
+{
+    return sizeof(int32_t) * (size_t(g.E) + 2 * size_t(AW) * g.NB + size_t(g.E) + 1 +
+                              size_t(g.chunk_tokens) * g.k);
+}
+
+// Rank the assignments of one chunk (pass 3): recount, per-warp bases =
+// chunk base + earlier warps, then each warp walks its assignments 32 at a
+// time and writes their slots (and, with pool_hdr, the kept slots' headers).
+// Expects bin_tab filled, hist and wmask zeroed and (ragged) off loaded, with the
+// block synchronised after; AW warps take part.
+__device__ __forceinline__ void rank_chunk(const RankArgs &p, const Smem &s, int chunk)
+{
+    const bool ragged = p.g.mode == MOE_PW_RAGGED;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int64_t a0, a1;
+    int group;
+    chunk_range(p.g, chunk, a0, a1, group);
+    const int n = int(a1 - a0);
+    load_bins(p, s, a0, n, true);
+    __syncthreads();
+    const int w0 = n * warp / AW, w1 = n * (warp + 1) / AW;
+    warp_hist(p, s, w0, w1, warp, lane);
+    __syncthreads();
+    // turn per-warp counts into per-warp starting ranks.  The chunk's base
+    // is the scan pass's output, or (few chunks per group) the sum of the
+    // earlier chunks' raw counts, taken here; then the group's last chunk
+    // also settles the pools' occupancy and drops, which the scan pass
+    // would have done.
+    const int cpg = p.g.chunks_per_group;
+    const int ci = chunk - group * cpg;
+    for (int b = threadIdx.x; b < p.g.NB; b += blockDim.x) {
+        int32_t run = 0;
+        if (p.fused_scan) {
+            const int32_t *col = p.counts + int64_t(group) * cpg * p.g.NB + b;
+            for (int c = 0; c < ci; ++c) run += col[int64_t(c) * p.g.NB];
+        } else {
+            run = p.counts[int64_t(chunk) * p.g.NB + b];
+        }
+        for (int w = 0; w < AW; ++w) {
+            const int32_t v = s.hist[w * p.g.NB + b];
+            s.hist[w * p.g.NB + b] = run;
+            run += v;
+        }
+        if (p.fused_scan && ci == cpg - 1) {
+            // run = the pool's total over the whole group
+            const int64_t kept = run < p.g.C_s ? run : p.g.C_s;
+            p.occ[int64_t(group) * p.g.NB + b] = int32_t(kept);
+            if (run > kept) atomicAdd(&p.ctr->sender_dropped, (unsigned long long)(run - kept));
+            atomicMax(&p.ctr->max_occ, int32_t(kept));
+        }
+    }
+    __syncthreads();
+    int32_t *h = s.hist + warp * p.g.NB;
+    uint32_t *wm = s.wmask + warp * p.g.NB;
+    const int64_t pool_base = int64_t(group) * p.g.NB;
+    for (int a = w0; a < w1; a += 32) {
+        const int i = a + lane;
+        const int32_t v = i < w1 ? s.bins[i] : -1;
+        const int32_t b = bin_part(v);
+        const unsigned same = equal_lanes_smem(b, wm, lane);
+        const int32_t r = (b >= 0 ? h[b] : 0) + __popc(same & lanemask_lt());
+        __syncwarp();
+        if (b >= 0 && lane == __ffs(same) - 1) {
+            h[b] += __popc(same);
+            wm[b] = 0u;
+        }
+        __syncwarp();
+        if (i < w1) {
+            int32_t slot = -1;
+            if (b >= 0) {
+                if (ragged)
+                    slot = s.off[b] + r;
+                else if (r < p.g.C_s)
+                    slot = int32_t((pool_base + b) * p.g.C_s + r);
+            }
+            p.slot_map[a0 + i] = slot;
+            if (p.pool_hdr && slot >= 0) p.pool_hdr[slot] = v >> 16;
+        }
+    }
+}
+
 
 __global__ void __launch_bounds__(AW * 32, AW_MIN_BLOCKS) assign_count(RankArgs p)
 {
@@ -244,80 +333,12 @@ __global__ void __launch_bounds__(AW * 32, AW_MIN_BLOCKS) assign_rank(RankArgs p
     extern __shared__ int32_t sm[];
     const Smem s = carve(p.g, sm);
     setup(p, s);
-    const bool ragged = p.g.mode == MOE_PW_RAGGED;
-    if (ragged)
+    if (p.g.mode == MOE_PW_RAGGED)
         for (int e = threadIdx.x; e <= p.g.E; e += blockDim.x) s.off[e] = p.occ[e];
     __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int64_t a0, a1;
-    int group;
-    chunk_range(p.g, blockIdx.x, a0, a1, group);
-    const int n = int(a1 - a0);
-    load_bins(p, s, a0, n, true);
-    __syncthreads();
-    const int w0 = n * warp / AW, w1 = n * (warp + 1) / AW;
-    warp_hist(p, s, w0, w1, warp, lane);
-    __syncthreads();
-    // turn per-warp counts into per-warp starting ranks.  The chunk's base
-    // is the scan pass's output, or (few chunks per group) the sum of the
-    // earlier chunks' raw counts, taken here; then the group's last chunk
-    // also settles the pools' occupancy and drops, which the scan pass
-    // would have done.
-    const int cpg = p.g.chunks_per_group;
-    const int ci = int(blockIdx.x) - group * cpg;
-    for (int b = threadIdx.x; b < p.g.NB; b += blockDim.x) {
-        int32_t run = 0;
-        if (p.fused_scan) {
-            const int32_t *col = p.counts + int64_t(group) * cpg * p.g.NB + b;
-            for (int c = 0; c < ci; ++c) run += col[int64_t(c) * p.g.NB];
-        } else {
-            run = p.counts[int64_t(blockIdx.x) * p.g.NB + b];
-        }
-        for (int w = 0; w < AW; ++w) {
-            const int32_t v = s.hist[w * p.g.NB + b];
-            s.hist[w * p.g.NB + b] = run;
-            run += v;
-        }
-        if (p.fused_scan && ci == cpg - 1) {
-            // run = the pool's total over the whole group
-            const int64_t kept = run < p.g.C_s ? run : p.g.C_s;
-            p.occ[int64_t(group) * p.g.NB + b] = int32_t(kept);
-            if (run > kept) atomicAdd(&p.ctr->sender_dropped, (unsigned long long)(run - kept));
-            atomicMax(&p.ctr->max_occ, int32_t(kept));
-        }
-    }
-    __syncthreads();
-    int32_t *h = s.hist + warp * p.g.NB;
-    const int64_t pool_base = int64_t(group) * p.g.NB;
-    const int nbits = 32 - __clz(p.g.NB);  // keys b + 1 in [0, NB]
-    for (int a = w0; a < w1; a += 32) {
-        const int i = a + lane;
-        const int32_t v = i < w1 ? s.bins[i] : -1;
-        const int32_t b = bin_part(v);
-        const unsigned same = equal_lanes(uint32_t(b + 1), nbits);
-        const int32_t r = (b >= 0 ? h[b] : 0) + __popc(same & lanemask_lt());
-        __syncwarp();
-        if (b >= 0 && lane == __ffs(same) - 1) h[b] += __popc(same);
-        __syncwarp();
-        if (i < w1) {
-            int32_t slot = -1;
-            if (b >= 0) {
-                if (ragged)
-                    slot = s.off[b] + r;
-                else if (r < p.g.C_s)
-                    slot = int32_t((pool_base + b) * p.g.C_s + r);
-            }
-            p.slot_map[a0 + i] = slot;
-            if (p.pool_hdr && slot >= 0) p.pool_hdr[slot] = v >> 16;
-        }
-    }
+    rank_chunk(p, s, int(blockIdx.x));
 }
 
-size_t rank_smem_bytes(const Geo &g)
-{
-    return sizeof(int32_t) * (size_t(g.E) + size_t(AW) * g.NB + size_t(g.E) + 1 +
-                              size_t(g.chunk_tokens) * g.k);
-}
 
 }  // namespace
 

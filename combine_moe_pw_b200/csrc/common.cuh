@@ -50,17 +50,18 @@ int dev_info(DevInfo *out);
 // Kernel launchers (asynchronous; return cudaError_t of the launch).
 cudaError_t launch_route(const Geo &g, const float *logits, int32_t *idx, float *gates,
                          cudaStream_t st);
-// Route and sender assignment (with the kept slots' headers) in one launch,
-// pooled mode on one GPU; zeroes *ctr first.  cudaErrorNotSupported (nothing
-// enqueued) when the batch's shape does not fit the launch or the batch is
-// large enough for the separate kernels to be faster: the caller then runs
-// launch_route and launch_assign.
+// Route and sender assignment (with the kept slots' headers) in one
+// clustered launch, pooled mode on one GPU; zeroes *ctr first.
+// cudaErrorNotSupported (nothing enqueued) when the batch takes the separate
+// kernels: the caller then runs launch_route and launch_assign.  form:
+// MOE_PW_RA_* to ask for one form (cudaErrorInvalidValue if the clustered
+// launch does not fit), -1 for the default choice.
 cudaError_t launch_route_assign(const Geo &g, const float *logits, int32_t *idx, float *gates,
                                 int32_t *slot_map, int32_t *occ, int32_t *pool_hdr,
-                                moe_pw_counters *ctr, cudaStream_t st);
-// Whether launch_route_assign takes the one launch for this batch on the
-// current device (*one_launch 1) or returns cudaErrorNotSupported (0).
-cudaError_t route_assign_plan(const Geo &g, int *one_launch);
+                                moe_pw_counters *ctr, cudaStream_t st, int form = -1);
+// The form launch_route_assign takes for this batch on the current device
+// (MOE_PW_RA_*; MOE_PW_RA_SEPARATE: it returns cudaErrorNotSupported).
+cudaError_t route_assign_plan(const Geo &g, int *form);
 // pool_hdr (optional): also write the kept slots' headers (the expert id),
 // as the fused pack + bucketing launch expects.
 cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, int32_t *occ,
@@ -282,17 +283,17 @@ __device__ __forceinline__ int32_t bin_of_expert(const Geo &g, int32_t e)
     return g.mode == MOE_PW_POOLED ? (e / g.L) * g.W + (e % g.L) / g.P : e;
 }
 
-// Lanes of the warp holding the same key as this lane (key in [0, 2^nbits)):
-// one ballot per key bit.  All lanes call it with the same nbits.
-__device__ __forceinline__ unsigned equal_lanes(uint32_t key, int nbits)
+// Lanes of the warp holding the same bin b >= 0 as this lane (b < 0: none),
+// through a per-warp array of lane masks in shared memory, zero on entry:
+// each lane sets its bit in mask[b] and reads the word back.  The caller's
+// lowest lane of each group (lane == __ffs(result) - 1) must set mask[b] back
+// to 0, after a __syncwarp, before the next call.  One shared-memory atomic
+// instead of a ballot per bit of the bin id.
+__device__ __forceinline__ unsigned equal_lanes_smem(int32_t b, uint32_t *mask, int lane)
 {
-    unsigned m = FULL_MASK;
-    for (int i = 0; i < nbits; ++i) {
-        const bool bit = (key >> i) & 1u;
-        const unsigned bal = __ballot_sync(FULL_MASK, bit);
-        m &= bit ? bal : ~bal;
-    }
-    return m;
+    if (b >= 0) atomicOr(&mask[b], 1u << lane);
+    __syncwarp();
+    return b >= 0 ? mask[b] : 0u;
 }
 
 __device__ __forceinline__ unsigned lanemask_lt()

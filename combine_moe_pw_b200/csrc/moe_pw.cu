@@ -269,15 +269,16 @@ int moe_pw_assign_headers(const moe_pw_config *cfg, const int32_t *idx, int32_t 
     return cuda_rc(launch_assign(g, idx, slot_map, occ, counters, workspace, stream, pool_hdr));
 }
 
-int moe_pw_route_assign(const moe_pw_config *cfg, const float *logits, int32_t *idx,
-                        float *gates, int32_t *slot_map, int32_t *occ, int32_t *pool_hdr,
-                        moe_pw_counters *counters, void *workspace, size_t workspace_bytes,
-                        cudaStream_t stream)
+int moe_pw_route_assign_form(const moe_pw_config *cfg, int32_t form, const float *logits,
+                             int32_t *idx, float *gates, int32_t *slot_map, int32_t *occ,
+                             int32_t *pool_hdr, moe_pw_counters *counters, void *workspace,
+                             size_t workspace_bytes, cudaStream_t stream)
 {
     Geo g;
     int rc = make_geo(cfg, &g);
     if (rc != MOE_PW_OK) return rc;
     if (g.mode != MOE_PW_POOLED || g.E % 4 != 0) return MOE_PW_EUNSUPPORTED;
+    if (form < -1 || form > MOE_PW_RA_CLUSTER) return MOE_PW_EINVAL;
     if (!counters || !occ) return MOE_PW_EINVAL;
     if (g.T > 0 && (!logits || !idx || !gates || !slot_map || !pool_hdr || !workspace))
         return MOE_PW_EINVAL;
@@ -287,9 +288,10 @@ int moe_pw_route_assign(const moe_pw_config *cfg, const float *logits, int32_t *
                      !aligned(slot_map, 4) || !aligned(pool_hdr, 4) ||
                      !aligned(workspace, 256))))
         return MOE_PW_EUNSUPPORTED;
-    if (g.T > 0) {
-        const cudaError_t e =
-            launch_route_assign(g, logits, idx, gates, slot_map, occ, pool_hdr, counters, stream);
+    if (g.T > 0 && form != MOE_PW_RA_SEPARATE) {
+        const cudaError_t e = launch_route_assign(g, logits, idx, gates, slot_map, occ, pool_hdr,
+                                                  counters, stream, form);
+        if (e == cudaErrorInvalidValue) return MOE_PW_EUNSUPPORTED;  // the form does not fit
         if (e != cudaErrorNotSupported) return cuda_rc(e);
     }
     rc = moe_pw_route(cfg, logits, idx, gates, stream);
@@ -298,15 +300,24 @@ int moe_pw_route_assign(const moe_pw_config *cfg, const float *logits, int32_t *
                                  workspace_bytes, stream);
 }
 
-int moe_pw_route_assign_plan(const moe_pw_config *cfg, int32_t *one_launch)
+int moe_pw_route_assign(const moe_pw_config *cfg, const float *logits, int32_t *idx,
+                        float *gates, int32_t *slot_map, int32_t *occ, int32_t *pool_hdr,
+                        moe_pw_counters *counters, void *workspace, size_t workspace_bytes,
+                        cudaStream_t stream)
+{
+    return moe_pw_route_assign_form(cfg, -1, logits, idx, gates, slot_map, occ, pool_hdr,
+                                    counters, workspace, workspace_bytes, stream);
+}
+
+int moe_pw_route_assign_plan(const moe_pw_config *cfg, int32_t *form)
 {
     Geo g;
     int rc = make_geo(cfg, &g);
     if (rc != MOE_PW_OK) return rc;
-    if (!one_launch) return MOE_PW_EINVAL;
-    int one = 0;
-    const cudaError_t e = route_assign_plan(g, &one);
-    *one_launch = one;
+    if (!form) return MOE_PW_EINVAL;
+    int f = MOE_PW_RA_SEPARATE;
+    const cudaError_t e = route_assign_plan(g, &f);
+    *form = f;
     return cuda_rc(e);
 }
 

@@ -18,15 +18,18 @@
 //      blocks through distributed shared memory (its base per pool); the
 //      cluster's last block also writes the occupancies and sender drops;
 //   3. each warp ranks its own choices in (t, j) order, 32 at a time (lanes
-//      with the same pool find each other by ballots) and writes slot_map and
-//      the kept slots' headers;
+//      with the same pool find each other through shared-memory lane masks)
+//      and writes slot_map and the kept slots' headers;
 //   4. cluster barrier before exit, so no block leaves while another may
 //      still read its shared memory.
 // The only waits are the two hardware cluster barriers: no block waits on
 // another cluster, so clusters may run in any order and in any number of
 // waves.  The cluster size is the largest (up to 16) at which every source's
-// cluster is resident at once, which keeps the route's token work spread
-// evenly over the SMs.
+// cluster is resident at once.
+//
+// Larger batches take route_kernel and the assignment passes instead: a
+// cluster is tied to one source shard, so its blocks cannot spread the route
+// work evenly over the SMs (see ra_form below).
 #include <cooperative_groups.h>
 
 #include <map>
@@ -49,6 +52,7 @@ constexpr int RA_MIN_BLOCKS = 32 / RA_WARPS;  // as the route kernel: 64 registe
 constexpr int RA_MAX_CLUSTER = 16;
 constexpr size_t RA_MAX_SMEM = 40 * 1024;  // keeps 4 blocks per SM
 
+
 struct RouteAssignArgs {
     const float *logits;
     int32_t *idx;
@@ -61,12 +65,12 @@ struct RouteAssignArgs {
     int32_t c;  // blocks per source (the cluster size)
 };
 
-// Dynamic shared memory: pool of each expert [E], per-warp pool counts
-// [RA_WARPS][NB], block totals [NB], expert id of each choice [tokens * k]
-// (int16).
+// Dynamic shared memory: pool of each expert [E], per-warp pool counts and
+// lane masks [2][RA_WARPS][NB], block totals [NB], expert id of each choice
+// [tokens * k] (int16).
 inline size_t ra_smem_bytes(const Geo &g, int64_t tok_cap)
 {
-    const size_t ints = size_t(g.E) + size_t(RA_WARPS + 1) * g.NB;
+    const size_t ints = size_t(g.E) + size_t(2 * RA_WARPS + 1) * g.NB;
     return (sizeof(int32_t) * ints + sizeof(int16_t) * size_t(tok_cap) * g.k + 15) & ~size_t(15);
 }
 
@@ -81,8 +85,9 @@ route_assign_kernel(RouteAssignArgs p)
     const int NB = p.g.NB;
     int32_t *bin_tab = dsm;                                    // [E]
     int32_t *hist = bin_tab + p.g.E;                           // [RA_WARPS][NB]
-    int32_t *tot = hist + RA_WARPS * NB;                       // [NB]
-    int16_t *choice = reinterpret_cast<int16_t *>(tot + NB);  // [tokens * k]
+    uint32_t *wmask = reinterpret_cast<uint32_t *>(hist + RA_WARPS * NB);  // [RA_WARPS][NB]
+    int32_t *tot = reinterpret_cast<int32_t *>(wmask + RA_WARPS * NB);     // [NB]
+    int16_t *choice = reinterpret_cast<int16_t *>(tot + NB);              // [tokens * k]
     const int k = KC ? KC : p.g.k;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int c = p.c;
@@ -94,7 +99,10 @@ route_assign_kernel(RouteAssignArgs p)
     const int tw0 = nb * warp / RA_WARPS, tw1 = nb * (warp + 1) / RA_WARPS;
 
     for (int e = threadIdx.x; e < p.g.E; e += blockDim.x) bin_tab[e] = bin_of_expert(p.g, e);
-    for (int i = threadIdx.x; i < RA_WARPS * NB; i += blockDim.x) hist[i] = 0;
+    for (int i = threadIdx.x; i < RA_WARPS * NB; i += blockDim.x) {
+        hist[i] = 0;
+        wmask[i] = 0u;
+    }
     __syncthreads();
 
     // route this warp's tokens (the next row loads during the selection)
@@ -154,16 +162,19 @@ route_assign_kernel(RouteAssignArgs p)
 
     // 3. rank this warp's choices in (t, j) order
     const int64_t pool_base = int64_t(s) * NB;
-    const int nbits = 32 - __clz(NB);  // keys b + 1 in [0, NB]
+    uint32_t *wm = wmask + warp * NB;
     const int aw0 = tw0 * k, aw1 = tw1 * k;
     for (int a = aw0; a < aw1; a += 32) {
         const int i = a + lane;
         const int32_t e = i < aw1 ? int32_t(choice[i]) : -1;
         const int32_t b = e >= 0 ? bin_tab[e] : -1;
-        const unsigned same = equal_lanes(uint32_t(b + 1), nbits);
+        const unsigned same = equal_lanes_smem(b, wm, lane);
         const int32_t r = (b >= 0 ? h[b] : 0) + __popc(same & lanemask_lt());
         __syncwarp();
-        if (b >= 0 && lane == __ffs(same) - 1) h[b] += __popc(same);
+        if (b >= 0 && lane == __ffs(same) - 1) {
+            h[b] += __popc(same);
+            wm[b] = 0u;
+        }
         __syncwarp();
         if (i < aw1) {
             int32_t slot = -1;
@@ -285,24 +296,20 @@ cudaError_t launch_ra_nv(const RouteAssignArgs &p, cudaStream_t st, int *c_out)
     }
 }
 
-// The one launch applies to the batch's shape, and pays off: a cluster is
-// tied to one source shard, so its blocks cannot spread the route's token
-// work evenly over the SMs (placement leaves some SMs a block more than
-// others, up to ~15% more tokens than the even share), while it saves the
-// assignment kernels' fixed latency (count, rank and a launch between).
-// Measured on B200 with 384 experts over 64 sources: at 65,536 tokens one
-// launch took 52 us against 60 us for route + assignment, at 262,144 tokens
-// 166 us against 159 us; the crossover lies near 1,024 tokens per SM.
+// Which form takes the batch.  The clustered launch pays off on small
+// batches: a cluster is tied to one source shard, so its blocks cannot spread
+// the route's token work evenly over the SMs (placement leaves some SMs a
+// block more than others, up to ~15% more tokens than the even share), while
+// it saves the assignment kernels' fixed latency.  Measured on B200 with 384
+// experts over 64 sources (kernels alone): at 65,536 tokens 46.5 us against
+// 50.6 us for route + assignment, at 262,144 tokens 153 us against 145 us;
+// the crossover lies near 1,024 tokens per SM.
 constexpr int64_t RA_MAX_TOKENS_PER_SM = 1024;
 
-bool ra_applies(const Geo &g)
+bool ra_shape_ok(const Geo &g)
 {
-    if (g.mode != MOE_PW_POOLED || g.ep_n != 1 || g.T == 0 || g.E % 4 != 0 || g.E > 32767 ||
-        g.k > 32)
-        return false;
-    DevInfo di;
-    if (dev_info(&di) != 0) return false;
-    return g.T <= RA_MAX_TOKENS_PER_SM * di.sms;
+    return g.mode == MOE_PW_POOLED && g.ep_n == 1 && g.T > 0 && g.E % 4 == 0 && g.E <= 32767 &&
+           g.k <= 32;
 }
 
 RouteAssignArgs ra_args(const Geo &g, const float *logits, int32_t *idx, float *gates,
@@ -321,26 +328,54 @@ RouteAssignArgs ra_args(const Geo &g, const float *logits, int32_t *idx, float *
     return p;
 }
 
+// Whether the clustered launch fits the batch on the current device.
+cudaError_t ra_cluster_fits(const Geo &g, bool *fits)
+{
+    *fits = false;
+    if (!ra_shape_ok(g)) return cudaSuccess;
+    int c = 0;
+    const cudaError_t err =
+        launch_ra_nv(ra_args(g, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr),
+                     nullptr, &c);
+    *fits = c > 0;
+    return err;
+}
+
+// The form the batch takes by default (MOE_PW_RA_*).
+cudaError_t ra_form(const Geo &g, int *form)
+{
+    *form = MOE_PW_RA_SEPARATE;
+    bool cluster = false;
+    const cudaError_t err = ra_cluster_fits(g, &cluster);
+    if (err != cudaSuccess) return err;
+    DevInfo di;
+    if (dev_info(&di) != 0) return cudaErrorUnknown;
+    if (cluster && g.T <= RA_MAX_TOKENS_PER_SM * di.sms) *form = MOE_PW_RA_CLUSTER;
+    return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_route_assign(const Geo &g, const float *logits, int32_t *idx, float *gates,
                                 int32_t *slot_map, int32_t *occ, int32_t *pool_hdr,
-                                moe_pw_counters *ctr, cudaStream_t st)
+                                moe_pw_counters *ctr, cudaStream_t st, int form)
 {
-    if (!ra_applies(g)) return cudaErrorNotSupported;
-    return launch_ra_nv(ra_args(g, logits, idx, gates, slot_map, occ, pool_hdr, ctr), st,
-                        nullptr);
+    cudaError_t err;
+    if (form < 0) {
+        if ((err = ra_form(g, &form)) != cudaSuccess) return err;
+    } else if (form == MOE_PW_RA_CLUSTER) {
+        bool fits = false;
+        if ((err = ra_cluster_fits(g, &fits)) != cudaSuccess) return err;
+        if (!fits) return cudaErrorInvalidValue;
+    } else if (form != MOE_PW_RA_SEPARATE) {
+        return cudaErrorInvalidValue;
+    }
+    if (form == MOE_PW_RA_CLUSTER)
+        return launch_ra_nv(ra_args(g, logits, idx, gates, slot_map, occ, pool_hdr, ctr), st,
+                            nullptr);
+    return cudaErrorNotSupported;
 }
 
-cudaError_t route_assign_plan(const Geo &g, int *one_launch)
-{
-    *one_launch = 0;
-    if (!ra_applies(g)) return cudaSuccess;
-    int c = 0;
-    const cudaError_t err = launch_ra_nv(
-        ra_args(g, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr), nullptr, &c);
-    *one_launch = c > 0;
-    return err;
-}
+cudaError_t route_assign_plan(const Geo &g, int *form) { return ra_form(g, form); }
 
 }  // namespace moe_pw

@@ -104,6 +104,8 @@ SIGNATURES = {
     "moe_pw_bucket": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_route_assign": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_route_assign_plan": [_CFG, ctypes.POINTER(ctypes.c_int32)],
+    "moe_pw_route_assign_form": [_CFG, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                 _SZ, _VP],
     "moe_pw_assign_headers": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_pack_bucket": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_dispatch": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
@@ -273,14 +275,28 @@ def moe_pw_route_assign(cfg, logits, idx, gates, slot_map, occ, pool_hdr, counte
         _ptr(pool_hdr), _ptr(counters), _ptr(workspace), wsb, _stream(stream)))
 
 
-def moe_pw_route_assign_plan(cfg) -> bool:
-    """True if moe_pw_route_assign takes its one clustered launch for this
-    batch on the current device."""
+RA_SEPARATE, RA_CLUSTER = 0, 1  # MOE_PW_RA_*
+
+
+def moe_pw_route_assign_form(cfg, form, logits, idx, gates, slot_map, occ, pool_hdr, counters,
+                             workspace, workspace_bytes=None, stream=None):
+    """moe_pw_route_assign in a given form (RA_*), or -1 for the default;
+    raises MoePwError (MOE_PW_EUNSUPPORTED) if the form does not fit."""
     c = _cfg(cfg)
-    one = ctypes.c_int32(0)
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check("moe_pw_route_assign_form", load_library().moe_pw_route_assign_form(
+        ctypes.byref(c), form, _ptr(logits), _ptr(idx), _ptr(gates), _ptr(slot_map), _ptr(occ),
+        _ptr(pool_hdr), _ptr(counters), _ptr(workspace), wsb, _stream(stream)))
+
+
+def moe_pw_route_assign_plan(cfg) -> int:
+    """The form moe_pw_route_assign takes for this batch on the current
+    device: RA_SEPARATE or RA_CLUSTER."""
+    c = _cfg(cfg)
+    form = ctypes.c_int32(0)
     _check("moe_pw_route_assign_plan",
-           load_library().moe_pw_route_assign_plan(ctypes.byref(c), ctypes.byref(one)))
-    return bool(one.value)
+           load_library().moe_pw_route_assign_plan(ctypes.byref(c), ctypes.byref(form)))
+    return int(form.value)
 
 
 def moe_pw_assign_headers(cfg, idx, slot_map, occ, pool_hdr, counters, workspace,
@@ -584,9 +600,12 @@ class Buffers:
         moe_pw_assign(self.cfg, self.idx, self.slot_map, self.occ, self.counters, self.workspace,
                       stream=stream)
 
-    def route_assign(self, stream=None):
-        moe_pw_route_assign(self.cfg, self.logits, self.idx, self.gates, self.slot_map, self.occ,
-                            self.pool_hdr, self.counters, self.workspace, stream=stream)
+    def route_assign(self, stream=None, form: int = -1):
+        """Route + assignment with the kept slots' headers; form: RA_* or -1
+        for the library's choice."""
+        moe_pw_route_assign_form(self.cfg, form, self.logits, self.idx, self.gates, self.slot_map,
+                                 self.occ, self.pool_hdr, self.counters, self.workspace,
+                                 stream=stream)
 
     def assign_headers(self, stream=None):
         moe_pw_assign_headers(self.cfg, self.idx, self.slot_map, self.occ, self.pool_hdr,

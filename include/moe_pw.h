@@ -261,17 +261,21 @@ int moe_pw_assign_noalloc(const moe_pw_config *cfg, const int32_t *idx, int32_t 
 
 /*
  * moe_pw_route followed by moe_pw_assign_headers, in one launch where the
- * batch allows (pooled mode, one GPU, and moe_pw_route_assign_plan below):
- * one thread-block cluster per source
- * shard routes the shard's tokens, exchanges the per-pool counts of its
- * blocks through distributed shared memory and ranks the choices, so the
- * assignment needs no separate count, scan and rank kernels and no global
- * workspace.  Outputs (idx, gates, slot_map, occ, the kept slots' headers in
+ * batch allows (pooled mode, one GPU; moe_pw_route_assign_plan says which
+ * form runs).  Outputs (idx, gates, slot_map, occ, the kept slots' headers in
  * pool_hdr, *counters zeroed and then the sender drops) equal those of the
- * two calls.  Where the one launch does not apply (shared memory per block,
- * no cluster placement on this device, or a batch large enough for the two
- * calls to be faster) the two calls are made, which is why workspace and
- * workspace_bytes are needed as for moe_pw_assign.  Pooled mode only
+ * two calls in either form:
+ *   - MOE_PW_RA_CLUSTER (up to 1,024 tokens per SM): one thread-block
+ *     cluster per source shard routes the shard's tokens, exchanges the
+ *     per-pool counts of its blocks through distributed shared memory and
+ *     ranks the choices; no global workspace is touched.  A cluster is tied
+ *     to one shard, so its route work cannot spread evenly over the SMs; on
+ *     larger batches that costs more than the assignment kernels' fixed
+ *     latency.
+ *   - MOE_PW_RA_SEPARATE: the two calls (larger batches, or a shape the
+ *     clustered launch does not fit: shared memory per block, or no cluster
+ *     placement on this device).
+ * workspace and workspace_bytes are as for moe_pw_assign.  Pooled mode only
  * (MOE_PW_EUNSUPPORTED otherwise).
  */
 int moe_pw_route_assign(const moe_pw_config *cfg, const float *logits, int32_t *idx,
@@ -279,16 +283,26 @@ int moe_pw_route_assign(const moe_pw_config *cfg, const float *logits, int32_t *
                         moe_pw_counters *counters, void *workspace, size_t workspace_bytes,
                         cudaStream_t stream);
 
+#define MOE_PW_RA_SEPARATE 0
+#define MOE_PW_RA_CLUSTER 1
+
 /*
- * Which form moe_pw_route_assign takes for this batch on the current device:
- * *one_launch = 1 for the one clustered launch, 0 for moe_pw_route followed
- * by moe_pw_assign_headers.  The one launch is taken where it applies (see
- * above) and the batch has at most 1,024 tokens per SM: a cluster is tied to
- * one source shard, so the route's token work cannot spread evenly over the
- * SMs, and on larger batches that costs more than the separate assignment
- * kernels' fixed latency.  Needs a CUDA device (occupancy queries; no launch).
+ * moe_pw_route_assign in the given form (MOE_PW_RA_*), or -1 for its default
+ * choice: for timing the forms against one another and testing each.
+ * MOE_PW_EUNSUPPORTED if the form does not fit the batch on this device
+ * (nothing enqueued); MOE_PW_RA_SEPARATE always fits.
  */
-int moe_pw_route_assign_plan(const moe_pw_config *cfg, int32_t *one_launch);
+int moe_pw_route_assign_form(const moe_pw_config *cfg, int32_t form, const float *logits,
+                             int32_t *idx, float *gates, int32_t *slot_map, int32_t *occ,
+                             int32_t *pool_hdr, moe_pw_counters *counters, void *workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * The form moe_pw_route_assign takes for this batch on the current device:
+ * *form = one of MOE_PW_RA_* above.  Needs a CUDA device (occupancy queries;
+ * nothing is launched).
+ */
+int moe_pw_route_assign_plan(const moe_pw_config *cfg, int32_t *form);
 
 /*
  * moe_pw_assign that also writes the header (the expert id) of every slot the

@@ -143,7 +143,11 @@ RA_CASES = {
 }
 
 
-RA_SEPARATE = {"fallback_long_sources", "E2048"}
+# cases the clustered launch does not fit (its call then refuses with
+# MOE_PW_EUNSUPPORTED): its shared memory per block would pass the launch's
+# limit with 48,000 tokens per source, and with 1,024 pools per source
+# (E2048: the per-warp pool counts alone take 32 KB)
+NOT_CLUSTER = {"fallback_long_sources", "E2048"}
 
 
 def _poison_route(b):
@@ -156,9 +160,9 @@ def _poison_route(b):
 
 @pytest.mark.parametrize("name", list(RA_CASES))
 def test_route_assign_equals_separate_launches(name):
-    """moe_pw_route_assign against moe_pw_route + moe_pw_assign_headers: ids,
-    gates (bit for bit: the same selection code), slots, occupancies, the
-    kept slots' headers and the sender counters."""
+    """The clustered launch of moe_pw_route_assign against moe_pw_route +
+    moe_pw_assign_headers: ids, gates (bit for bit: the same selection code),
+    slots, occupancies, the kept slots' headers and the sender counters."""
     w = RA_CASES[name]
     lg, x, s = _inputs(w)
     ref = _fresh(w, lg, x, s)
@@ -168,19 +172,41 @@ def test_route_assign_equals_separate_launches(name):
     st_ref = ref.stats()
 
     b = _fresh(w, lg, x, s)
-    # every case runs the one clustered launch but two whose shared memory
-    # per block would pass the launch's limit: 48,000 tokens per source, and
-    # 1,024 pools per source (E2048: the per-warp pool counts alone take 32 KB)
-    assert mp.moe_pw_route_assign_plan(b.cfg) == (name not in RA_SEPARATE)
     _poison_route(b)
     b.counters.fill_(-1)  # the call zeroes the counters itself
-    b.route_assign()
+    if name in NOT_CLUSTER:
+        with pytest.raises(mp.MoePwError) as ei:
+            b.route_assign(form=mp.RA_CLUSTER)
+        assert ei.value.code == mp.MOE_PW_EUNSUPPORTED
+        return
+    b.route_assign(form=mp.RA_CLUSTER)
     st = b.stats()
     torch.cuda.synchronize()
     for n in RA_OUTPUTS:
         assert torch.equal(getattr(b, n), getattr(ref, n)), n
     assert (st.assignments, st.sender_dropped, st.max_occ, st.error) == (
         st_ref.assignments, st_ref.sender_dropped, st_ref.max_occ, st_ref.error)
+
+
+@pytest.mark.parametrize("name", list(RA_CASES))
+def test_route_assign_default_form(name):
+    """The default form: the clustered launch on these small batches where it
+    fits, else the two calls; same outputs either way."""
+    w = RA_CASES[name]
+    cfg = mp.Config.from_workload(w)
+    expect = mp.RA_CLUSTER if name not in NOT_CLUSTER else mp.RA_SEPARATE
+    assert mp.moe_pw_route_assign_plan(cfg) == expect
+    lg, x, s = _inputs(w)
+    ref = _fresh(w, lg, x, s)
+    _poison_route(ref)
+    ref.route()
+    ref.assign_headers()
+    b = _fresh(w, lg, x, s)
+    _poison_route(b)
+    b.route_assign()
+    torch.cuda.synchronize()
+    for n in RA_OUTPUTS:
+        assert torch.equal(getattr(b, n), getattr(ref, n)), n
 
 
 @pytest.mark.parametrize("name", ["k16", "E2048", "fallback_long_sources"])
@@ -198,10 +224,11 @@ def test_route_assign_step_full_parity(name):
 
 
 def test_route_assign_plan_follows_tokens_per_sm():
-    """One launch up to 1,024 tokens per SM: the 65,536-token layer batch
-    takes it, the 262,144-token rack batch (above 148 * 1,024) does not."""
+    """The clustered launch up to 1,024 tokens per SM: the 65,536-token layer
+    batch takes it, the 262,144-token rack batch (above 148 * 1,024) takes the
+    separate kernels."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    for name in ["layer", "rack"]:
+    for name in ["layer", "rack", "long"]:
         w = synth.WORKLOADS[name]
-        expect = w.T <= 1024 * sms
+        expect = mp.RA_CLUSTER if w.T <= 1024 * sms else mp.RA_SEPARATE
         assert mp.moe_pw_route_assign_plan(mp.Config.from_workload(w)) == expect, name
