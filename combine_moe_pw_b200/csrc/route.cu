@@ -26,8 +26,9 @@ route_kernel(const float *__restrict__ logits, int32_t *__restrict__ idx,
              float *__restrict__ gates, int64_t T, int E, int k_rt)
 {
     // per warp: candidate list and the selected compound keys in rank order
-    __shared__ unsigned long long cand_sm[ROUTE_WARPS][32];
+    __shared__ __align__(16) unsigned long long cand_sm[ROUTE_WARPS][32];
     __shared__ unsigned long long sel_sm[ROUTE_WARPS][32];
+    __shared__ uint4 key_sm[ROUTE_WARPS][KeyRows<NV>::V][32];
     const int k = KC ? KC : k_rt;
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
@@ -38,8 +39,8 @@ route_kernel(const float *__restrict__ logits, int32_t *__restrict__ idx,
     auto one = [&](int64_t t, const float4 (&row)[NV]) {
         int32_t sel_idx;
         float ex, sum;
-        route_select<NV, FULL, KC, ROUTE_WARPS>(row, k, E4, lane, wib, cand_sm, sel_sm, sel_idx,
-                                                ex, sum);
+        route_select<NV, FULL, KC, ROUTE_WARPS>(row, k, E4, lane, wib, cand_sm, sel_sm, key_sm,
+                                                sel_idx, ex, sum);
         if (lane < k) {
             idx[t * k + lane] = sel_idx;
             gates[t * k + lane] = ex / sum;

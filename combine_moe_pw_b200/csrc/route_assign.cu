@@ -78,8 +78,9 @@ template <int NV, bool FULL, int KC>
 __global__ void __launch_bounds__(RA_WARPS * 32, RA_MIN_BLOCKS)
 route_assign_kernel(RouteAssignArgs p)
 {
-    __shared__ unsigned long long cand_sm[RA_WARPS][32];
+    __shared__ __align__(16) unsigned long long cand_sm[RA_WARPS][32];
     __shared__ unsigned long long sel_sm[RA_WARPS][32];
+    __shared__ uint4 key_sm[RA_WARPS][KeyRows<NV>::V][32];
     extern __shared__ __align__(16) int32_t dsm[];
     cg::cluster_group cluster = cg::this_cluster();
     const int NB = p.g.NB;
@@ -111,8 +112,8 @@ route_assign_kernel(RouteAssignArgs p)
     auto one = [&](int t, const float4 (&row)[NV]) {
         int32_t e;
         float ex, sum;
-        route_select<NV, FULL, KC, RA_WARPS>(row, k, E4, lane, warp, cand_sm, sel_sm, e, ex,
-                                             sum);
+        route_select<NV, FULL, KC, RA_WARPS>(row, k, E4, lane, warp, cand_sm, sel_sm, key_sm, e,
+                                             ex, sum);
         if (lane < k) {
             const int64_t a = (tb0 + t) * k + lane;
             p.idx[a] = e;

@@ -54,12 +54,17 @@ __device__ __forceinline__ void load_row(const float *__restrict__ logits, int64
 // its expert id and the two parts of its softmax gate, ex / sum (the caller
 // divides, for lanes j < k only).  NV: float4s per lane; FULL: E == 128*NV
 // (no bounds checks); KC: k fixed at compile time (0: run-time k).
-// cand_sm[wib], sel_sm[wib]: this warp's shared scratch (NW warps per
-// block).  All 32 lanes call it.
+// cand_sm[wib], sel_sm[wib], key_sm[wib]: this warp's shared scratch (NW
+// warps per block; key_sm holds a lane's keys, used when NV <= 4, so that
+// only the few candidates are read back for the compaction).  All 32 lanes
+// call it.
+template <int NV> struct KeyRows { static constexpr int V = NV <= 4 ? NV : 1; };
+
 template <int NV, bool FULL, int KC, int NW>
 __device__ __forceinline__ void route_select(const float4 (&cur)[NV], int k, int E4, int lane,
                                              int wib, unsigned long long (&cand_sm)[NW][32],
                                              unsigned long long (&sel_sm)[NW][32],
+                                             uint4 (&key_sm)[NW][KeyRows<NV>::V][32],
                                              int32_t &sel_idx_out, float &ex_out,
                                              float &sum_out)
 {
@@ -92,11 +97,22 @@ __device__ __forceinline__ void route_select(const float4 (&cur)[NV], int k, int
             tau = __reduce_max_sync(FULL_MASK, rem);
             rem = (rem == tau) ? 0u : rem;
         }
+    // candidates of this lane; NV <= 4: bit 4v + c of cmask for key[v][c] >= tau
+    uint32_t cmask = 0;
     int cnt = 0;
+    if (NV <= 4) {
 #pragma unroll
-    for (int v = 0; v < NV; ++v)
+        for (int v = 0; v < KeyRows<NV>::V; ++v)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) cnt += key[v][c] >= tau;
+            for (int c = 0; c < 4; ++c)
+                if (key[v][c] >= tau) cmask |= 1u << (4 * v + c);
+        cnt = __popc(cmask);
+    } else {
+#pragma unroll
+        for (int v = 0; v < NV; ++v)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) cnt += key[v][c] >= tau;
+    }
     const int C = tau ? int(__reduce_add_sync(FULL_MASK, unsigned(cnt))) : 1 << 30;
 
     uint32_t sel_key = 0;
@@ -110,24 +126,44 @@ __device__ __forceinline__ void route_select(const float4 (&cur)[NV], int k, int
             if (lane >= o) pos += u;
         }
         pos -= cnt;
+        if (NV <= 4) {
+            // the lane's keys go to shared memory in NV 16-byte stores, and
+            // only its candidates (set bits of cmask, ~9 per token over the
+            // warp) are read back: no predicated store per logit.  A lane
+            // reads only what it wrote, so no barrier is needed.
 #pragma unroll
-        for (int v = 0; v < NV; ++v)
+            for (int v = 0; v < KeyRows<NV>::V; ++v)
+                key_sm[wib][v][lane] = make_uint4(key[v][0], key[v][1], key[v][2], key[v][3]);
+            uint32_t m = cmask;
+            while (m) {
+                const int j = __ffs(m) - 1;
+                m &= m - 1;
+                const int v = j >> 2, c = j & 3;
+                const uint32_t kj = reinterpret_cast<const uint32_t *>(&key_sm[wib][v][lane])[c];
+                cand_sm[wib][pos++] =
+                    (static_cast<unsigned long long>(kj) << 32) | ~(base + 128u * v + c);
+            }
+        } else {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                if (key[v][c] >= tau)
-                    cand_sm[wib][pos++] = (static_cast<unsigned long long>(key[v][c]) << 32) |
-                                          ~(base + 128u * v + c);
+            for (int v = 0; v < NV; ++v)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (key[v][c] >= tau)
+                        cand_sm[wib][pos++] = (static_cast<unsigned long long>(key[v][c]) << 32) |
+                                              ~(base + 128u * v + c);
+        }
         if (lane >= C) cand_sm[wib][lane] = 0ull;  // ranks below every candidate
         __syncwarp();
-        // ... and rank each one against all of them
+        // ... and rank each one against all of them, two per 16-byte load
         const unsigned long long me = cand_sm[wib][lane];
         int rank = 0;
-        const int C4 = (C + 3) & ~3;
-        for (int i = 0; i < C4; i += 4) {
-            rank += cand_sm[wib][i] > me;
-            rank += cand_sm[wib][i + 1] > me;
-            rank += cand_sm[wib][i + 2] > me;
-            rank += cand_sm[wib][i + 3] > me;
+        const int C2 = (C + 1) & ~1;
+        const ulonglong2 *pairs = reinterpret_cast<const ulonglong2 *>(&cand_sm[wib][0]);
+#pragma unroll 2
+        for (int i = 0; i < C2; i += 2) {
+            const ulonglong2 q = pairs[i >> 1];
+            rank += q.x > me;
+            rank += q.y > me;
         }
         if (lane < C && rank < k) sel_sm[wib][rank] = me;
         __syncwarp();
