@@ -224,11 +224,16 @@ __device__ __forceinline__ void rank_chunk(const RankArgs &p, const Smem &s, int
 }
 
 
+// Launched as a programmatic dependent of the route: the shared-memory
+// set-up overlaps the route's last blocks.  Zeroes the counters.
 __global__ void __launch_bounds__(AW * 32, AW_MIN_BLOCKS) assign_count(RankArgs p)
 {
     extern __shared__ int32_t sm[];
     const Smem s = carve(p.g, sm);
     setup(p, s);
+    griddep_wait();
+    if (blockIdx.x == 0 && threadIdx.x < sizeof(moe_pw_counters) / sizeof(uint32_t))
+        reinterpret_cast<uint32_t *>(p.ctr)[threadIdx.x] = 0u;
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int64_t a0, a1;
@@ -328,11 +333,13 @@ __global__ void __launch_bounds__(1024) ragged_offsets(RankArgs p)
     if (threadIdx.x == blockDim.x - 1) p.occ[E] = run;
 }
 
+// Launched as a programmatic dependent of the count (or scan) pass.
 __global__ void __launch_bounds__(AW * 32, AW_MIN_BLOCKS) assign_rank(RankArgs p)
 {
     extern __shared__ int32_t sm[];
     const Smem s = carve(p.g, sm);
     setup(p, s);
+    griddep_wait();
     if (p.g.mode == MOE_PW_RAGGED)
         for (int e = threadIdx.x; e <= p.g.E; e += blockDim.x) s.off[e] = p.occ[e];
     __syncthreads();
@@ -345,10 +352,13 @@ __global__ void __launch_bounds__(AW * 32, AW_MIN_BLOCKS) assign_rank(RankArgs p
 cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, int32_t *occ,
                           moe_pw_counters *ctr, void *ws, cudaStream_t st, int32_t *pool_hdr)
 {
-    cudaError_t err = cudaMemsetAsync(ctr, 0, sizeof(moe_pw_counters), st);
-    if (err != cudaSuccess) return err;
+    cudaError_t err;
     const int64_t occ_len = g.mode == MOE_PW_POOLED ? g.n_pools : int64_t(g.E) + 1;
-    if (g.T == 0) return cudaMemsetAsync(occ, 0, sizeof(int32_t) * occ_len, st);
+    if (g.T == 0) {
+        if ((err = cudaMemsetAsync(ctr, 0, sizeof(moe_pw_counters), st)) != cudaSuccess)
+            return err;
+        return cudaMemsetAsync(occ, 0, sizeof(int32_t) * occ_len, st);
+    }
 
     RankArgs p;
     memset(&p, 0, sizeof(p));
@@ -376,8 +386,19 @@ cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, i
     // with at most MAX_FUSED_CHUNKS chunks per source the rank pass sums the
     // earlier chunks' counts itself and the scan pass is skipped (pooled mode)
     p.fused_scan = g.mode == MOE_PW_POOLED && g.chunks_per_group <= MAX_FUSED_CHUNKS;
-    assign_count<<<g.n_chunks, AW * 32, smem, st>>>(p);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    // the count and rank passes start under the previous kernel's tail
+    // (programmatic dependent launch; they wait for it before any global access)
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(unsigned(g.n_chunks));
+    cfg.blockDim = dim3(AW * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((err = cudaLaunchKernelEx(&cfg, assign_count, p)) != cudaSuccess) return err;
     if (!p.fused_scan) {
         dim3 sgrid((g.NB + 31) / 32, g.n_groups);
         assign_scan<<<sgrid, 1024, 0, st>>>(p);
@@ -387,8 +408,7 @@ cudaError_t launch_assign(const Geo &g, const int32_t *idx, int32_t *slot_map, i
         ragged_offsets<<<1, 1024, 0, st>>>(p);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
-    assign_rank<<<g.n_chunks, AW * 32, smem, st>>>(p);
-    return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, assign_rank, p);
 }
 
 }  // namespace moe_pw

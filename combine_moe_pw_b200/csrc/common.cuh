@@ -296,6 +296,16 @@ __device__ __forceinline__ unsigned equal_lanes_smem(int32_t b, uint32_t *mask, 
     return b >= 0 ? mask[b] : 0u;
 }
 
+// Programmatic dependent launch: a kernel launched with
+// cudaLaunchAttributeProgrammaticStreamSerialization may start while the
+// previous kernel in its stream is finishing; griddep_wait() returns once
+// that kernel has completed and its memory is visible (at once for a normal
+// launch).  Only shared-memory set-up may come before it.
+__device__ __forceinline__ void griddep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ unsigned lanemask_lt()
 {
     unsigned m;

@@ -285,6 +285,7 @@ __global__ void __launch_bounds__(32 + BKF_THREADS) pack_bucket_kernel(PackArgs 
 {
     extern __shared__ __align__(128) unsigned char smem[];
     pack_init(p, smem, 1, blockDim.x);
+    griddep_wait();  // launched as a programmatic dependent of the assignment
     __syncthreads();
     if (threadIdx.x < 32) {
         pack_warp<LAG, false, false>(p, smem, 0, threadIdx.x, 1);
@@ -350,9 +351,21 @@ cudaError_t launch_fused_lag(const PackArgs &p, const BucketArgs &b, uint32_t bu
     cudaError_t err =
         persistent_blocks(pack_bucket_kernel<LAGT>, 32 + BKF_THREADS, smem, di, units, &blocks);
     if (err != cudaSuccess) return err;
-    if ((err = cudaMemsetAsync(&p.ctr->work, 0, sizeof(int32_t), st)) != cudaSuccess) return err;
-    pack_bucket_kernel<LAGT><<<unsigned(blocks), 32 + BKF_THREADS, smem, st>>>(p, b, bucket_off);
-    return cudaGetLastError();
+    // the zero-fill hand-out counter (counters->work) starts at 0: the
+    // assignment before this launch zeroed the counters.  The launch is a
+    // programmatic dependent of it, so its set-up overlaps the assignment's
+    // last blocks.
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(unsigned(blocks));
+    cfg.blockDim = dim3(32 + BKF_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, pack_bucket_kernel<LAGT>, p, b, bucket_off);
 }
 
 PackArgs pack_args(const Geo &g, const uint16_t *x, const int32_t *idx, const int32_t *slot_map,

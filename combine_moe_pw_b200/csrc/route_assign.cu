@@ -298,14 +298,16 @@ cudaError_t launch_ra_nv(const RouteAssignArgs &p, cudaStream_t st, int *c_out)
 }
 
 // Which form takes the batch.  The clustered launch pays off on small
-// batches: a cluster is tied to one source shard, so its blocks cannot spread
-// the route's token work evenly over the SMs (placement leaves some SMs a
-// block more than others, up to ~15% more tokens than the even share), while
-// it saves the assignment kernels' fixed latency.  Measured on B200 with 384
-// experts over 64 sources (kernels alone): at 65,536 tokens 46.5 us against
-// 50.6 us for route + assignment, at 262,144 tokens 153 us against 145 us;
-// the crossover lies near 1,024 tokens per SM.
-constexpr int64_t RA_MAX_TOKENS_PER_SM = 1024;
+// batches, where the separate kernels' fixed latency (three launches) weighs
+// most; on larger ones a cluster, tied to one source shard, cannot spread the
+// route's token work evenly over the SMs (placement leaves some SMs a block
+// more than others, up to ~15% more tokens than the even share).  Measured
+// on B200 with 384 experts over 64 sources (kernels alone, route + assignment
+// with its count and rank passes launched as programmatic dependents):
+// 19.0 / 26.6 us (clustered / separate) at 8,192 tokens, 27.1 / 28.0 at
+// 32,768, 45.5 / 44.4 at 65,536, 80.1 / 76.6 at 131,072, 149.4 / 135.7 at
+// 262,144: the crossover lies near 256 tokens per SM.
+constexpr int64_t RA_MAX_TOKENS_PER_SM = 256;
 
 bool ra_shape_ok(const Geo &g)
 {

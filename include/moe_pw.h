@@ -265,12 +265,12 @@ int moe_pw_assign_noalloc(const moe_pw_config *cfg, const int32_t *idx, int32_t 
  * form runs).  Outputs (idx, gates, slot_map, occ, the kept slots' headers in
  * pool_hdr, *counters zeroed and then the sender drops) equal those of the
  * two calls in either form:
- *   - MOE_PW_RA_CLUSTER (up to 1,024 tokens per SM): one thread-block
+ *   - MOE_PW_RA_CLUSTER (up to 256 tokens per SM): one thread-block
  *     cluster per source shard routes the shard's tokens, exchanges the
  *     per-pool counts of its blocks through distributed shared memory and
  *     ranks the choices; no global workspace is touched.  A cluster is tied
  *     to one shard, so its route work cannot spread evenly over the SMs; on
- *     larger batches that costs more than the assignment kernels' fixed
+ *     larger batches that costs more than the separate kernels' fixed
  *     latency.
  *   - MOE_PW_RA_SEPARATE: the two calls (larger batches, or a shape the
  *     clustered launch does not fit: shared memory per block, or no cluster
@@ -326,7 +326,10 @@ int moe_pw_assign_headers(const moe_pw_config *cfg, const int32_t *idx, int32_t 
  * recv_row, bucket_slot and expert_counts, and adds receiver drops and kept
  * rows to *counters: every output equals moe_pw_pack followed by
  * moe_pw_bucket.  Ragged mode: MOE_PW_EUNSUPPORTED.  T = 0: the two calls
- * are made one after the other.  Uses counters->work like moe_pw_pack.
+ * are made one after the other.  Hands the empty pool tails out through
+ * counters->work, which must be 0 on entry: the assignment call before it
+ * (moe_pw_assign_headers or moe_pw_route_assign) zeroes the counters, and
+ * nothing else may run on these counters in between.
  */
 int moe_pw_pack_bucket(const moe_pw_config *cfg, const uint16_t *x, const int32_t *idx,
                        const int32_t *slot_map, const int32_t *occ, uint16_t *pool_x,

@@ -190,23 +190,30 @@ def test_route_assign_equals_separate_launches(name):
 
 @pytest.mark.parametrize("name", list(RA_CASES))
 def test_route_assign_default_form(name):
-    """The default form: the clustered launch on these small batches where it
-    fits, else the two calls; same outputs either way."""
+    """The default form: the clustered launch up to 256 tokens per SM where
+    it fits, else the two calls; same outputs either way."""
     w = RA_CASES[name]
     cfg = mp.Config.from_workload(w)
-    expect = mp.RA_CLUSTER if name not in NOT_CLUSTER else mp.RA_SEPARATE
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    small = w.T <= 256 * sms
+    expect = mp.RA_CLUSTER if small and name not in NOT_CLUSTER else mp.RA_SEPARATE
     assert mp.moe_pw_route_assign_plan(cfg) == expect
     lg, x, s = _inputs(w)
     ref = _fresh(w, lg, x, s)
     _poison_route(ref)
     ref.route()
     ref.assign_headers()
+    st_ref = ref.stats()
     b = _fresh(w, lg, x, s)
     _poison_route(b)
+    b.counters.fill_(-1)  # zeroed by the call, whichever form runs
     b.route_assign()
+    st = b.stats()
     torch.cuda.synchronize()
     for n in RA_OUTPUTS:
         assert torch.equal(getattr(b, n), getattr(ref, n)), n
+    assert (st.sender_dropped, st.max_occ, st.error, st.kept) == (
+        st_ref.sender_dropped, st_ref.max_occ, st_ref.error, st_ref.kept)
 
 
 @pytest.mark.parametrize("name", ["k16", "E2048", "fallback_long_sources"])
@@ -224,11 +231,12 @@ def test_route_assign_step_full_parity(name):
 
 
 def test_route_assign_plan_follows_tokens_per_sm():
-    """The clustered launch up to 1,024 tokens per SM: the 65,536-token layer
-    batch takes it, the 262,144-token rack batch (above 148 * 1,024) takes the
-    separate kernels."""
+    """The clustered launch up to 256 tokens per SM: a 16,384-token batch of
+    the layer shapes takes it; the 65,536-token layer and 262,144-token rack
+    batches (above 148 * 256) take the separate kernels."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    for name in ["layer", "rack", "long"]:
-        w = synth.WORKLOADS[name]
-        expect = mp.RA_CLUSTER if w.T <= 1024 * sms else mp.RA_SEPARATE
-        assert mp.moe_pw_route_assign_plan(mp.Config.from_workload(w)) == expect, name
+    cases = [synth.WORKLOADS["layer"].with_(T=16384)] + [synth.WORKLOADS[n] for n in
+                                                         ["layer", "rack", "long"]]
+    for w in cases:
+        expect = mp.RA_CLUSTER if w.T <= 256 * sms else mp.RA_SEPARATE
+        assert mp.moe_pw_route_assign_plan(mp.Config.from_workload(w)) == expect, w.T
