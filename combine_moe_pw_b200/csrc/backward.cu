@@ -77,7 +77,10 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(
                     d0[u] = __ldcs(drow + 2 * (c0 + 32 * u));
                     d1[u] = __ldcs(drow + 2 * (c0 + 32 * u) + 1);
                 }
-            // rows in groups of eight: the loads of a group, then its arithmetic
+            // rows in groups of eight: the loads of a group, then its arithmetic.
+            // The gathered rows take the read-only path with the default cache
+            // policy, as in the forward combine (measured ~1.5% faster than
+            // evict-first streaming loads)
 #pragma unroll
             for (int jg = 0; jg < KMAX; jg += 8) {
                 uint4 y[8][BU];
@@ -88,7 +91,7 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(
 #pragma unroll
                         for (int u = 0; u < BU; ++u)
                             if (c0 + 32 * u < cpr)
-                                y[jj][u] = __ldcs(ret_x + int64_t(slot[j]) * cpr + c0 + 32 * u);
+                                y[jj][u] = __ldg(ret_x + int64_t(slot[j]) * cpr + c0 + 32 * u);
                 }
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {

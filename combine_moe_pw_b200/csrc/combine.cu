@@ -14,7 +14,10 @@
 // warp broadcasts them into registers; then each lane owns 16-byte chunks of
 // the row (8 bf16), issues the loads of all k rows for two chunks before
 // accumulating, and writes 2 x 16 bytes of fp32 per chunk.  Skipped terms are
-// warp-uniform branches.
+// warp-uniform branches.  The row loads go through the read-only data path
+// with the default cache policy: on B200 that measured 4% faster than
+// evict-first streaming loads (rack batch 1.77 against 1.85 ms; dropless
+// 2.37 against 2.47 ms), the output stores stream (evict-first).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -109,7 +112,7 @@ __global__ void MOE_PW_COMBINE_BOUNDS combine_kernel(const uint4 *__restrict__ r
                         const uint4 *row = ret_x + int64_t(slot[j]) * cpr;
 #pragma unroll
                         for (int u = 0; u < U; ++u)
-                            if (c0 + 32 * u < cpr) v[jj][u] = __ldcs(row + c0 + 32 * u);
+                            if (c0 + 32 * u < cpr) v[jj][u] = __ldg(row + c0 + 32 * u);
                     }
                 }
 #pragma unroll
