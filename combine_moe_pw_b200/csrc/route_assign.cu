@@ -50,8 +50,7 @@ namespace {
 constexpr int RA_WARPS = MOE_PW_RA_WARPS;   // warps per block
 constexpr int RA_MIN_BLOCKS = 32 / RA_WARPS;  // as the route kernel: 64 registers
 constexpr int RA_MAX_CLUSTER = 16;
-constexpr size_t RA_MAX_SMEM = 40 * 1024;  // keeps 4 blocks per SM
-
+constexpr size_t RA_MAX_SMEM = 40 * 1024;  // dynamic, beside the static; keeps 4 blocks per SM
 
 struct RouteAssignArgs {
     const float *logits;
@@ -204,7 +203,7 @@ inline void cluster_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, c
     cfg.numAttrs = 1;
 }
 
-// Cluster size per (kernel, device, sources, tokens per source): the largest
+// Cluster size per (kernel, device, batch shape): the largest
 // c <= min(16, T_s) whose blocks fit RA_MAX_SMEM and at which every source's
 // cluster is resident at once, else the smallest c that fits and can be
 // placed at all (the clusters then run in waves); 0 if none.  Cached: the
@@ -213,11 +212,14 @@ template <typename Kern>
 int pick_cluster(Kern kern, const Geo &g)
 {
     static std::mutex mu;
-    static std::map<std::tuple<const void *, int, int64_t, int64_t, int32_t, int32_t>, int> cache;
+    static std::map<std::tuple<const void *, int, int64_t, int64_t, int32_t, int32_t, int32_t>,
+                    int>
+        cache;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    // everything the shared memory per block and the grid depend on
     const auto key = std::make_tuple(reinterpret_cast<const void *>(kern), dev, int64_t(g.R),
-                                     g.T_s, g.E, g.NB);
+                                     g.T_s, g.E, g.NB, g.k);
     {
         std::lock_guard<std::mutex> lk(mu);
         const auto it = cache.find(key);
@@ -255,6 +257,9 @@ cudaError_t launch_ra(const RouteAssignArgs &p0, cudaStream_t st, int *c_out)
     auto kern = route_assign_kernel<NV, FULL, KC>;
     const Geo &g = p0.g;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (err != cudaSuccess) return err;
+    // up to RA_MAX_SMEM of dynamic shared memory beside the static arrays
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(RA_MAX_SMEM));
     if (err != cudaSuccess) return err;
     const int c = pick_cluster(kern, g);
     if (c_out) {
