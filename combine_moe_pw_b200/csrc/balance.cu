@@ -12,19 +12,26 @@
 //   dlogits[t][e] = alpha / L * p[t][e] * (f[s][e] - sum_i f[s][i] p[t][i])
 // (the routing held fixed: top-k is piecewise constant in the logits).
 //
-// Three kernels, all deterministic (fixed summation orders, integer counts):
-//   1. stats: block per (sequence, chunk of BAL_CHUNK tokens); a warp per
-//      token (the next row loaded while this one is reduced) computes the
-//      row's max and sum of exponentials (warp reductions) and adds p into
-//      per-lane accumulators of the experts it holds, tokens in order; the
-//      block sums its warps in order and writes the chunk's partial sums; the
-//      chunk's expert counts come from shared-memory atomics on idx
-//      (integers: order does not matter);
-//   2. finish: block per sequence; partial sums over chunks in order, f, P and
-//      the loss (a fixed-order block reduction over experts);
-//   3. grad (optional): a warp per token (next row in flight), p again,
-//      dot = sum_i f_i p_i by a fixed xor tree, dlogits written or added.
-// Reads the logits once per pass (HBM-bound); no tensor cores.
+// The gradient needs f, which is fixed by the routing (the counts of idx),
+// not by the probabilities, so the counts come first and one pass over the
+// logits then gives both the probability sums and the gradient: the logits
+// are read once.  Kernels, all deterministic (fixed summation orders,
+// integer counts):
+//   1. counts: block per (sequence, chunk of BAL_CHUNK tokens); the chunk's
+//      ids counted in shared memory (atomics on integers: order does not
+//      matter), then added to the sequence's counts in the workspace;
+//   2. pass: block per (sequence, chunk); a warp per token (the next row
+//      loaded while this one is reduced) computes the softmax (warp
+//      reductions) and adds p into per-lane accumulators of the experts it
+//      holds, tokens in order; the block sums its warps in order and writes
+//      the chunk's partial sums.  With the gradient it also forms
+//      dlogits = alpha / L * p * (f - dot), dot = sum_i f_i p_i by a fixed
+//      xor tree, from its sequence's f (counts times E / (k L)), written or
+//      added;
+//   3. finish: block per sequence, a thread per expert; partial sums over
+//      chunks in order, f, P and the loss (a fixed-order block reduction over
+//      experts).
+// HBM-bound (the logits in, dlogits out); no tensor cores.
 #include "common.cuh"
 
 namespace moe_pw {
@@ -40,7 +47,7 @@ struct BalArgs {
     const int32_t *idx;
     float *f, *P, *loss, *dlogits;
     float *part;      // [n_seq][chunks][E] partial probability sums
-    int32_t *cnt;     // [n_seq][chunks][E] partial assignment counts
+    int32_t *cnt;     // [n_seq][E] assignment counts (zeroed before the counts pass)
     int64_t T, L;
     int32_t E, k, chunks;
     float alpha;
@@ -89,23 +96,58 @@ __device__ __forceinline__ void softmax_row(float (&x)[NV * 4])
     for (int i = 0; i < NV * 4; ++i) x[i] = x[i] * inv;
 }
 
-template <int NV>
-__global__ void __launch_bounds__(BAL_THREADS) balance_stats(BalArgs a)
+// Token range of block (chunk c, sequence s).
+__device__ __forceinline__ void chunk_tokens(const BalArgs &a, int64_t s, int64_t c, int64_t &t0,
+                                             int64_t &t1)
 {
-    extern __shared__ float bsm[];  // [BAL_WARPS][E] probabilities, then [E] counts
-    int32_t *csm = reinterpret_cast<int32_t *>(bsm + BAL_WARPS * a.E);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t s = blockIdx.y, c = blockIdx.x;
-    const int64_t t0 = s * a.L + c * BAL_CHUNK;
-    int64_t t1 = t0 + BAL_CHUNK;
+    t0 = s * a.L + c * BAL_CHUNK;
+    t1 = t0 + BAL_CHUNK;
     if (t1 > (s + 1) * a.L) t1 = (s + 1) * a.L;
+}
+
+__global__ void __launch_bounds__(BAL_THREADS) balance_counts(BalArgs a)
+{
+    extern __shared__ int32_t csm[];  // [E]
+    const int64_t s = blockIdx.y;
+    int64_t t0, t1;
+    chunk_tokens(a, s, blockIdx.x, t0, t1);
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) csm[e] = 0;
     __syncthreads();
-    // counts of the chunk's assignments
     for (int64_t i = t0 * a.k + threadIdx.x; i < t1 * a.k; i += blockDim.x) {
         const int32_t e = a.idx[i];
         if (e >= 0 && e < a.E) atomicAdd(&csm[e], 1);
     }
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+        if (csm[e]) atomicAdd(&a.cnt[s * a.E + e], csm[e]);
+}
+
+// GRAD: also the gradient (launched as a programmatic dependent of the
+// counts pass, whose counts it reads; without it, of nothing it reads).
+template <int NV, bool GRAD>
+__global__ void __launch_bounds__(BAL_THREADS) balance_pass(BalArgs a)
+{
+    extern __shared__ float bsm[];  // [BAL_WARPS][E] probabilities
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t s = blockIdx.y, c = blockIdx.x;
+    int64_t t0, t1;
+    chunk_tokens(a, s, c, t0, t1);
+    const int E4 = a.E >> 2;
+    griddep_wait();
+    // the sequence's f, lane l holding the experts of its logits
+    float fv[NV * 4];
+    if (GRAD) {
+        const float scale_f = float(a.E) / (float(a.k) * float(a.L));
+        const int32_t *crow = a.cnt + s * a.E;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            const int q = lane + 32 * v;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+                fv[4 * v + cc] = q < E4 ? float(crow[4 * q + cc]) * scale_f : 0.0f;
+        }
+    }
+    const float g = a.alpha / float(a.L);
     // probabilities: warp w takes tokens t0 + w, t0 + w + BAL_WARPS, ...
     float acc[NV * 4];
 #pragma unroll
@@ -121,8 +163,33 @@ __global__ void __launch_bounds__(BAL_THREADS) balance_stats(BalArgs a)
         softmax_row<NV>(x);
 #pragma unroll
         for (int i = 0; i < NV * 4; ++i) acc[i] += x[i];
+        if (GRAD) {
+            float dot = 0.0f;
+#pragma unroll
+            for (int i = 0; i < NV * 4; ++i) dot = fmaf(fv[i], x[i], dot);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(FULL_MASK, dot, o);
+            float4 *row = reinterpret_cast<float4 *>(a.dlogits + t * a.E);
+#pragma unroll
+            for (int v = 0; v < NV; ++v) {
+                const int q = lane + 32 * v;
+                if (q >= E4) continue;
+                float4 d;
+                d.x = g * x[4 * v + 0] * (fv[4 * v + 0] - dot);
+                d.y = g * x[4 * v + 1] * (fv[4 * v + 1] - dot);
+                d.z = g * x[4 * v + 2] * (fv[4 * v + 2] - dot);
+                d.w = g * x[4 * v + 3] * (fv[4 * v + 3] - dot);
+                if (a.accumulate) {
+                    const float4 o = row[q];
+                    d.x += o.x;
+                    d.y += o.y;
+                    d.z += o.z;
+                    d.w += o.w;
+                }
+                row[q] = d;
+            }
+        }
     }
-    const int E4 = a.E >> 2;
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
         const int q = lane + 32 * v;
@@ -136,34 +203,36 @@ __global__ void __launch_bounds__(BAL_THREADS) balance_stats(BalArgs a)
         float sum = 0.0f;
         for (int w = 0; w < BAL_WARPS; ++w) sum += bsm[w * a.E + e];
         a.part[base + e] = sum;
-        a.cnt[base + e] = csm[e];
     }
 }
 
-__global__ void __launch_bounds__(BAL_THREADS) balance_finish(BalArgs a)
+// 512 threads: one expert per thread for E <= 512, so that all of a thread's
+// chunk loads are in flight together (with 256 threads the second expert's
+// loads waited for the first's: the pass took ~23 us for 64 sequences).
+constexpr int FIN_THREADS = 512;
+
+// Launched as a programmatic dependent of the probability pass.
+__global__ void __launch_bounds__(FIN_THREADS) balance_finish(BalArgs a)
 {
-    __shared__ float red[BAL_THREADS];
+    __shared__ float red[FIN_THREADS];
     const int64_t s = blockIdx.x;
     const float scale_f = float(a.E) / (float(a.k) * float(a.L));
-    float mine = 0.0f;  // this thread's experts e = tid, tid + 256, ... in order
+    griddep_wait();
+    float mine = 0.0f;  // this thread's experts e = tid, tid + 512, ... in order
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
         float sum = 0.0f;
-        int64_t n = 0;
         // chunks in order; unrolled so the loads of 8 chunks are in flight together
 #pragma unroll 8
-        for (int c = 0; c < a.chunks; ++c) {
-            sum += __ldcg(a.part + (s * a.chunks + c) * a.E + e);
-            n += __ldcg(a.cnt + (s * a.chunks + c) * a.E + e);
-        }
+        for (int c = 0; c < a.chunks; ++c) sum += __ldcg(a.part + (s * a.chunks + c) * a.E + e);
         const float P = sum / float(a.L);
-        const float f = float(n) * scale_f;
+        const float f = float(__ldcg(a.cnt + s * a.E + e)) * scale_f;
         a.P[s * a.E + e] = P;
         a.f[s * a.E + e] = f;
         mine = fmaf(f, P, mine);
     }
     red[threadIdx.x] = mine;
     __syncthreads();
-    for (int h = BAL_THREADS / 2; h > 0; h >>= 1) {
+    for (int h = FIN_THREADS / 2; h > 0; h >>= 1) {
         if (threadIdx.x < h) red[threadIdx.x] += red[threadIdx.x + h];
         __syncthreads();
     }
@@ -171,93 +240,39 @@ __global__ void __launch_bounds__(BAL_THREADS) balance_finish(BalArgs a)
 }
 
 template <int NV>
-__global__ void __launch_bounds__(BAL_THREADS) balance_grad(BalArgs a)
-{
-    const int lane = threadIdx.x & 31;
-    const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarp = (int64_t(gridDim.x) * blockDim.x) >> 5;
-    const int E4 = a.E >> 2;
-    // the next token's logits and its sequence's f row are loaded while the
-    // current token is worked on
-    float nx[NV * 4], nf[NV * 4];
-    auto load_f = [&](int64_t t, float (&fo)[NV * 4]) {
-        const float4 *frow = reinterpret_cast<const float4 *>(a.f + (t / a.L) * a.E);
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            const int q = lane + 32 * v;
-            const float4 f4 = q < E4 ? __ldg(frow + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-            fo[4 * v + 0] = f4.x;
-            fo[4 * v + 1] = f4.y;
-            fo[4 * v + 2] = f4.z;
-            fo[4 * v + 3] = f4.w;
-        }
-    };
-    if (warp < a.T) {
-        load_row<NV>(a, warp, lane, nx);
-        load_f(warp, nf);
-    }
-    for (int64_t t = warp; t < a.T; t += nwarp) {
-        float x[NV * 4], fv[NV * 4];
-#pragma unroll
-        for (int i = 0; i < NV * 4; ++i) {
-            x[i] = nx[i];
-            fv[i] = nf[i];
-        }
-        if (t + nwarp < a.T) {
-            load_row<NV>(a, t + nwarp, lane, nx);
-            load_f(t + nwarp, nf);
-        }
-        softmax_row<NV>(x);
-        float dot = 0.0f;
-#pragma unroll
-        for (int i = 0; i < NV * 4; ++i) dot = fmaf(fv[i], x[i], dot);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(FULL_MASK, dot, o);
-        const float g = a.alpha / float(a.L);
-        float4 *row = reinterpret_cast<float4 *>(a.dlogits + t * a.E);
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            const int q = lane + 32 * v;
-            if (q >= E4) continue;
-            float4 d;
-            d.x = g * x[4 * v + 0] * (fv[4 * v + 0] - dot);
-            d.y = g * x[4 * v + 1] * (fv[4 * v + 1] - dot);
-            d.z = g * x[4 * v + 2] * (fv[4 * v + 2] - dot);
-            d.w = g * x[4 * v + 3] * (fv[4 * v + 3] - dot);
-            if (a.accumulate) {
-                const float4 o = row[q];
-                d.x += o.x;
-                d.y += o.y;
-                d.z += o.z;
-                d.w += o.w;
-            }
-            row[q] = d;
-        }
-    }
-}
-
-template <int NV>
 cudaError_t launch_nv(const BalArgs &a, int64_t n_seq, cudaStream_t st)
 {
-    DevInfo di;
-    if (dev_info(&di) != 0) return cudaErrorUnknown;
-    const size_t smem = sizeof(float) * BAL_WARPS * a.E + sizeof(int32_t) * a.E;
     cudaError_t err;
+    if ((err = cudaMemsetAsync(a.cnt, 0, sizeof(int32_t) * size_t(n_seq) * a.E, st)) !=
+        cudaSuccess)
+        return err;
+    const dim3 grid(unsigned(a.chunks), unsigned(n_seq));
+    balance_counts<<<grid, BAL_THREADS, sizeof(int32_t) * a.E, st>>>(a);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    // the probability pass and the finish start under their predecessor's
+    // tail (programmatic dependent launches; each waits for it before
+    // reading its outputs)
+    const size_t smem = sizeof(float) * BAL_WARPS * a.E;
+    auto pass = a.dlogits ? balance_pass<NV, true> : balance_pass<NV, false>;
     if (smem > 48 * 1024 &&
-        (err = cudaFuncSetAttribute(balance_stats<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (err = cudaFuncSetAttribute(pass, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     int(smem))) != cudaSuccess)
         return err;
-    balance_stats<NV><<<dim3(unsigned(a.chunks), unsigned(n_seq)), BAL_THREADS, smem, st>>>(a);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    balance_finish<<<unsigned(n_seq), BAL_THREADS, 0, st>>>(a);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if (a.dlogits) {
-        int64_t blocks = (a.T + BAL_WARPS - 1) / BAL_WARPS;
-        if (blocks > int64_t(di.sms) * 8) blocks = int64_t(di.sms) * 8;
-        balance_grad<NV><<<unsigned(blocks), BAL_THREADS, 0, st>>>(a);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    }
-    return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.stream = st;
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(BAL_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    if ((err = cudaLaunchKernelEx(&cfg, pass, a)) != cudaSuccess) return err;
+    cfg.gridDim = dim3(unsigned(n_seq));
+    cfg.blockDim = dim3(FIN_THREADS);
+    cfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cfg, balance_finish, a);
 }
 
 }  // namespace
@@ -267,7 +282,7 @@ int64_t balance_ws_bytes(int64_t T, int64_t L, int32_t E)
     if (L <= 0) return 0;
     const int64_t chunks = (L + BAL_CHUNK - 1) / BAL_CHUNK;
     const int64_t n = (T / L) * chunks * E;
-    return align256(4 * n) + align256(4 * n);
+    return align256(4 * n) + align256(4 * (T / L) * int64_t(E));
 }
 
 cudaError_t launch_balance(const Geo &g, int64_t seq_len, float alpha, const float *logits,
