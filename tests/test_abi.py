@@ -168,3 +168,31 @@ def test_fused_dispatch_entries_validate_before_any_launch(lib):
     with pytest.raises(mp.MoePwError) as ei:
         mp.moe_pw_pack_bucket(tiny, odd + 8, *[good] * 9, stream=0)  # x needs 16 bytes
     assert ei.value.code == mp.MOE_PW_EUNSUPPORTED
+
+
+def test_route_assign_entries_validate_before_any_launch(lib):
+    """moe_pw_route_assign(_form): pooled mode only, a known form, buffers
+    present and aligned, a large enough workspace: all checked on the host."""
+    tiny = mp.Config.from_workload(synth.WORKLOADS["tiny"])
+    ragged = mp.Config(**{**tiny.__dict__, "mode": synth.MODE_RAGGED, "cf_send_pct": 0,
+                          "cf_recv_pct": 0})
+    good, odd = 1 << 20, (1 << 20) + 4  # placeholder addresses, never dereferenced
+    ws = mp.moe_pw_plan(tiny).workspace_bytes
+    args = [good] * 7  # logits, idx, gates, slot_map, occ, pool_hdr, counters
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_route_assign_form(ragged, -1, *args, good, ws, stream=0)
+    assert ei.value.code == mp.MOE_PW_EUNSUPPORTED
+    for form in (-2, 2, 7):
+        with pytest.raises(mp.MoePwError) as ei:
+            mp.moe_pw_route_assign_form(tiny, form, *args, good, ws, stream=0)
+        assert ei.value.code == mp.MOE_PW_EINVAL
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_route_assign_form(tiny, -1, good, good, good, None, good, good, good, good, ws,
+                                    stream=0)  # no slot_map
+    assert ei.value.code == mp.MOE_PW_EINVAL
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_route_assign_form(tiny, -1, *args, good, ws - 256, stream=0)  # workspace short
+    assert ei.value.code == mp.MOE_PW_EINVAL
+    with pytest.raises(mp.MoePwError) as ei:
+        mp.moe_pw_route_assign_form(tiny, -1, odd + 8, *args[1:], good, ws, stream=0)
+    assert ei.value.code == mp.MOE_PW_EUNSUPPORTED  # logits need 16 bytes
