@@ -783,7 +783,7 @@ def main():
             if ev is not None:
                 ev[1].record(stream)
             mp.moe_pw_expert(cfg, b.d_ret, b.pool_hdr, b.recv_row, b.scale, b.d_pool,
-                             b.d_pool_hdr, stream)
+                             b.d_pool_hdr, b.counters, stream)
             if ev is not None:
                 ev[2].record(stream)
             mp.moe_pw_dispatch_backward(cfg, b.d_pool, b.recv_row, b.slot_map, b.dx, b.counters,

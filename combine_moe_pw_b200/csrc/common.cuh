@@ -88,10 +88,12 @@ cudaError_t launch_bucket(const Geo &g, const int32_t *pool_hdr, const int32_t *
                           moe_pw_counters *ctr, cudaStream_t st, uint32_t wave_mask = ~0u);
 // ep (optional): the return pools of every GPU; results then go to the
 // source's GPU, only for waves in wave_mask.
+// ctr: MOE_PW_DEVERR_TIMEOUT of the bulk-copy kernel (nullptr: the kernel
+// without waits runs).
 cudaError_t launch_expert(const Geo &g, const uint16_t *pool_x, const int32_t *pool_hdr,
                           const int32_t *recv_row, const float *scale, uint16_t *ret_x,
-                          int32_t *ret_hdr, cudaStream_t st, const EpRows *ep = nullptr,
-                          uint32_t wave_mask = ~0u);
+                          int32_t *ret_hdr, moe_pw_counters *ctr, cudaStream_t st,
+                          const EpRows *ep = nullptr, uint32_t wave_mask = ~0u);
 cudaError_t launch_combine(const Geo &g, const uint16_t *ret_x, const int32_t *ret_hdr,
                            const int32_t *slot_map, const float *gates, float *out,
                            moe_pw_counters *ctr, cudaStream_t st);

@@ -6,8 +6,20 @@
 // all-to-all ("535B大模型“直播”训练三个月", MoE / token dropping section) would
 // carry back.  Slots the receiver did not keep return zeros and header -1.
 //
-// Streaming kernel over slots: one warp per slot row, 16-byte loads and
-// stores, four chunks in flight per lane.
+// Two kernels.  expert_ring_kernel (one GPU, rows up to what a block's
+// shared memory holds) streams the rows through shared memory with bulk
+// copies: persistent, RING_WARPS warps per block; warp w walks slots
+// w, w + GW, ... (GW warps in the grid) through a ring of RING_NS row
+// buffers.  Lane 0 loads the kept rows of the next slots ahead
+// (cp.async.bulk, evict-first), the lanes scale the current row in place,
+// and lane 0 writes it back with one bulk store; a slot the receiver did not
+// keep gets one bulk store from a zero row.  A row buffer is reloaded once
+// the bulk store of its previous row has read it.  Measured on the
+// 262,144-token rack batch (14.2 GB of return rows written, 9.1 GB of kept
+// rows read): 3.59 ms, against 3.89 ms for expert_kernel's 16-byte loads and
+// stores.  expert_kernel (expert-parallel runs, whose results go to peer
+// GPUs, and wider rows): one warp per slot row, 16-byte loads and stores,
+// four chunks in flight per lane.
 #include <cuda_bf16.h>
 
 #include <cstring>
@@ -42,6 +54,7 @@ struct ExpertArgs {
     uint32_t wave_mask;
     Geo geo;
     EpRows ep;
+    moe_pw_counters *ctr;  // expert_ring_kernel: MOE_PW_DEVERR_TIMEOUT
 };
 
 template <bool EP>
@@ -111,18 +124,128 @@ __global__ void __launch_bounds__(256) expert_kernel(ExpertArgs a)
     if (EP) __threadfence_system();  // peer stores ordered before any later signal
 }
 
+
+constexpr int RING_WARPS = 4, RING_NS = 3;
+constexpr uint32_t RING_WAIT_LIMIT = 1u << 22;
+// barriers [RING_WARPS][RING_NS] in the first 128 bytes, a zero row, then
+// each warp's RING_NS row buffers
+constexpr size_t RING_BAR_BYTES = 128;
+static_assert(RING_WARPS * RING_NS * 8 <= RING_BAR_BYTES, "barrier region");
+
+inline size_t ring_smem_bytes(int cpr)
+{
+    return RING_BAR_BYTES + size_t(cpr) * 16 * (1 + RING_WARPS * RING_NS);
+}
+
+__device__ __forceinline__ bool keeps_slot(const ExpertArgs &a, int64_t slot, int32_t &e)
+{
+    e = a.pool_hdr[slot];
+    return a.recv_row[slot] >= 0 && e >= 0 && e < a.E;
+}
+
+__global__ void __launch_bounds__(RING_WARPS * 32) expert_ring_kernel(ExpertArgs a)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int cpr = a.cpr;
+    const uint32_t rb = uint32_t(cpr) * 16u;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem) + wib * RING_NS;
+    unsigned char *zero = smem + RING_BAR_BYTES;
+    unsigned char *ring = zero + rb + size_t(wib) * RING_NS * rb;
+    for (int c = threadIdx.x; c < cpr; c += blockDim.x)
+        reinterpret_cast<uint4 *>(zero)[c] = make_uint4(0, 0, 0, 0);
+    if (lane == 0)
+        for (int s = 0; s < RING_NS; ++s) mbar_init(&bar[s], 1);
+    fence_init_and_proxy();
+    __syncthreads();
+
+    const int64_t gw = int64_t(blockIdx.x) * RING_WARPS + wib;
+    const int64_t GW = int64_t(gridDim.x) * RING_WARPS;
+    const int64_t n = a.n_slots;
+    const uint64_t pol = policy_evict_first();
+    // step i of this warp is slot gw + i * GW; a kept row uses stage i % RING_NS
+    uint32_t armed = 0;  // lane 0: stages with a load in flight
+    auto issue = [&](int64_t i) {
+        const int64_t slot = gw + i * GW;
+        int32_t e;
+        if (slot >= n || !keeps_slot(a, slot, e)) return;
+        const int s = int(i % RING_NS);
+        mbar_arrive_expect_tx(&bar[s], rb);
+        bulk_g2s(ring + size_t(s) * rb, a.pool_x + slot * cpr, rb, &bar[s], pol);
+        armed |= 1u << s;
+    };
+    if (lane == 0)
+        for (int i = 0; i < RING_NS; ++i) issue(i);
+
+    uint32_t phase = 0;  // parity of each stage's next load completion
+    bool ok = true;
+    int64_t i = 0;
+    for (int64_t slot = gw; slot < n; slot += GW, ++i) {
+        const int s = int(i % RING_NS);
+        int32_t e;
+        const bool keep = keeps_slot(a, slot, e);
+        uint4 *dst = a.ret_x + slot * cpr;
+        if (keep) {
+            const bool landed = mbar_wait_bounded(&bar[s], (phase >> s) & 1u, RING_WAIT_LIMIT);
+            if (!__all_sync(FULL_MASK, landed)) {
+                ok = false;
+                break;
+            }
+            phase ^= 1u << s;
+            armed &= ~(1u << s);
+            const float sc = a.scale[e];
+            uint4 *row = reinterpret_cast<uint4 *>(ring + size_t(s) * rb);
+            for (int c = lane; c < cpr; c += 32) {
+                const uint4 v = row[c];
+                uint4 y;
+                y.x = scale_pair(v.x, sc);
+                y.y = scale_pair(v.y, sc);
+                y.z = scale_pair(v.z, sc);
+                y.w = scale_pair(v.w, sc);
+                row[c] = y;
+            }
+            // the lanes' writes, then the bulk store that reads them
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) bulk_s2g(dst, row, rb, pol);
+        } else if (lane == 0) {
+            bulk_s2g(dst, zero, rb, pol);
+        }
+        if (lane == 0) {
+            a.ret_hdr[slot] = keep ? e : -1;
+            bulk_commit();
+            // the previous step's row has been read out of its stage: load
+            // the row RING_NS steps after it there
+            if (i > 0) {
+                bulk_wait_read<1>();
+                issue(i - 1 + RING_NS);
+            }
+        }
+        __syncwarp();
+    }
+    if (lane == 0) {
+        if (!ok) {
+            set_error(a.ctr, MOE_PW_DEVERR_TIMEOUT);
+            // loads still in flight write this CTA's shared memory: wait for
+            // each (bounded) before the CTA retires
+            for (int s = 0; s < RING_NS; ++s)
+                if ((armed >> s) & 1u)
+                    mbar_wait_bounded(&bar[s], (phase >> s) & 1u, RING_WAIT_LIMIT);
+        }
+        bulk_wait_all();
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_expert(const Geo &g, const uint16_t *pool_x, const int32_t *pool_hdr,
                           const int32_t *recv_row, const float *scale, uint16_t *ret_x,
-                          int32_t *ret_hdr, cudaStream_t st, const EpRows *ep,
-                          uint32_t wave_mask)
+                          int32_t *ret_hdr, moe_pw_counters *ctr, cudaStream_t st,
+                          const EpRows *ep, uint32_t wave_mask)
 {
     if (g.n_slots == 0) return cudaSuccess;
     DevInfo di;
     if (dev_info(&di) != 0) return cudaErrorUnknown;
-    int64_t blocks = (g.n_slots + 7) / 8;
-    if (blocks > int64_t(di.sms) * 8) blocks = int64_t(di.sms) * 8;
     ExpertArgs a;
     a.pool_x = reinterpret_cast<const uint4 *>(pool_x);
     a.pool_hdr = pool_hdr;
@@ -135,6 +258,33 @@ cudaError_t launch_expert(const Geo &g, const uint16_t *pool_x, const int32_t *p
     a.E = g.E;
     a.wave_mask = wave_mask;
     a.geo = g;
+    a.ctr = ctr;
+    const size_t ring_smem = ring_smem_bytes(a.cpr);
+    if (!ep && ctr && ring_smem <= size_t(di.smem_optin)) {
+        std::memset(&a.ep, 0, sizeof(a.ep));
+        cudaError_t err = cudaFuncSetAttribute(
+            expert_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(ring_smem));
+        if (err != cudaSuccess) return err;
+        int per_sm = 0;
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_ring_kernel,
+                                                            RING_WARPS * 32, ring_smem);
+        if (err != cudaSuccess) return err;
+        // On 6 KB rows, 2 blocks per SM measured best (96 KB of loads
+        // ahead per SM; 3 stages per warp beat 2 and 4, and one block of 6
+        // stages was slower still).  Narrower rows take more blocks, for
+        // about the same bytes ahead, as far as they fit.
+        const size_t ahead = size_t(RING_WARPS) * (RING_NS - 1) * a.cpr * 16;
+        const int want = int((98304 + ahead - 1) / ahead);
+        if (per_sm > want) per_sm = want;
+        if (per_sm < 1) per_sm = 1;
+        int64_t blocks = int64_t(di.sms) * per_sm;
+        const int64_t need = (g.n_slots + RING_WARPS - 1) / RING_WARPS;
+        if (blocks > need) blocks = need;
+        expert_ring_kernel<<<unsigned(blocks), RING_WARPS * 32, ring_smem, st>>>(a);
+        return cudaGetLastError();
+    }
+    int64_t blocks = (g.n_slots + 7) / 8;
+    if (blocks > int64_t(di.sms) * 8) blocks = int64_t(di.sms) * 8;
     if (ep) {
         a.ep = *ep;
         expert_kernel<true><<<unsigned(blocks), 256, 0, st>>>(a);

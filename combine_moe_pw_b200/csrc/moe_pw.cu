@@ -371,17 +371,20 @@ int moe_pw_dispatch(const moe_pw_config *cfg, const uint16_t *x, const int32_t *
 
 int moe_pw_expert(const moe_pw_config *cfg, const uint16_t *pool_x, const int32_t *pool_hdr,
                   const int32_t *recv_row, const float *scale, uint16_t *ret_x, int32_t *ret_hdr,
-                  cudaStream_t stream)
+                  moe_pw_counters *counters, cudaStream_t stream)
 {
     Geo g;
     int rc = make_geo(cfg, &g);
     if (rc != MOE_PW_OK) return rc;
     if (g.n_slots == 0) return MOE_PW_OK;
-    if (!pool_x || !pool_hdr || !recv_row || !scale || !ret_x || !ret_hdr) return MOE_PW_EINVAL;
+    if (!pool_x || !pool_hdr || !recv_row || !scale || !ret_x || !ret_hdr || !counters)
+        return MOE_PW_EINVAL;
     if (!aligned(pool_x, 16) || !aligned(ret_x, 16) || !aligned(pool_hdr, 4) ||
-        !aligned(recv_row, 4) || !aligned(scale, 4) || !aligned(ret_hdr, 4))
+        !aligned(recv_row, 4) || !aligned(scale, 4) || !aligned(ret_hdr, 4) ||
+        !aligned(counters, 8))
         return MOE_PW_EUNSUPPORTED;
-    return cuda_rc(launch_expert(g, pool_x, pool_hdr, recv_row, scale, ret_x, ret_hdr, stream));
+    return cuda_rc(launch_expert(g, pool_x, pool_hdr, recv_row, scale, ret_x, ret_hdr, counters,
+                                 stream));
 }
 
 int moe_pw_combine(const moe_pw_config *cfg, const uint16_t *ret_x, const int32_t *ret_hdr,
@@ -744,7 +747,7 @@ extern "C" int moe_pw_step_host(const moe_pw_config *cfg, const float *h_logits,
             return rc;
     }
     if ((rc = moe_pw_expert(cfg, dev->pool_x, dev->pool_hdr, dev->recv_row, dev->scale,
-                            dev->ret_x, dev->ret_hdr, compute)) != MOE_PW_OK)
+                            dev->ret_x, dev->ret_hdr, dev->counters, compute)) != MOE_PW_OK)
         return rc;
     if ((rc = moe_pw_combine(cfg, dev->ret_x, dev->ret_hdr, dev->slot_map, dev->gates, dev->out,
                              dev->counters, compute)) != MOE_PW_OK)
@@ -899,7 +902,8 @@ int moe_pw_ep_expert(const moe_pw_config *cfg, const moe_pw_ep *ep, const moe_pw
         return MOE_PW_EUNSUPPORTED;
     EpRows rows;
     if ((rc = ep_rows(g, peers->ret_x, peers->ret_hdr, &rows)) != MOE_PW_OK) return rc;
-    return cuda_rc(launch_expert(g, recv_x, recv_hdr, recv_row, scale, nullptr, nullptr, stream,
+    return cuda_rc(launch_expert(g, recv_x, recv_hdr, recv_row, scale, nullptr, nullptr, nullptr,
+                                 stream,
                                  &rows, wave_bits(g, wave_mask)));
 }
 

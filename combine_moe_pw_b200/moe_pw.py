@@ -109,7 +109,7 @@ SIGNATURES = {
     "moe_pw_assign_headers": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "moe_pw_pack_bucket": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_dispatch": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
-    "moe_pw_expert": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+    "moe_pw_expert": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_combine": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_combine_bf16": [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "moe_pw_combine_bf16_rows": [_CFG, _VP, _VP, _VP, _VP, _I64, _I64, _VP, _VP, _VP],
@@ -330,11 +330,12 @@ def moe_pw_dispatch(cfg, x, idx, slot_map, occ, pool_x, pool_hdr, recv_row, buck
         _ptr(workspace), wsb, _stream(stream)))
 
 
-def moe_pw_expert(cfg, pool_x, pool_hdr, recv_row, scale, ret_x, ret_hdr, stream=None):
+def moe_pw_expert(cfg, pool_x, pool_hdr, recv_row, scale, ret_x, ret_hdr, counters,
+                  stream=None):
     c = _cfg(cfg)
     _check("moe_pw_expert", load_library().moe_pw_expert(
         ctypes.byref(c), _ptr(pool_x), _ptr(pool_hdr), _ptr(recv_row), _ptr(scale), _ptr(ret_x),
-        _ptr(ret_hdr), _stream(stream)))
+        _ptr(ret_hdr), _ptr(counters), _stream(stream)))
 
 
 def moe_pw_combine(cfg, ret_x, ret_hdr, slot_map, gates, out, counters, stream=None):
@@ -626,7 +627,7 @@ class Buffers:
 
     def expert(self, stream=None):
         moe_pw_expert(self.cfg, self.pool_x, self.pool_hdr, self.recv_row, self.scale,
-                      self.ret_x, self.ret_hdr, stream)
+                      self.ret_x, self.ret_hdr, self.counters, stream)
 
     def combine(self, stream=None):
         moe_pw_combine(self.cfg, self.ret_x, self.ret_hdr, self.slot_map, self.gates, self.out,
@@ -658,7 +659,7 @@ class Buffers:
                                 self.idx, self.gates, self.d_ret, self.dgates, self.dlogits,
                                 self.counters, stream)
         moe_pw_expert(self.cfg, self.d_ret, self.pool_hdr, self.recv_row, self.scale,
-                      self.d_pool, self.d_pool_hdr, stream)
+                      self.d_pool, self.d_pool_hdr, self.counters, stream)
         moe_pw_dispatch_backward(self.cfg, self.d_pool, self.recv_row, self.slot_map, self.dx,
                                  self.counters, stream)
 

@@ -350,11 +350,14 @@ int moe_pw_dispatch(const moe_pw_config *cfg, const uint16_t *x, const int32_t *
  * Per-expert op and return layout (stand-in for the expert network; huxiu:
  * results return by a second all-to-all).  For every slot: if the receiver
  * kept it (recv_row >= 0), ret_x = bf16_rn(scale[e] * pool_x) and ret_hdr = e;
- * otherwise ret_x = 0 and ret_hdr = -1.
+ * otherwise ret_x = 0 and ret_hdr = -1.  On one GPU the rows stream through
+ * shared memory by bulk copies with bounded waits: a wait that gives up sets
+ * MOE_PW_DEVERR_TIMEOUT in counters->error (device memory, 8-byte aligned;
+ * nothing else in *counters is touched).
  */
 int moe_pw_expert(const moe_pw_config *cfg, const uint16_t *pool_x, const int32_t *pool_hdr,
                   const int32_t *recv_row, const float *scale, uint16_t *ret_x,
-                  int32_t *ret_hdr, cudaStream_t stream);
+                  int32_t *ret_hdr, moe_pw_counters *counters, cudaStream_t stream);
 
 /*
  * Combine (section 四: a dropped assignment leaves the token, so its term is

@@ -98,7 +98,7 @@ def test_null_pointers_rejected_before_any_launch(lib):
     cfg = mp.Config.from_workload(synth.WORKLOADS["tiny"])
     for fn, args in [
         (mp.moe_pw_route, (0, 0, 0)),
-        (mp.moe_pw_expert, (0, 0, 0, 0, 0, 0)),
+        (mp.moe_pw_expert, (0, 0, 0, 0, 0, 0, 0)),
         (mp.moe_pw_combine, (0, 0, 0, 0, 0, 0)),
     ]:
         with pytest.raises(mp.MoePwError) as ei:
