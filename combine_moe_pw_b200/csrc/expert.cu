@@ -16,8 +16,8 @@
 // keep gets one bulk store from a zero row.  A row buffer is reloaded once
 // the bulk store of its previous row has read it.  Measured on the
 // 262,144-token rack batch (14.2 GB of return rows written, 9.1 GB of kept
-// rows read): 3.59 ms, against 3.89 ms for expert_kernel's 16-byte loads and
-// stores.  expert_kernel (expert-parallel runs, whose results go to peer
+// rows read): 3.59-3.63 ms, against 3.89 ms for expert_kernel's 16-byte
+// loads and stores.  expert_kernel (expert-parallel runs, whose results go to peer
 // GPUs, and wider rows): one warp per slot row, 16-byte loads and stores,
 // four chunks in flight per lane.
 #include <cuda_bf16.h>
@@ -123,7 +123,6 @@ __global__ void __launch_bounds__(256) expert_kernel(ExpertArgs a)
     }
     if (EP) __threadfence_system();  // peer stores ordered before any later signal
 }
-
 
 constexpr int RING_WARPS = 4, RING_NS = 3;
 constexpr uint32_t RING_WAIT_LIMIT = 1u << 22;
