@@ -58,6 +58,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
     ap.add_argument("--cpu-sample-sources", type=int, default=16)
+    ap.add_argument("--cpu-sample-reps", type=int, default=3)
     ap.add_argument("--no-graph", action="store_true",
                     help="skip the CUDA-graph timing of the whole forward step")
     ap.add_argument("--no-backward", action="store_true",
@@ -387,21 +388,24 @@ def host_cpu():
     return {"host_cores": os.cpu_count(), "cpu_model": model}
 
 
-def cpu_oracle_sample(w, n_src: int):
+def cpu_oracle_sample(w, n_src: int, reps: int = 1):
     """Time the CPU oracle (single thread) on the first n_src source shards of
-    the batch: route, assignment, pack, bucketing, expert op and combine."""
+    the batch: route, assignment, pack, bucketing, expert op and combine, run
+    `reps` times on the same inputs.  Returns (assignments routed, seconds)."""
     import oracle
     from combine_moe_pw_b200 import synth
-    T = n_src * (w.T // w.R) if w.mode == 0 else n_src * (w.T // w.R)
+    T = n_src * (w.T // w.R)
     ws = w.with_(T=T)
     lg, x, s = synth.logits(ws), synth.x_bf16(ws), synth.scales(w)
-    t0 = time.perf_counter()
-    if w.mode == 0:
-        oracle.run(w, lg, x, s, T=T)
-    else:
-        oracle.run(ws, lg, x, s)
-    dt = time.perf_counter() - t0
-    return T * w.k, dt
+    dt = 0.0
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        if w.mode == 0:
+            oracle.run(w, lg, x, s, T=T)
+        else:
+            oracle.run(ws, lg, x, s)
+        dt += time.perf_counter() - t0
+    return reps * T * w.k, dt
 
 
 def run_reference(a):
@@ -887,11 +891,12 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        u, dt = cpu_oracle_sample(base, a.cpu_sample_sources)
+        u, dt = cpu_oracle_sample(base, a.cpu_sample_sources, a.cpu_sample_reps)
         cpu = {"value": u / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"first {a.cpu_sample_sources} of {base.R} source shards "
                          f"({a.cpu_sample_sources * (base.T // base.R)} tokens) of the {base.name} "
-                         f"batch, whole oracle path (route..combine), one thread, {dt:.1f} s",
+                         f"batch, whole oracle path (route..combine), one thread, "
+                         f"{a.cpu_sample_reps} runs on the same inputs, {dt:.1f} s in all",
                **host_cpu()}
 
     if rank == 0:
