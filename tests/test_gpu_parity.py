@@ -175,9 +175,10 @@ SMALL_CASES = {
     "min_width": TINY.with_(D=8),
     "odd_width": TINY.with_(D=136),
     # 8928: the widest row the expert op streams through its shared-memory
-    # ring (13 row buffers in one block's 227 KB); 12288 takes its
-    # register-copy kernel
+    # ring (13 row buffers in one block's 227 KB); 6144: one ring block per
+    # SM (156 KB); 12288 takes its register-copy kernel
     "ring_max_width": TINY.with_(T=256, D=8928),
+    "ring_one_block_per_sm": TINY.with_(T=256, D=6144),
     "max_width": TINY.with_(T=256, D=12288),
     "single_pool": TINY.with_(R=1, L=16, W=1, P=16, T=512, cf_send_pct=30),
     "ragged_tail": TINY.with_(T=8 * 37, seq_len=37),
