@@ -30,6 +30,7 @@ CASES = {
     "wide_E": SMALL_CASES["wide_E"],
     "E2048": SMALL_CASES["E2048"],              # 1024 items: several per block
     "pages_ranks_small": SMALL_CASES["pages_ranks_small"],
+    "max_P": SMALL_CASES["max_P"],                # 32 experts per bucket item
     # 2 sources of 10,000 tokens: ~29,000 positions per item, 8 tiles
     "long_sources": SMALL_CASES["long_sources"],
     "multi_tile_ragged_tail": synth.Workload("multi_tile", T=8 * 5001, R=8, L=6, W=3, P=2, k=8,

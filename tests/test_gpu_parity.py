@@ -195,6 +195,9 @@ SMALL_CASES = {
                             logit_kind=synth.LOGIT_IID),
     "pages_ranks_small": synth.Workload("pages_ranks_small", T=64 * 64, R=64, L=6, W=3, P=2, k=8,
                                         D=256, seq_len=1024, logit_kind=synth.LOGIT_SEQBIAS),
+    # 32 experts per wave, the most a receiver bucket item takes
+    "max_P": synth.Workload("max_P", T=2 * 512, R=2, L=64, W=2, P=32, k=8, D=64, seq_len=512,
+                            logit_kind=synth.LOGIT_ZIPF, cf_send_pct=80, cf_recv_pct=90),
 }
 
 
