@@ -14,12 +14,13 @@ import pytest
 
 import oracle
 from combine_moe_pw_b200 import synth
-from fuzz_cases import random_workload
+from fuzz_cases import random_wide_workload, random_workload
 from test_gpu_parity import _inputs, check_full, run_gpu
 
 N_CASES = 24
 N_BACKWARD = 12
 N_PROJECT = 12
+N_WIDE = 8
 
 
 def test_draws_are_varied():
@@ -27,12 +28,25 @@ def test_draws_are_varied():
     assert len({(w.R, w.L, w.W, w.P, w.k, w.D) for w in ws}) > N_CASES // 2
     assert any(w.mode == synth.MODE_RAGGED for w in ws)
     assert any(w.cf_send_pct and w.cf_send_pct < 100 for w in ws)
+    wide = [random_wide_workload(i) for i in range(N_WIDE)]
+    assert len({w.D for w in wide}) > 1 and len({(w.R, w.L, w.k) for w in wide}) > N_WIDE // 2
 
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("i", range(N_CASES))
 def test_random_config_full_parity(i):
     w = random_workload(i)
+    lg, x, s = _inputs(w)
+    b, st = run_gpu(w, lg, x, s)
+    check_full(w, lg, x, s, b, st)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("i", range(N_WIDE))
+def test_random_wide_config_full_parity(i):
+    """Seeded draws at 1024 to 6144 bf16 per row (the pack's and the expert
+    op's shared-memory rings then hold few rows per block)."""
+    w = random_wide_workload(i)
     lg, x, s = _inputs(w)
     b, st = run_gpu(w, lg, x, s)
     check_full(w, lg, x, s, b, st)
