@@ -1,8 +1,9 @@
 """The route kernel alone against the oracle's route, on shapes the
 end-to-end parity cases do not reach: 128, 256, 320 and 384 experts, odd
-token counts, a single token, k = 6 with 384 experts, many exact ties (tokens
-with more than 32 logits at or above the threshold take the exact rounds),
-all-equal logits, signed zeros and masked (-inf) experts.  Ids bit for bit,
+token counts, a single token, k = 6 with 384 experts, many exact ties (ranked
+among the candidates, or, with more than 32 logits at or above the
+threshold, by the exact rounds), all-equal logits, signed zeros and masked
+(-inf) experts.  Ids bit for bit,
 gates within the gate tolerance of the parity tests.
 """
 import numpy as np
@@ -54,14 +55,18 @@ def test_route_against_oracle(name):
     _route(w, synth.logits(w))
 
 
+@pytest.mark.parametrize("grid", [0.5, 2.0])
 @pytest.mark.parametrize("name", ["E384_odd_T", "E128_odd_T", "E320"])
-def test_route_ties(name):
-    """Logits on a 0.5 grid: most tokens have far more than 32 logits at or
-    above the threshold and take the exact rounds; every third token keeps
-    its fine values and ranks its candidates."""
+def test_route_ties(name, grid):
+    """Logits rounded to a grid, so many tie exactly.  On the 0.5 grid the
+    ties fall among the ranked candidates (at most 32 logits at or above the
+    threshold); on the 2.0 grid every such token of the 320- and 384-expert
+    shapes, and about a third of the 128-expert one, has more than 32 and
+    takes the exact rounds.  Every third token keeps its fine values, so a
+    launch mixes both paths."""
     w = SHAPES[name]
     lg = synth.logits(w)
-    q = (np.round(lg * 2) / 2).astype(np.float32)
+    q = (np.round(lg / grid) * grid).astype(np.float32)
     q[::3] = lg[::3]
     q[::7, 5] = -0.0
     q[::7, 9] = 0.0
